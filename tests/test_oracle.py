@@ -1,0 +1,442 @@
+"""Pins of the CPU oracle against facts fixed outside it (no GPU needed).
+
+Each pin checks the oracle against something it does not compute itself:
+hand-worked examples (tests/golden), an exact rational brute force, exact
+integer arithmetic, a library matmul in float64, closed forms and
+invariants. ``test_planted_mistakes_are_caught`` plants plausible mistakes
+in wrappers around the oracle and checks that at least one pin fails for
+each, so that the pins are known to have teeth.
+"""
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+from gemm_epilogues_tcgen05_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+DT = {"fp16": 0, "bf16": 1}
+
+
+def _bits(values, dtype):
+    t = torch.tensor(values, dtype=torch.float64).to(synth.DTYPES[dtype])
+    return synth.bits_u16(t)
+
+
+def _load(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------- decoders
+
+def test_decode_half_every_pattern(oracle_mod):
+    pats = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    mine = oracle_mod.decode(pats, oracle_mod.F16)
+    ref = pats.view(np.float16).astype(np.float64)
+    assert np.array_equal(np.isnan(mine), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(mine[ok], ref[ok])
+    assert np.array_equal(np.signbit(mine[ok]), np.signbit(ref[ok]))
+
+
+def test_decode_bf16_every_pattern(oracle_mod):
+    pats = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    mine = oracle_mod.decode(pats, oracle_mod.BF16)
+    ref = torch.from_numpy(pats.view(np.int16).copy()).view(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(np.isnan(mine), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(mine[ok], ref[ok])
+
+
+# ----------------------------------------------------------- pin functions
+# Each pin takes (fwd, bwd) callables with the oracle's signatures and
+# returns a list of failure strings (empty = pass).
+
+def pin_golden_forward(fwd, bwd):
+    g = _load("linear_fwd_hand.json")
+    fails = []
+    for dtype in ("fp16", "bf16"):
+        X, W, b = _bits(g["X"], dtype), _bits(g["W"], dtype), _bits(g["bias"], dtype)
+        for ep, ykey in (("BIAS", "Y_BIAS"), ("RELU_BIAS", "Y_RELU"), ("RELU_AUX_BIAS", "Y_RELU")):
+            r = fwd(X, W, b, DT[dtype], ep)
+            if not np.array_equal(r["Z"], np.array(g["Z"], dtype=float)):
+                fails.append(f"golden fwd Z {dtype} {ep}")
+            if not np.array_equal(r["S"], np.array(g["S"], dtype=float)):
+                fails.append(f"golden fwd S {dtype} {ep}")
+            if not np.array_equal(r["Y"], np.array(g[ykey], dtype=float)):
+                fails.append(f"golden fwd Y {dtype} {ep}")
+            if ep == "RELU_AUX_BIAS" and not np.array_equal(r["aux"], np.array(g["aux"], dtype=np.uint32)):
+                fails.append(f"golden fwd aux {dtype}")
+    return fails
+
+
+def pin_golden_mask_layout(fwd, bwd):
+    g = _load("relu_aux_layout_hand.json")
+    N = g["N"]
+    w = np.full((1, N), -1.0)
+    w[0, g["positive"]] = 1.0
+    w[0, g["zero"]] = 0.0
+    fails = []
+    for dtype in ("fp16", "bf16"):
+        r = fwd(_bits([[1.0]], dtype), _bits(w, dtype), _bits(np.zeros(N), dtype), DT[dtype], "RELU_AUX_BIAS")
+        if not np.array_equal(r["aux"], np.array(g["aux"], dtype=np.uint32)):
+            fails.append(f"golden mask layout {dtype}: {r['aux']}")
+    return fails
+
+
+def pin_golden_backward(fwd, bwd):
+    g = _load("drelu_bgrad_hand.json")
+    fails = []
+    for dtype in ("fp16", "bf16"):
+        r = bwd(_bits(g["dY2"], dtype), _bits(g["W2"], dtype), np.array(g["aux"], dtype=np.uint32),
+                DT[dtype], 3)
+        for key in ("G", "S", "dZ", "dbias", "Sb"):
+            if not np.array_equal(r[key], np.array(g[key], dtype=float)):
+                fails.append(f"golden bwd {key} {dtype}: {r[key]}")
+    return fails
+
+
+def _exact_linear(Xf, Wf, bf):
+    """Exact rational Z and S of small float matrices (brute force)."""
+    T, K = len(Xf), len(Xf[0])
+    N = len(Wf[0])
+    Z = [[None] * N for _ in range(T)]
+    S = [[None] * N for _ in range(T)]
+    for t in range(T):
+        for n in range(N):
+            acc = Fraction(0)
+            sc = Fraction(0)
+            for k in range(K):
+                p = Fraction(Xf[t][k]) * Fraction(Wf[k][n])
+                acc += p
+                sc += abs(p)
+            if bf is not None:
+                acc += Fraction(bf[n])
+                sc += abs(Fraction(bf[n]))
+            Z[t][n] = acc
+            S[t][n] = sc
+    return Z, S
+
+
+def pin_bruteforce_rational(fwd, bwd):
+    """Tiny random fp16/bf16 inputs: oracle within K * 2^-52 * S of the exact value."""
+    fails = []
+    shapes = [(1, 1, 1), (3, 5, 2), (5, 33, 7), (2, 17, 16), (4, 9, 33), (7, 40, 3)]
+    for i, (T, N, K) in enumerate(shapes):
+        for dtype in ("fp16", "bf16"):
+            inp = synth.make_shape_inputs(T, N, K, dtype, seed=100 + i)
+            X, W, b = (synth.bits_u16(inp[k]) for k in ("X", "W", "bias"))
+            Xf = inp["X"].double().tolist()
+            Wf = inp["W"].double().tolist()
+            bf = inp["bias"].double().tolist()
+            Zx, Sx = _exact_linear(Xf, Wf, bf)
+            r = fwd(X, W, b, DT[dtype], "RELU_AUX_BIAS")
+            for t in range(T):
+                for n in range(N):
+                    err = abs(Fraction(float(r["Z"][t, n])) - Zx[t][n])
+                    bound = Fraction(K + 1) * Fraction(2) ** -52 * Sx[t][n]
+                    if err > bound:
+                        fails.append(f"bruteforce Z {dtype} {T}x{N}x{K} at {t},{n}")
+                    if abs(Fraction(float(r["S"][t, n])) - Sx[t][n]) > bound:
+                        fails.append(f"bruteforce S {dtype} {T}x{N}x{K} at {t},{n}")
+                    if bool(r["bits"][t, n]) != (Zx[t][n] > 0):
+                        fails.append(f"bruteforce bit {dtype} at {t},{n}")
+            # backward: G = dY2 . W2 exactly, masked by bits from an independent source
+            D2 = max(1, K - 1)
+            inb = synth.make_shape_inputs(T, N, K, dtype, seed=200 + i, D2=D2)
+            dY = inb["dY2"].double().tolist()
+            W2 = inb["W2"].double().tolist()
+            Gx, Gs = _exact_linear(dY, W2, None)
+            rng = np.random.default_rng(7 + i)
+            mask = rng.integers(0, 2, size=(T, N)).astype(bool)
+            words = np.zeros((T, (N + 31) // 32), dtype=np.uint32)
+            for t in range(T):
+                for n in range(N):
+                    if mask[t, n]:
+                        words[t, n // 32] |= np.uint32(1 << (n % 32))
+            rb = bwd(synth.bits_u16(inb["dY2"]), synth.bits_u16(inb["W2"]), words, DT[dtype], N)
+            for n in range(N):
+                col = Fraction(0)
+                for t in range(T):
+                    dz = Gx[t][n] if mask[t, n] else Fraction(0)
+                    col += dz
+                    bound = Fraction(D2 + 1) * Fraction(2) ** -52 * Gs[t][n]
+                    if abs(Fraction(float(rb["dZ"][t, n])) - dz) > bound:
+                        fails.append(f"bruteforce dZ {dtype} at {t},{n}")
+                sb = sum((abs(Gx[t][n]) if mask[t, n] else 0) for t in range(T))
+                bound = Fraction(2) ** -40 * (sb + sum(Gs[t][n] for t in range(T)))
+                if abs(Fraction(float(rb["dbias"][n])) - col) > bound:
+                    fails.append(f"bruteforce dbias {dtype} at {n}")
+    return fails
+
+
+def pin_integer_exact(fwd, bwd):
+    """Integer inputs in [-3, 3]: Z, G, dZ, dbias equal exact int64 arithmetic."""
+    fails = []
+    for i, (T, N, K, D2) in enumerate([(17, 40, 24, 9), (33, 65, 16, 31), (8, 8, 8, 8), (1, 96, 64, 64)]):
+        for dtype in ("fp16", "bf16"):
+            inp = synth.make_shape_inputs(T, N, K, dtype, seed=300 + i, D2=D2, kind="int")
+            Xi, Wi, bi = (inp[k].to(torch.int64).numpy() for k in ("X", "W", "bias"))
+            Zi = Xi @ Wi + bi[None, :]
+            Si = np.abs(Xi[:, :, None] * Wi[None, :, :]).sum(axis=1) + np.abs(bi)[None, :]
+            r = fwd(*(synth.bits_u16(inp[k]) for k in ("X", "W", "bias")), DT[dtype], "RELU_AUX_BIAS")
+            if not np.array_equal(r["Z"], Zi.astype(float)):
+                fails.append(f"int Z {dtype} {T}x{N}x{K}")
+            if not np.array_equal(r["S"], Si.astype(float)):
+                fails.append(f"int S {dtype}")
+            if not np.array_equal(r["Y"], np.maximum(Zi, 0).astype(float)):
+                fails.append(f"int Y {dtype}")
+            expect_words = np.zeros((T, (N + 31) // 32), dtype=np.uint64)
+            for t in range(T):
+                for n in range(N):
+                    if Zi[t, n] > 0:
+                        expect_words[t, n // 32] += 1 << (n % 32)
+            if not np.array_equal(r["aux"], expect_words.astype(np.uint32)):
+                fails.append(f"int aux {dtype}")
+            dYi, W2i = inp["dY2"].to(torch.int64).numpy(), inp["W2"].to(torch.int64).numpy()
+            Gi = dYi @ W2i
+            dZi = np.where(Zi > 0, Gi, 0)
+            rb = bwd(synth.bits_u16(inp["dY2"]), synth.bits_u16(inp["W2"]), r["aux"], DT[dtype], N)
+            if not np.array_equal(rb["G"], Gi.astype(float)):
+                fails.append(f"int G {dtype}")
+            if not np.array_equal(rb["dZ"], dZi.astype(float)):
+                fails.append(f"int dZ {dtype}")
+            if not np.array_equal(rb["dbias"], dZi.sum(axis=0).astype(float)):
+                fails.append(f"int dbias {dtype}")
+    return fails
+
+
+def pin_library_matmul(fwd, bwd):
+    """Zero bias: Z equals torch.matmul in float64; S equals |X| @ |W|."""
+    fails = []
+    for i, (T, N, K) in enumerate([(37, 72, 130), (64, 40, 257)]):
+        for dtype in ("fp16", "bf16"):
+            inp = synth.make_shape_inputs(T, N, K, dtype, seed=400 + i)
+            zero_b = torch.zeros(N, dtype=synth.DTYPES[dtype])
+            r = fwd(synth.bits_u16(inp["X"]), synth.bits_u16(inp["W"]), synth.bits_u16(zero_b), DT[dtype], "BIAS")
+            x, w = inp["X"].double(), inp["W"].double()
+            ref = (x @ w).numpy()
+            sref = (x.abs() @ w.abs()).numpy()
+            if np.max(np.abs(r["Z"] - ref) / sref) > 1e-12:
+                fails.append(f"library Z {dtype}")
+            if np.max(np.abs(r["S"] - sref) / sref) > 1e-12:
+                fails.append(f"library S {dtype}")
+            rr = fwd(synth.bits_u16(inp["X"]), synth.bits_u16(inp["W"]), synth.bits_u16(zero_b), DT[dtype], "RELU_BIAS")
+            if np.max(np.abs(rr["Y"] - np.maximum(ref, 0)) / sref) > 1e-12:
+                fails.append(f"library relu {dtype}")
+    return fails
+
+
+def pin_identity_closed_form(fwd, bwd):
+    """X = I (T = K): Z = W + b exactly, per element."""
+    fails = []
+    T = N = 24
+    for dtype in ("fp16", "bf16"):
+        inp = synth.make_shape_inputs(T, N, T, dtype, seed=500)
+        eye = torch.eye(T, dtype=synth.DTYPES[dtype])
+        r = fwd(synth.bits_u16(eye), synth.bits_u16(inp["W"]), synth.bits_u16(inp["bias"]), DT[dtype], "RELU_BIAS")
+        exact = inp["W"].double().numpy() + inp["bias"].double().numpy()[None, :]
+        if not np.array_equal(r["Z"], exact):
+            fails.append(f"identity Z {dtype}")
+        if not np.array_equal(r["Y"], np.maximum(exact, 0)):
+            fails.append(f"identity Y {dtype}")
+    return fails
+
+
+def pin_backward_library(fwd, bwd):
+    """G equals torch.matmul in float64; dbias equals ones^T . dZ; mask bits select G."""
+    fails = []
+    T, N, D2 = 45, 72, 100
+    for dtype in ("fp16", "bf16"):
+        inp = synth.make_shape_inputs(T, N, 64, dtype, seed=600, D2=D2)
+        fw = fwd(*(synth.bits_u16(inp[k]) for k in ("X", "W", "bias")), DT[dtype], "RELU_AUX_BIAS")
+        rb = bwd(synth.bits_u16(inp["dY2"]), synth.bits_u16(inp["W2"]), fw["aux"], DT[dtype], N)
+        Gref = (inp["dY2"].double() @ inp["W2"].double()).numpy()
+        Sref = (inp["dY2"].double().abs() @ inp["W2"].double().abs()).numpy()
+        if np.max(np.abs(rb["G"] - Gref) / Sref) > 1e-12:
+            fails.append(f"bwd G {dtype}")
+        mask = fw["Z"] > 0
+        if not np.array_equal(rb["dZ"][~mask], np.zeros(int((~mask).sum()))):
+            fails.append(f"bwd dZ off-mask {dtype}")
+        if np.max(np.abs(rb["dZ"][mask] - Gref[mask]) / Sref[mask]) > 1e-12:
+            fails.append(f"bwd dZ on-mask {dtype}")
+        ones = torch.ones(1, T, dtype=torch.float64)
+        dref = (ones @ torch.from_numpy(np.where(mask, Gref, 0.0))).numpy()[0]
+        if np.max(np.abs(rb["dbias"] - dref) / (rb["Sb"] + 1e-300)) > 1e-12:
+            fails.append(f"bwd dbias {dtype}")
+    return fails
+
+
+PINS = [pin_golden_forward, pin_golden_mask_layout, pin_golden_backward, pin_bruteforce_rational,
+        pin_integer_exact, pin_library_matmul, pin_identity_closed_form, pin_backward_library]
+
+
+def _real(oracle_mod):
+    return oracle_mod.linear_fwd, (lambda dY2, W2, aux, dt, N, **kw: oracle_mod.drelu_bgrad(dY2, W2, aux, dt, N, **kw))
+
+
+@pytest.mark.parametrize("pin", PINS, ids=lambda p: p.__name__)
+def test_oracle_pin(oracle_mod, pin):
+    fwd, bwd = _real(oracle_mod)
+    fails = pin(fwd, bwd)
+    assert not fails, fails[:10]
+
+
+# --------------------------------------------------------- planted mistakes
+
+def _mutants(oracle_mod):
+    o = oracle_mod
+
+    def fwd_bias_per_row(X, W, b, dt, ep, **kw):
+        r = o.linear_fwd(X, W, None if False else b, dt, ep, **kw)
+        T = r["Z"].shape[0]
+        bvals = o.decode(b, dt)
+        Z = r["Z"] - bvals[None, :] + bvals[np.arange(T) % len(bvals)][:, None]
+        return _refinish(o, Z, r["S"], ep)
+
+    def fwd_transposed_w(X, W, b, dt, ep, **kw):
+        if W.shape[0] != W.shape[1]:
+            return o.linear_fwd(X, W, b, dt, ep, **kw)
+        return o.linear_fwd(X, np.ascontiguousarray(W.T), b, dt, ep, **kw)
+
+    def fwd_dropped_bias(X, W, b, dt, ep, **kw):
+        return o.linear_fwd(X, W, np.zeros_like(b), dt, ep, **kw)
+
+    def fwd_tie_inclusive(X, W, b, dt, ep, **kw):
+        r = o.linear_fwd(X, W, b, dt, ep, **kw)
+        if "bits" in r:
+            r["bits"] = r["Z"] >= 0
+            r["aux"] = o.relu_aux_words(r["bits"])
+        return r
+
+    def fwd_inverted_polarity(X, W, b, dt, ep, **kw):
+        r = o.linear_fwd(X, W, b, dt, ep, **kw)
+        if "bits" in r:
+            r["bits"] = r["Z"] < 0
+            r["aux"] = o.relu_aux_words(r["bits"])
+        return r
+
+    def fwd_msb_first(X, W, b, dt, ep, **kw):
+        r = o.linear_fwd(X, W, b, dt, ep, **kw)
+        if "aux" in r:
+            rev = np.zeros_like(r["aux"])
+            for j in range(32):
+                rev |= ((r["aux"] >> np.uint32(j)) & np.uint32(1)) << np.uint32(31 - j)
+            r["aux"] = rev
+        return r
+
+    def fwd_sign_flip_product(X, W, b, dt, ep, **kw):
+        r = o.linear_fwd(X, W, b, dt, ep, **kw)
+        bvals = o.decode(b, dt)
+        Z = -(r["Z"] - bvals[None, :]) + bvals[None, :]
+        return _refinish(o, Z, r["S"], ep)
+
+    real_bwd = lambda dY2, W2, aux, dt, N, **kw: o.drelu_bgrad(dY2, W2, aux, dt, N, **kw)
+
+    def bwd_dbias_over_cols(dY2, W2, aux, dt, N, **kw):
+        r = o.drelu_bgrad(dY2, W2, aux, dt, N, **kw)
+        if "dbias" in r:
+            s = r["dZ"].sum(axis=1)
+            r["dbias"] = np.resize(s, r["dbias"].shape)
+        return r
+
+    def bwd_mask_ignored(dY2, W2, aux, dt, N, **kw):
+        r = o.drelu_bgrad(dY2, W2, aux, dt, N, **kw)
+        r["dZ"] = r["G"].copy()
+        r["dbias"] = r["dZ"].sum(axis=0)
+        r["Sb"] = np.abs(r["dZ"]).sum(axis=0)
+        return r
+
+    def bwd_w2_transposed(dY2, W2, aux, dt, N, **kw):
+        if W2.shape[0] != W2.shape[1]:
+            return o.drelu_bgrad(dY2, W2, aux, dt, N, **kw)
+        return o.drelu_bgrad(dY2, np.ascontiguousarray(W2.T), aux, dt, N, **kw)
+
+    def bwd_dropped_last_term(dY2, W2, aux, dt, N, **kw):
+        W2z = W2.copy()
+        W2z[-1, :] = 0
+        return o.drelu_bgrad(dY2, W2z, aux, dt, N, **kw)
+
+    fwd = o.linear_fwd
+    return {
+        "bias per row": (fwd_bias_per_row, real_bwd),
+        "W transposed": (fwd_transposed_w, real_bwd),
+        "bias dropped": (fwd_dropped_bias, real_bwd),
+        "tie Z==0 sets bit": (fwd_tie_inclusive, real_bwd),
+        "mask polarity inverted": (fwd_inverted_polarity, real_bwd),
+        "mask MSB first": (fwd_msb_first, real_bwd),
+        "product sign flipped": (fwd_sign_flip_product, real_bwd),
+        "dbias summed over columns": (fwd, bwd_dbias_over_cols),
+        "mask ignored in backward": (fwd, bwd_mask_ignored),
+        "W2 transposed": (fwd, bwd_w2_transposed),
+        "last contraction term dropped": (fwd, bwd_dropped_last_term),
+    }
+
+
+def _refinish(o, Z, S, ep):
+    out = {"Z": Z, "S": S, "Y": Z.copy() if ep == "BIAS" else np.maximum(Z, 0.0)}
+    if ep == "RELU_AUX_BIAS":
+        out["bits"] = Z > 0
+        out["aux"] = o.relu_aux_words(out["bits"])
+    return out
+
+
+def test_planted_mistakes_are_caught(oracle_mod):
+    caught = {}
+    for name, (fwd, bwd) in _mutants(oracle_mod).items():
+        n_fail = 0
+        for pin in PINS:
+            try:
+                n_fail += len(pin(fwd, bwd))
+            except Exception:  # a crash also counts as caught
+                n_fail += 1
+        caught[name] = n_fail
+    missed = [k for k, v in caught.items() if v == 0]
+    assert not missed, f"pins did not catch: {missed}"
+
+
+# ------------------------------------------------------------ misc behaviour
+
+def test_row_col_subsets_match_full(oracle_mod):
+    inp = synth.make_shape_inputs(40, 70, 33, "bf16", seed=700)
+    X, W, b = (synth.bits_u16(inp[k]) for k in ("X", "W", "bias"))
+    full = oracle_mod.linear_fwd(X, W, b, 1, "RELU_AUX_BIAS")
+    rows, cols = [0, 7, 39], [1, 32, 69]
+    part = oracle_mod.linear_fwd(X, W, b, 1, "RELU_AUX_BIAS", rows=rows, cols=cols)
+    assert np.array_equal(part["Z"], full["Z"][np.ix_(rows, cols)])
+    assert np.array_equal(part["S"], full["S"][np.ix_(rows, cols)])
+    single = oracle_mod.linear_fwd(X, W, b, 1, "RELU_AUX_BIAS", threads=1)
+    assert np.array_equal(single["Z"], full["Z"])
+
+
+def test_bad_arguments_rejected(oracle_mod):
+    X = np.zeros((2, 3), np.uint16)
+    W = np.zeros((3, 4), np.uint16)
+    with pytest.raises(ValueError):
+        oracle_mod.matmul_bias(X, np.zeros((2, 4), np.uint16), None, 0)
+    with pytest.raises(ValueError):
+        oracle_mod.matmul_bias(X, W, None, 0, rows=[5])
+    with pytest.raises(ValueError):
+        oracle_mod.matmul_bias(X, W, None, 0, cols=[-1])
+    with pytest.raises(ValueError):
+        oracle_mod.matmul_bias(X, W, None, 7)
+    C, S = oracle_mod.matmul_bias(X, W, None, 0, rows=[])
+    assert C.shape == (0, 4)
+
+
+def test_mask_pack_roundtrip(oracle_mod):
+    rng = np.random.default_rng(1)
+    for N in (1, 31, 32, 33, 64, 100):
+        bits = rng.integers(0, 2, size=(5, N)).astype(bool)
+        words = oracle_mod.relu_aux_words(bits)
+        assert words.shape == (5, math.ceil(N / 32))
+        assert np.array_equal(oracle_mod.relu_aux_bits(words, N), bits)
+        # pad bits past N are zero
+        tail = N % 32
+        if tail:
+            assert np.all(words[:, -1] >> np.uint32(tail) == 0)
