@@ -1,0 +1,209 @@
+"""ctypes binding of ``libgemm_epi.so`` (the C ABI in include/gemm_epi.h).
+
+Argument marshalling only: tensors are checked for device, dtype, shape and
+contiguity, then their ``data_ptr()`` and the current CUDA stream are passed
+to the C function of the same name. All arithmetic happens in the library's
+kernels; if the library is missing, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+F16, BF16 = 0, 1
+BIAS, RELU_BIAS, RELU_AUX_BIAS, DRELU_BGRAD = 0, 1, 2, 3
+EPILOGS = {"BIAS": BIAS, "RELU_BIAS": RELU_BIAS, "RELU_AUX_BIAS": RELU_AUX_BIAS, "DRELU_BGRAD": DRELU_BGRAD}
+DTYPES = {torch.float16: F16, torch.bfloat16: BF16}
+
+OK = 0
+ERR_INVALID_ARG = -1
+ERR_MISALIGNED = -2
+ERR_EPILOG_MISMATCH = -3
+ERR_CUDA = -4
+ERR_TIMEOUT = -5
+ERR_UNSUPPORTED = -6
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgemm_epi.so")
+
+EXPORTED = ["gemm_epi_plan", "gemm_epi_execute", "drelu_bgrad_execute", "gemm_epi_free", "gemm_epi_last_error",
+            "gemm_epi_query", "gemm_epi_status", "gemm_epi_unfused_execute", "drelu_bgrad_unfused_execute"]
+
+
+class GemmEpiError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"gemm_epi error {code}: {msg}")
+        self.code = code
+
+
+class Info(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int64), ("N", ctypes.c_int64), ("K", ctypes.c_int64),
+                ("dtype", ctypes.c_int), ("epilog", ctypes.c_int), ("kernel", ctypes.c_int),
+                ("tile_m", ctypes.c_int), ("tile_n", ctypes.c_int), ("tile_k", ctypes.c_int),
+                ("stages", ctypes.c_int), ("split_k", ctypes.c_int), ("grid", ctypes.c_int),
+                ("launches", ctypes.c_int), ("num_sms", ctypes.c_int), ("workspace_bytes", ctypes.c_size_t)]
+
+    def as_dict(self) -> dict:
+        return {name: getattr(self, name) for name, _ in self._fields_}
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load the library (once). Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with python -m gemm_epilogues_tcgen05_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i64, ci = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+        L.gemm_epi_plan.restype = vp
+        L.gemm_epi_plan.argtypes = [i64, i64, i64, ci, ci]
+        L.gemm_epi_execute.restype = ci
+        L.gemm_epi_execute.argtypes = [vp] * 7
+        L.drelu_bgrad_execute.restype = ci
+        L.drelu_bgrad_execute.argtypes = [vp] * 7
+        L.gemm_epi_free.restype = None
+        L.gemm_epi_free.argtypes = [vp]
+        L.gemm_epi_last_error.restype = ctypes.c_char_p
+        L.gemm_epi_last_error.argtypes = []
+        L.gemm_epi_query.restype = ci
+        L.gemm_epi_query.argtypes = [vp, ctypes.POINTER(Info)]
+        L.gemm_epi_status.restype = ci
+        L.gemm_epi_status.argtypes = [vp]
+        L.gemm_epi_unfused_execute.restype = ci
+        L.gemm_epi_unfused_execute.argtypes = [vp] * 9
+        L.drelu_bgrad_unfused_execute.restype = ci
+        L.drelu_bgrad_unfused_execute.argtypes = [vp] * 8
+        _lib = L
+    return _lib
+
+
+def gemm_epi_last_error() -> str:
+    return lib().gemm_epi_last_error().decode()
+
+
+def _check(rc: int):
+    if rc != OK:
+        raise GemmEpiError(rc, gemm_epi_last_error())
+
+
+def _stream_ptr(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t, shape, dtype, name) -> int | None:
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be on a CUDA device")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def gemm_epi_plan(T: int, N: int, K: int, dtype, epilog) -> int:
+    """Raw handle (int) from the C gemm_epi_plan; raises on error."""
+    if isinstance(dtype, torch.dtype):
+        dtype = DTYPES[dtype]
+    if isinstance(epilog, str):
+        epilog = EPILOGS[epilog]
+    h = lib().gemm_epi_plan(T, N, K, dtype, epilog)
+    if not h:
+        raise GemmEpiError(ERR_INVALID_ARG, gemm_epi_last_error())
+    return h
+
+
+def gemm_epi_free(handle) -> None:
+    lib().gemm_epi_free(handle)
+
+
+class Plan:
+    """A plan for one (T, N, K, dtype, epilog); execute any number of times."""
+
+    def __init__(self, T: int, N: int, K: int, dtype: torch.dtype, epilog: str | int):
+        self.T, self.N, self.K = T, N, K
+        self.dtype = dtype
+        self.epilog = EPILOGS[epilog] if isinstance(epilog, str) else epilog
+        self.aux_words = (N + 31) // 32
+        self.handle = gemm_epi_plan(T, N, K, dtype, self.epilog)
+
+    # life cycle ----------------------------------------------------------
+    def free(self):
+        if self.handle:
+            gemm_epi_free(self.handle)
+            self.handle = None
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.free()
+
+    def __del__(self):
+        try:
+            self.free()
+        except Exception:
+            pass
+
+    def info(self) -> dict:
+        inf = Info()
+        _check(lib().gemm_epi_query(self.handle, ctypes.byref(inf)))
+        return inf.as_dict()
+
+    def status(self) -> int:
+        """OK, or ERR_TIMEOUT if a kernel of this plan gave up a wait (after a sync)."""
+        return lib().gemm_epi_status(self.handle)
+
+    # calls -------------------------------------------------------------
+    def gemm_epi_execute(self, X, W, bias, Y, aux=None, stream=None):
+        T, N, K, dt = self.T, self.N, self.K, self.dtype
+        args = (_ptr(X, (T, K), dt, "X"), _ptr(W, (K, N), dt, "W"), _ptr(bias, (N,), dt, "bias"),
+                _ptr(Y, (T, N), dt, "Y"), _ptr(aux, (T, self.aux_words), torch.int32, "aux"))
+        _check(lib().gemm_epi_execute(self.handle, *args, _stream_ptr(stream)))
+
+    def drelu_bgrad_execute(self, dY2, W2, aux, dZ, dbias, stream=None):
+        T, N, K, dt = self.T, self.N, self.K, self.dtype
+        args = (_ptr(dY2, (T, K), dt, "dY2"), _ptr(W2, (K, N), dt, "W2"),
+                _ptr(aux, (T, self.aux_words), torch.int32, "aux"), _ptr(dZ, (T, N), dt, "dZ"),
+                _ptr(dbias, (N,), torch.float32, "dbias"))
+        _check(lib().drelu_bgrad_execute(self.handle, *args, _stream_ptr(stream)))
+
+    def gemm_epi_unfused_execute(self, X, W, bias, T1, T2, Y, aux=None, stream=None):
+        T, N, K, dt = self.T, self.N, self.K, self.dtype
+        args = (_ptr(X, (T, K), dt, "X"), _ptr(W, (K, N), dt, "W"), _ptr(bias, (N,), dt, "bias"),
+                _ptr(T1, (T, N), dt, "T1"), _ptr(T2, (T, N), dt, "T2"), _ptr(Y, (T, N), dt, "Y"),
+                _ptr(aux, (T, self.aux_words), torch.int32, "aux"))
+        _check(lib().gemm_epi_unfused_execute(self.handle, *args, _stream_ptr(stream)))
+
+    def drelu_bgrad_unfused_execute(self, dY2, W2, aux, G, dZ, dbias, stream=None):
+        T, N, K, dt = self.T, self.N, self.K, self.dtype
+        args = (_ptr(dY2, (T, K), dt, "dY2"), _ptr(W2, (K, N), dt, "W2"),
+                _ptr(aux, (T, self.aux_words), torch.int32, "aux"), _ptr(G, (T, N), dt, "G"),
+                _ptr(dZ, (T, N), dt, "dZ"), _ptr(dbias, (N,), torch.float32, "dbias"))
+        _check(lib().drelu_bgrad_unfused_execute(self.handle, *args, _stream_ptr(stream)))
+
+    # conveniences that allocate their outputs (allocation happens in torch,
+    # outside the library; the library call itself allocates nothing)
+    def forward(self, X, W, bias, stream=None):
+        Y = torch.empty((self.T, self.N), dtype=self.dtype, device=X.device)
+        aux = (torch.empty((self.T, self.aux_words), dtype=torch.int32, device=X.device)
+               if self.epilog == RELU_AUX_BIAS else None)
+        self.gemm_epi_execute(X, W, bias, Y, aux, stream)
+        return Y, aux
+
+    def backward(self, dY2, W2, aux, stream=None):
+        dZ = torch.empty((self.T, self.N), dtype=self.dtype, device=dY2.device)
+        dbias = torch.empty((self.N,), dtype=torch.float32, device=dY2.device)
+        self.drelu_bgrad_execute(dY2, W2, aux, dZ, dbias, stream)
+        return dZ, dbias

@@ -1,0 +1,482 @@
+// gemm_epi.cu -- C ABI of the fused linear-layer GEMM + epilogue library
+// (declared in include/gemm_epi.h): plan validation and kernel choice,
+// TMA descriptor encoding, launches, the watchdog status word and errors.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <unordered_set>
+
+#include "../../include/gemm_epi.h"
+#include "aux_kernels.cuh"
+#include "tile_kernel.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(GEMM_EPI_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorString(e), cudaGetErrorName(e));
+}
+
+// ---------------------------------------------------------------- registry
+std::mutex g_mu;
+std::unordered_set<gemm_epi_plan_s*>& live_plans() {
+  static std::unordered_set<gemm_epi_plan_s*> s;
+  return s;
+}
+
+// ----------------------------------------------------- driver entry points
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D row-major tensor of 16-bit elements: `inner` contiguous columns,
+// `outer` rows; box of box_inner x box_outer with 128-byte swizzle.
+int encode_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+              uint32_t box_outer, const char* name) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(GEMM_EPI_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {inner * 2};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(GEMM_EPI_ERR_CUDA, "tensor map encode for %s failed (CUresult %d)", name, (int)r);
+  return GEMM_EPI_OK;
+}
+
+using TileKernelFn = void (*)(CUtensorMap, CUtensorMap, ge::TileParams);
+
+template <int BN, int ST, bool BF>
+TileKernelFn pick_epi(int epi) {
+  switch (epi) {
+    case ge::EPI_BIAS: return ge::tile_kernel<BN, ST, ge::EPI_BIAS, BF>;
+    case ge::EPI_RELU_BIAS: return ge::tile_kernel<BN, ST, ge::EPI_RELU_BIAS, BF>;
+    case ge::EPI_RELU_AUX_BIAS: return ge::tile_kernel<BN, ST, ge::EPI_RELU_AUX_BIAS, BF>;
+    case ge::EPI_DRELU_BGRAD: return ge::tile_kernel<BN, ST, ge::EPI_DRELU_BGRAD, BF>;
+    default: return ge::tile_kernel<BN, ST, ge::EPI_STORE, BF>;
+  }
+}
+
+struct TileCfg {
+  int BN = 256, stages = 4;
+  TileKernelFn fn = nullptr;
+  uint32_t smem = 0;
+};
+
+TileCfg tile_cfg(int BN, int epi, bool bf16) {
+  TileCfg c;
+  c.BN = BN;
+  if (BN == 256) {
+    c.stages = 4;
+    c.smem = ge::TileSmem<256, 4>::BYTES;
+    c.fn = bf16 ? pick_epi<256, 4, true>(epi) : pick_epi<256, 4, false>(epi);
+  } else if (BN == 128) {
+    c.stages = 6;
+    c.smem = ge::TileSmem<128, 6>::BYTES;
+    c.fn = bf16 ? pick_epi<128, 6, true>(epi) : pick_epi<128, 6, false>(epi);
+  } else {
+    c.BN = 64;
+    c.stages = 8;
+    c.smem = ge::TileSmem<64, 8>::BYTES;
+    c.fn = bf16 ? pick_epi<64, 8, true>(epi) : pick_epi<64, 8, false>(epi);
+  }
+  return c;
+}
+
+int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
+
+}  // namespace
+
+struct gemm_epi_plan_s {
+  int64_t T, N, K;
+  int dtype, epilog;
+  int device, num_sms;
+  int m_tiles, n_tiles, k_blocks, num_tiles, aux_words, grid;
+  TileCfg cfg;       // fused kernel
+  TileCfg cfg_store; // unfused GEMM (plain store)
+  float* partials = nullptr;  // DRELU_BGRAD: m_tiles x N
+  size_t partial_bytes = 0;
+  int* status_host = nullptr;
+  int* status_dev = nullptr;
+  uint64_t timeout_ns = 0;
+  // tensor-map cache
+  const void* a_ptr = nullptr;
+  const void* b_ptr = nullptr;
+  CUtensorMap tmA, tmB;
+};
+
+namespace {
+
+gemm_epi_plan_s* lookup(gemm_epi_plan_t p) {
+  std::lock_guard<std::mutex> g(g_mu);
+  return live_plans().count(p) ? p : nullptr;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int take_status(gemm_epi_plan_s* p) {
+  volatile int* s = p->status_host;
+  const int v = *s;
+  if (v != 0) {
+    *s = 0;
+    return fail(GEMM_EPI_ERR_TIMEOUT, "a kernel of this plan gave up waiting (watchdog code 0x%x)", v);
+  }
+  return GEMM_EPI_OK;
+}
+
+int prepare_maps(gemm_epi_plan_s* p, const void* A, const void* B) {
+  if (A != p->a_ptr) {
+    int rc = encode_2d(&p->tmA, A, (uint64_t)p->K, (uint64_t)p->T, ge::kBK, ge::kBM, "the row operand");
+    if (rc) return rc;
+    p->a_ptr = A;
+  }
+  if (B != p->b_ptr) {
+    int rc = encode_2d(&p->tmB, B, (uint64_t)p->N, (uint64_t)p->K, 64, ge::kBK, "the weight operand");
+    if (rc) return rc;
+    p->b_ptr = B;
+  }
+  return GEMM_EPI_OK;
+}
+
+ge::TileParams base_params(const gemm_epi_plan_s* p) {
+  ge::TileParams k{};
+  k.T = (int32_t)p->T;
+  k.N = (int32_t)p->N;
+  k.K = (int32_t)p->K;
+  k.m_tiles = p->m_tiles;
+  k.n_tiles = p->n_tiles;
+  k.k_blocks = p->k_blocks;
+  k.num_tiles = p->num_tiles;
+  k.aux_words = p->aux_words;
+  k.status = p->status_dev;
+  k.timeout_ns = p->timeout_ns;
+  return k;
+}
+
+int launch_tile(const gemm_epi_plan_s* p, const TileCfg& c, const ge::TileParams& k, cudaStream_t s) {
+  c.fn<<<p->grid, ge::kThreads, c.smem, s>>>(p->tmA, p->tmB, k);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "tile kernel launch");
+  return GEMM_EPI_OK;
+}
+
+int choose_bn(int64_t T, int64_t N, int num_sms) {
+  if (const char* f = getenv("GEMM_EPI_FORCE_BN")) {
+    int v = atoi(f);
+    if (v == 64 || v == 128 || v == 256) return v;
+  }
+  const int64_t m_tiles = (T + ge::kBM - 1) / ge::kBM;
+  // widest tile that still gives every SM at least one tile, else the
+  // narrowest: wide tiles need the least shared-memory bandwidth per MMA
+  for (int bn : {256, 128}) {
+    if (m_tiles * ((N + bn - 1) / bn) >= num_sms) return bn;
+  }
+  return 64;
+}
+
+}  // namespace
+
+extern "C" {
+
+gemm_epi_plan_t gemm_epi_plan(int64_t T, int64_t N, int64_t K, gemm_epi_dtype dtype, gemm_epi_epilog epilog) {
+  if (T < 1 || N < 8 || K < 8 || (N % 8) != 0 || (K % 8) != 0) {
+    fail(GEMM_EPI_ERR_INVALID_ARG, "bad shape T=%lld N=%lld K=%lld (need T>=1, N,K>=8 and multiples of 8)",
+         (long long)T, (long long)N, (long long)K);
+    return nullptr;
+  }
+  if (T > (int64_t)1 << 30 || N > (int64_t)1 << 24 || K > (int64_t)1 << 24 || T * N > ((int64_t)1 << 40)) {
+    fail(GEMM_EPI_ERR_INVALID_ARG, "shape too large for 32-bit tile coordinates");
+    return nullptr;
+  }
+  if (dtype != GEMM_EPI_F16 && dtype != GEMM_EPI_BF16) {
+    fail(GEMM_EPI_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    return nullptr;
+  }
+  if (epilog < GEMM_EPI_BIAS || epilog > GEMM_EPI_DRELU_BGRAD) {
+    fail(GEMM_EPI_ERR_INVALID_ARG, "unknown epilog %d", (int)epilog);
+    return nullptr;
+  }
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    cuda_fail(e, "cudaGetDevice");
+    return nullptr;
+  }
+  int major = 0, minor = 0, sms = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (major != 10 || minor != 0) {
+    fail(GEMM_EPI_ERR_UNSUPPORTED, "device %d has compute capability %d.%d; this library needs 10.0 (sm_100a)", dev,
+         major, minor);
+    return nullptr;
+  }
+
+  auto* p = new gemm_epi_plan_s();
+  p->T = T;
+  p->N = N;
+  p->K = K;
+  p->dtype = dtype;
+  p->epilog = epilog;
+  p->device = dev;
+  p->num_sms = sms;
+  const bool bf16 = dtype == GEMM_EPI_BF16;
+  const int bn = choose_bn(T, N, sms);
+  p->cfg = tile_cfg(bn, (int)epilog, bf16);
+  p->cfg_store = tile_cfg(bn, ge::EPI_STORE, bf16);
+  p->m_tiles = ceil_div(T, ge::kBM);
+  p->n_tiles = ceil_div(N, bn);
+  p->k_blocks = ceil_div(K, ge::kBK);
+  p->num_tiles = p->m_tiles * p->n_tiles;
+  p->aux_words = ceil_div(N, 32);
+  p->grid = p->num_tiles < sms ? p->num_tiles : sms;
+  p->timeout_ns = 2000000000ull;  // 2 s per wait
+  if (const char* t = getenv("GEMM_EPI_WAIT_TIMEOUT_MS")) {
+    long long ms = atoll(t);
+    if (ms > 0) p->timeout_ns = (uint64_t)ms * 1000000ull;
+  }
+
+  auto cleanup = [&](int rc) {
+    if (p->partials) cudaFree(p->partials);
+    if (p->status_host) cudaFreeHost(p->status_host);
+    delete p;
+    (void)rc;
+    return nullptr;
+  };
+
+  for (const TileCfg* c : {&p->cfg, &p->cfg_store}) {
+    e = cudaFuncSetAttribute(c->fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)c->smem);
+    if (e != cudaSuccess) return cleanup(cuda_fail(e, "cudaFuncSetAttribute(max dynamic shared memory)"));
+  }
+  e = cudaHostAlloc((void**)&p->status_host, sizeof(int), cudaHostAllocMapped);
+  if (e != cudaSuccess) return cleanup(cuda_fail(e, "cudaHostAlloc(status word)"));
+  *p->status_host = 0;
+  e = cudaHostGetDevicePointer((void**)&p->status_dev, p->status_host, 0);
+  if (e != cudaSuccess) return cleanup(cuda_fail(e, "cudaHostGetDevicePointer(status word)"));
+  // the column partials are needed by the fused and the unfused backward
+  p->partial_bytes = (size_t)p->m_tiles * (size_t)N * sizeof(float);
+  if (epilog == GEMM_EPI_DRELU_BGRAD) {
+    if (getenv("GEMM_EPI_INJECT_PLAN_ALLOC_FAILURE"))
+      return cleanup(fail(GEMM_EPI_ERR_CUDA, "injected workspace allocation failure"));
+    e = cudaMalloc((void**)&p->partials, p->partial_bytes);
+    if (e != cudaSuccess) return cleanup(cuda_fail(e, "cudaMalloc(workspace)"));
+  }
+  {
+    std::lock_guard<std::mutex> g(g_mu);
+    live_plans().insert(p);
+  }
+  g_last_error.clear();
+  return p;
+}
+
+void gemm_epi_free(gemm_epi_plan_t plan) {
+  if (!plan) return;
+  {
+    std::lock_guard<std::mutex> g(g_mu);
+    if (!live_plans().erase(plan)) {
+      g_last_error = "gemm_epi_free: not a live plan (ignored)";
+      return;
+    }
+  }
+  if (plan->partials) cudaFree(plan->partials);
+  if (plan->status_host) cudaFreeHost(plan->status_host);
+  delete plan;
+}
+
+const char* gemm_epi_last_error(void) { return g_last_error.c_str(); }
+
+int gemm_epi_query(gemm_epi_plan_t plan, gemm_epi_info* info) {
+  gemm_epi_plan_s* p = lookup(plan);
+  if (!p || !info) return fail(GEMM_EPI_ERR_INVALID_ARG, "gemm_epi_query: unknown plan or NULL info");
+  memset(info, 0, sizeof(*info));
+  info->T = p->T;
+  info->N = p->N;
+  info->K = p->K;
+  info->dtype = p->dtype;
+  info->epilog = p->epilog;
+  info->kernel = 0;
+  info->tile_m = ge::kBM;
+  info->tile_n = p->cfg.BN;
+  info->tile_k = ge::kBK;
+  info->stages = p->cfg.stages;
+  info->split_k = 1;
+  info->grid = p->grid;
+  info->launches = p->epilog == GEMM_EPI_DRELU_BGRAD ? 2 : 1;
+  info->num_sms = p->num_sms;
+  info->workspace_bytes = p->epilog == GEMM_EPI_DRELU_BGRAD ? p->partial_bytes : 0;
+  return GEMM_EPI_OK;
+}
+
+int gemm_epi_status(gemm_epi_plan_t plan) {
+  gemm_epi_plan_s* p = lookup(plan);
+  if (!p) return fail(GEMM_EPI_ERR_INVALID_ARG, "gemm_epi_status: unknown plan");
+  return take_status(p);
+}
+
+int gemm_epi_execute(gemm_epi_plan_t plan, const void* X, const void* W, const void* bias, void* Y, uint32_t* aux,
+                     cudaStream_t stream) {
+  gemm_epi_plan_s* p = lookup(plan);
+  if (!p) return fail(GEMM_EPI_ERR_INVALID_ARG, "gemm_epi_execute: unknown plan");
+  if (p->epilog == GEMM_EPI_DRELU_BGRAD)
+    return fail(GEMM_EPI_ERR_EPILOG_MISMATCH, "gemm_epi_execute called on a DRELU_BGRAD plan");
+  if (!X || !W || !bias || !Y) return fail(GEMM_EPI_ERR_INVALID_ARG, "gemm_epi_execute: NULL X, W, bias or Y");
+  if (p->epilog == GEMM_EPI_RELU_AUX_BIAS && !aux)
+    return fail(GEMM_EPI_ERR_EPILOG_MISMATCH, "RELU_AUX_BIAS needs an aux buffer");
+  if (!aligned(X, 16) || !aligned(W, 16) || !aligned(Y, 16) || !aligned(bias, 2) ||
+      (p->epilog == GEMM_EPI_RELU_AUX_BIAS && !aligned(aux, 4)))
+    return fail(GEMM_EPI_ERR_MISALIGNED, "gemm_epi_execute: X, W, Y need 16-byte, bias 2-byte, aux 4-byte alignment");
+  int rc = take_status(p);
+  if (rc) return rc;
+  rc = prepare_maps(p, X, W);
+  if (rc) return rc;
+  ge::TileParams k = base_params(p);
+  k.bias = bias;
+  k.out = Y;
+  k.aux_out = aux;
+  return launch_tile(p, p->cfg, k, stream);
+}
+
+int drelu_bgrad_execute(gemm_epi_plan_t plan, const void* dY2, const void* W2, const uint32_t* aux, void* dZ,
+                        float* dbias, cudaStream_t stream) {
+  gemm_epi_plan_s* p = lookup(plan);
+  if (!p) return fail(GEMM_EPI_ERR_INVALID_ARG, "drelu_bgrad_execute: unknown plan");
+  if (p->epilog != GEMM_EPI_DRELU_BGRAD)
+    return fail(GEMM_EPI_ERR_EPILOG_MISMATCH, "drelu_bgrad_execute called on a forward plan");
+  if (!dY2 || !W2 || !aux || !dZ || !dbias)
+    return fail(GEMM_EPI_ERR_INVALID_ARG, "drelu_bgrad_execute: NULL dY2, W2, aux, dZ or dbias");
+  if (!aligned(dY2, 16) || !aligned(W2, 16) || !aligned(dZ, 16) || !aligned(aux, 4) || !aligned(dbias, 4))
+    return fail(GEMM_EPI_ERR_MISALIGNED,
+                "drelu_bgrad_execute: dY2, W2, dZ need 16-byte, aux and dbias 4-byte alignment");
+  int rc = take_status(p);
+  if (rc) return rc;
+  rc = prepare_maps(p, dY2, W2);
+  if (rc) return rc;
+  ge::TileParams k = base_params(p);
+  k.out = dZ;
+  k.aux_in = aux;
+  k.partials = p->partials;
+  rc = launch_tile(p, p->cfg, k, stream);
+  if (rc) return rc;
+  ge::dbias_finish_kernel<<<ceil_div(p->N, 256), 256, 0, stream>>>(p->partials, p->m_tiles, (int)p->N, dbias);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "dbias finish launch");
+  return GEMM_EPI_OK;
+}
+
+int gemm_epi_unfused_execute(gemm_epi_plan_t plan, const void* X, const void* W, const void* bias, void* T1, void* T2,
+                             void* Y, uint32_t* aux, cudaStream_t stream) {
+  gemm_epi_plan_s* p = lookup(plan);
+  if (!p) return fail(GEMM_EPI_ERR_INVALID_ARG, "gemm_epi_unfused_execute: unknown plan");
+  if (p->epilog == GEMM_EPI_DRELU_BGRAD)
+    return fail(GEMM_EPI_ERR_EPILOG_MISMATCH, "gemm_epi_unfused_execute called on a DRELU_BGRAD plan");
+  if (!X || !W || !bias || !T1 || !T2 || !Y) return fail(GEMM_EPI_ERR_INVALID_ARG, "unfused: NULL pointer");
+  if (p->epilog == GEMM_EPI_RELU_AUX_BIAS && !aux)
+    return fail(GEMM_EPI_ERR_EPILOG_MISMATCH, "RELU_AUX_BIAS needs an aux buffer");
+  if (!aligned(X, 16) || !aligned(W, 16) || !aligned(T1, 16) || !aligned(T2, 16) || !aligned(Y, 16) ||
+      !aligned(bias, 2) || (aux && !aligned(aux, 4)))
+    return fail(GEMM_EPI_ERR_MISALIGNED, "unfused: misaligned pointer");
+  int rc = take_status(p);
+  if (rc) return rc;
+  rc = prepare_maps(p, X, W);
+  if (rc) return rc;
+  ge::TileParams k = base_params(p);
+  k.out = T1;
+  rc = launch_tile(p, p->cfg_store, k, stream);
+  if (rc) return rc;
+  const bool bf16 = p->dtype == GEMM_EPI_BF16;
+  const int blocks = p->num_sms * 8;
+  if (bf16)
+    ge::bias_add_kernel<true><<<blocks, 256, 0, stream>>>((const uint4*)T1, bias, (uint4*)T2, p->T, (int)p->N);
+  else
+    ge::bias_add_kernel<false><<<blocks, 256, 0, stream>>>((const uint4*)T1, bias, (uint4*)T2, p->T, (int)p->N);
+  if (p->epilog != GEMM_EPI_BIAS) {
+    const bool want_aux = p->epilog == GEMM_EPI_RELU_AUX_BIAS;
+    auto* in = (const uint16_t*)T2;
+    auto* out = (uint16_t*)Y;
+    if (bf16) {
+      if (want_aux)
+        ge::relu_mask_kernel<true, true><<<blocks, 256, 0, stream>>>(in, out, aux, p->T, (int)p->N, p->aux_words);
+      else
+        ge::relu_mask_kernel<true, false><<<blocks, 256, 0, stream>>>(in, out, aux, p->T, (int)p->N, p->aux_words);
+    } else {
+      if (want_aux)
+        ge::relu_mask_kernel<false, true><<<blocks, 256, 0, stream>>>(in, out, aux, p->T, (int)p->N, p->aux_words);
+      else
+        ge::relu_mask_kernel<false, false><<<blocks, 256, 0, stream>>>(in, out, aux, p->T, (int)p->N, p->aux_words);
+    }
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "unfused elementwise launch");
+  return GEMM_EPI_OK;
+}
+
+int drelu_bgrad_unfused_execute(gemm_epi_plan_t plan, const void* dY2, const void* W2, const uint32_t* aux, void* G,
+                                void* dZ, float* dbias, cudaStream_t stream) {
+  gemm_epi_plan_s* p = lookup(plan);
+  if (!p) return fail(GEMM_EPI_ERR_INVALID_ARG, "drelu_bgrad_unfused_execute: unknown plan");
+  if (p->epilog != GEMM_EPI_DRELU_BGRAD)
+    return fail(GEMM_EPI_ERR_EPILOG_MISMATCH, "drelu_bgrad_unfused_execute called on a forward plan");
+  if (!dY2 || !W2 || !aux || !G || !dZ || !dbias) return fail(GEMM_EPI_ERR_INVALID_ARG, "unfused: NULL pointer");
+  if (!aligned(dY2, 16) || !aligned(W2, 16) || !aligned(G, 16) || !aligned(dZ, 16) || !aligned(aux, 4) ||
+      !aligned(dbias, 4))
+    return fail(GEMM_EPI_ERR_MISALIGNED, "unfused: misaligned pointer");
+  int rc = take_status(p);
+  if (rc) return rc;
+  rc = prepare_maps(p, dY2, W2);
+  if (rc) return rc;
+  ge::TileParams k = base_params(p);
+  k.out = G;
+  rc = launch_tile(p, p->cfg_store, k, stream);
+  if (rc) return rc;
+  const int blocks = p->num_sms * 8;
+  const bool bf16 = p->dtype == GEMM_EPI_BF16;
+  if (bf16)
+    ge::mask_apply_kernel<true><<<blocks, 256, 0, stream>>>((const uint16_t*)G, aux, (uint16_t*)dZ, p->T, (int)p->N,
+                                                             p->aux_words);
+  else
+    ge::mask_apply_kernel<false><<<blocks, 256, 0, stream>>>((const uint16_t*)G, aux, (uint16_t*)dZ, p->T, (int)p->N,
+                                                              p->aux_words);
+  dim3 cgrid(ceil_div(p->N, 256), p->m_tiles);
+  if (bf16)
+    ge::colsum_partial_kernel<true><<<cgrid, 256, 0, stream>>>((const uint16_t*)dZ, p->T, (int)p->N, p->partials);
+  else
+    ge::colsum_partial_kernel<false><<<cgrid, 256, 0, stream>>>((const uint16_t*)dZ, p->T, (int)p->N, p->partials);
+  ge::dbias_finish_kernel<<<ceil_div(p->N, 256), 256, 0, stream>>>(p->partials, p->m_tiles, (int)p->N, dbias);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "unfused backward launch");
+  return GEMM_EPI_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,366 @@
+// tile_kernel.cuh -- persistent tcgen05 GEMM with the fused linear-layer
+// epilogues (BIAS, RELU_BIAS, RELU_AUX_BIAS, DRELU_BGRAD, and a plain store
+// for the unfused measurement path).
+//
+// One CTA per SM walks a static tile schedule. Warp roles:
+//   warp 0      TMA producer: X tile (128 x 64, K-major) and W tile
+//               (64 x BN, N-major) per stage into a STAGES-deep ring of
+//               128-byte-swizzled shared memory, guarded by full/empty mbarriers
+//   warp 1      allocates tensor memory; one lane issues tcgen05.mma
+//               (M=128, N=BN, K=16) into one of two fp32 accumulators and
+//               commits each stage back to the producer
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator (one row per thread,
+//               32 consecutive columns per load), bias from shared memory,
+//               ReLU, mask words, 16-bit stores; for DRELU_BGRAD the mask is
+//               applied and each tile's column sums are reduced in a fixed
+//               order and written as one partial row per 128-row tile.
+// The two accumulators let the epilogue of tile i overlap the MMAs of tile
+// i+1.
+//
+// Every wait on an mbarrier is bounded: on expiry the kernel records a code
+// in the plan's status word, raises a CTA-wide abort flag, lets its issued
+// copies and MMAs finish, frees its tensor memory and returns.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace ge {
+
+enum EpiKind : int { EPI_BIAS = 0, EPI_RELU_BIAS = 1, EPI_RELU_AUX_BIAS = 2, EPI_DRELU_BGRAD = 3, EPI_STORE = 4 };
+
+struct TileParams {
+  int32_t T, N, K;
+  int32_t m_tiles, n_tiles, k_blocks, num_tiles;
+  int32_t aux_words;        // ceil(N / 32)
+  const void* bias;         // N values of the 16-bit type (forward)
+  void* out;                // T x N, 16-bit: Y, dZ, or the unfused intermediate
+  uint32_t* aux_out;        // RELU_AUX_BIAS mask words
+  const uint32_t* aux_in;   // DRELU_BGRAD mask words
+  float* partials;          // DRELU_BGRAD: m_tiles x N column partial sums
+  int* status;              // watchdog report (host-visible)
+  uint64_t timeout_ns;
+};
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;
+constexpr int kThreads = 192;
+constexpr int kGroupM = 8;
+
+template <int BN, int STAGES>
+struct TileSmem {
+  static constexpr uint32_t A_BYTES = kBM * kBK * 2;          // 16 KB
+  static constexpr uint32_t B_CHUNK = kBK * 64 * 2;           // 8 KB: 64 K-rows x 64 N
+  static constexpr uint32_t B_BYTES = (BN / 64) * B_CHUNK;
+  static constexpr uint32_t OFF_A = 0;
+  static constexpr uint32_t OFF_B = OFF_A + STAGES * A_BYTES;
+  static constexpr uint32_t OFF_BAR = OFF_B + STAGES * B_BYTES;
+  static constexpr uint32_t N_BARS = 2 * STAGES + 5;          // full, empty, tfull[2], tempty[2], drain
+  static constexpr uint32_t OFF_MISC = OFF_BAR + N_BARS * 8;  // tmem slot, abort flag
+  static constexpr uint32_t OFF_BIAS = (OFF_MISC + 16 + 15) / 16 * 16;
+  static constexpr uint32_t OFF_COLP = OFF_BIAS + 2 * BN * 4;
+  static constexpr uint32_t END = OFF_COLP + 2 * 4 * BN * 4;
+  static constexpr uint32_t BYTES = END + 1024;               // + alignment slack
+};
+
+__device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, int& mb, int& nb) {
+  const int per_group = kGroupM * n_tiles;
+  const int g = tile / per_group;
+  const int first_m = g * kGroupM;
+  const int gsize = min(m_tiles - first_m, kGroupM);
+  const int r = tile - g * per_group;
+  mb = first_m + r % gsize;
+  nb = r / gsize;
+}
+
+__device__ __noinline__ void report_timeout(int* status, volatile int* abort_flag, int site) {
+  *abort_flag = 1;
+  if (status) {
+    *reinterpret_cast<volatile int*>(status) = 0x7100 | site;
+    __threadfence_system();
+  }
+}
+
+// Wait for the phase of parity `parity` on `bar`. Returns false if the CTA
+// is aborting or the wait exceeded the time limit (then it raises the abort).
+__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, const TileParams& p,
+                                             volatile int* abort_flag, int site, bool honour_abort = true) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t n = 1;; ++n) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((n & 63u) == 0) {
+      if (honour_abort && *abort_flag) return false;
+      if (globaltimer_ns() - t0 > p.timeout_ns) {
+        report_timeout(p.status, abort_flag, site);
+        return false;
+      }
+    }
+  }
+}
+
+template <bool BF16>
+__device__ __forceinline__ float load_16(const void* base, int64_t i) {
+  if constexpr (BF16)
+    return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(base)[i]);
+  else
+    return __half2float(reinterpret_cast<const __half*>(base)[i]);
+}
+
+template <bool BF16>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  if constexpr (BF16) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+  } else {
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+}
+
+// Sum 32 per-lane vectors across the warp: on return, v[0] of lane j holds
+// the sum over all 32 lanes of their v[j]. Each step halves the columns a
+// lane keeps and swaps the other half with its partner, in a fixed order.
+__device__ __forceinline__ void warp_transpose_reduce32(float (&v)[32]) {
+  const uint32_t lane = lane_id();
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    const bool upper = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < off; ++i) {
+      const float send = upper ? v[i] : v[i + off];
+      const float keep = upper ? v[i + off] : v[i];
+      const float recv = __shfl_xor_sync(0xffffffffu, send, off);
+      v[i] = keep + recv;
+    }
+  }
+}
+
+template <int BN, int STAGES, int EPI, bool BF16>
+__global__ void __launch_bounds__(kThreads, 1)
+    tile_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const TileParams p) {
+  using L = TileSmem<BN, STAGES>;
+  static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN must be 64, 128, 192 or 256");
+  constexpr uint32_t TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
+                                 : (2 * BN <= 256) ? 256 : 512;
+  constexpr uint32_t IDESC = idesc_f16(BF16, /*A MN-major*/ false, /*B MN-major*/ true, kBM, BN);
+  constexpr uint32_t STAGE_TX = L::A_BYTES + L::B_BYTES;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem + L::OFF_A;
+  uint8_t* sB = smem + L::OFF_B;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+  float* bias_s = reinterpret_cast<float*>(smem + L::OFF_BIAS);  // [2][BN]
+  float* colp_s = reinterpret_cast<float*>(smem + L::OFF_COLP);  // [2][4][BN]
+
+  const uint32_t warp = threadIdx.x >> 5;
+  const uint32_t lane = lane_id();
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+        int mb, nb;
+        tile_coords(tile, p.m_tiles, p.n_tiles, mb, nb);
+        const int m0 = mb * kBM, n0 = nb * BN;
+        for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+          const uint32_t s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1u;
+          if (!wait_bounded(&empty[s], ph ^ 1u, p, abort_flag, 1)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[s], STAGE_TX);
+          tma_load_2d(sA + s * L::A_BYTES, &tmA, &full[s], kb * kBK, m0);
+#pragma unroll
+          for (int j = 0; j < BN / 64; ++j)
+            tma_load_2d(sB + s * L::B_BYTES + j * L::B_CHUNK, &tmB, &full[s], n0 + j * 64, kb * kBK);
+        }
+      }
+      // let every issued copy land before the CTA can exit
+      const uint32_t inflight = it < STAGES ? it : STAGES;
+      for (uint32_t i = it - inflight; i < it; ++i)
+        wait_bounded(&full[i % STAGES], (i / STAGES) & 1u, p, abort_flag, 2, /*honour_abort=*/false);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA
+    if (lane == 0) {
+      uint32_t it = 0, tcount = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++tcount) {
+        const uint32_t buf = tcount & 1u;
+        const uint32_t tph = (tcount >> 1) & 1u;
+        if (!wait_bounded(&tempty[buf], tph ^ 1u, p, abort_flag, 3)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + buf * BN;
+        for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+          const uint32_t s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1u;
+          if (!wait_bounded(&full[s], ph, p, abort_flag, 4)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + s * L::A_BYTES);
+          const uint32_t b0 = smem_u32(sB + s * L::B_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            // A: K-major, 128-byte rows, 8-row groups 1024 B apart; a K step of
+            // 16 elements is 32 bytes inside the swizzle atom.
+            const uint64_t adesc = smem_desc_sw128(a0 + kk * 32, 16, 1024);
+            // B: N-major, 64-wide N chunks 8 KB apart (LBO), 8 K-rows 1024 B
+            // apart (SBO); a K step of 16 rows is 2048 bytes.
+            const uint64_t bdesc = smem_desc_sw128(b0 + kk * 2048, L::B_CHUNK, 1024);
+            umma_f16(d_tmem, adesc, bdesc, IDESC, (kb | kk) != 0 ? 1u : 0u);
+          }
+          umma_commit(&empty[s]);
+        }
+        if (!ok) break;
+        umma_commit(&tfull[buf]);
+      }
+      // every MMA issued above must finish before tensor memory is freed
+      umma_commit(drain);
+      wait_bounded(drain, 0, p, abort_flag, 5, /*honour_abort=*/false);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const uint32_t ew = warp & 3u;        // TMEM lane quarter this warp may access
+    const uint32_t et = threadIdx.x - 64;  // 0..127
+    uint32_t tcount = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tcount) {
+      int mb, nb;
+      tile_coords(tile, p.m_tiles, p.n_tiles, mb, nb);
+      const int m0 = mb * kBM, n0 = nb * BN;
+      const uint32_t buf = tcount & 1u;
+      const uint32_t tph = (tcount >> 1) & 1u;
+      float* bs = bias_s + buf * BN;
+      float* cp = colp_s + buf * 4 * BN;
+      if constexpr (EPI == EPI_BIAS || EPI == EPI_RELU_BIAS || EPI == EPI_RELU_AUX_BIAS) {
+        for (int c = et; c < BN; c += 128) {
+          const int n = n0 + c;
+          bs[c] = n < p.N ? load_16<BF16>(p.bias, n) : 0.f;
+        }
+      }
+      named_bar_sync(1, 128);
+      if (ok) ok = wait_bounded(&tfull[buf], tph, p, abort_flag, 6);
+      ok = __all_sync(0xffffffffu, ok);
+      if (ok) {
+        tc_fence_after();
+        const int row = m0 + static_cast<int>(ew * 32 + lane);
+        const bool row_ok = row < p.T;
+        const uint32_t tbase = tmem_base + ((ew * 32u) << 16) + buf * BN;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          const int nc0 = n0 + c * 32;
+          if (nc0 >= p.N) break;  // warp-uniform
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(tbase + c * 32, r);
+          tmem_wait_ld();
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+          if constexpr (EPI == EPI_DRELU_BGRAD) {
+            const uint32_t m = row_ok ? __ldg(p.aux_in + static_cast<int64_t>(row) * p.aux_words + (nc0 >> 5)) : 0u;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = ((m >> j) & 1u) ? v[j] : 0.f;
+          } else if constexpr (EPI != EPI_STORE) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] += bs[c * 32 + j];
+            if constexpr (EPI == EPI_RELU_BIAS || EPI == EPI_RELU_AUX_BIAS) {
+              uint32_t m = 0;
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                const bool pos = v[j] > 0.f;
+                m |= (pos ? 1u : 0u) << j;
+                v[j] = pos ? v[j] : 0.f;
+              }
+              if constexpr (EPI == EPI_RELU_AUX_BIAS) {
+                const int valid = p.N - nc0;
+                if (valid < 32) m &= (1u << valid) - 1u;
+                if (row_ok) p.aux_out[static_cast<int64_t>(row) * p.aux_words + (nc0 >> 5)] = m;
+              }
+            }
+          }
+          if (row_ok) {
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.out) +
+                                                  static_cast<int64_t>(row) * p.N + nc0);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              if (nc0 + 8 * q < p.N) {
+                uint4 w;
+                w.x = pack2<BF16>(v[8 * q + 0], v[8 * q + 1]);
+                w.y = pack2<BF16>(v[8 * q + 2], v[8 * q + 3]);
+                w.z = pack2<BF16>(v[8 * q + 4], v[8 * q + 5]);
+                w.w = pack2<BF16>(v[8 * q + 6], v[8 * q + 7]);
+                dst[q] = w;
+              }
+            }
+          }
+          if constexpr (EPI == EPI_DRELU_BGRAD) {
+            warp_transpose_reduce32(v);
+            cp[ew * BN + c * 32 + lane] = v[0];
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[buf]);
+      }
+      if constexpr (EPI == EPI_DRELU_BGRAD) {
+        named_bar_sync(1, 128);
+        if (ok) {
+          for (int c = et; c < BN; c += 128) {
+            const int n = n0 + c;
+            if (n < p.N)
+              p.partials[static_cast<int64_t>(mb) * p.N + n] = ((cp[0 * BN + c] + cp[1 * BN + c]) + cp[2 * BN + c]) +
+                                                               cp[3 * BN + c];
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+}
+
+}  // namespace ge

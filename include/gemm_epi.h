@@ -1,0 +1,172 @@
+/*
+ * gemm_epi.h -- C ABI of the fused linear-layer GEMM + epilogue library for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The library mirrors the plan / execute / free life cycle of the pages'
+ * stateful matmul object ("Fusing bias addition into matrix multiplication
+ * with nvmath-python", life-cycle and stream items of its checklist;
+ * "nvmath-python cuBLASLt bindings for PyTorch fusion", the three-step
+ * init / plan / execute pattern): a plan fixes the shape, the 16-bit type and
+ * the epilog once, and is then executed any number of times.
+ *
+ * Layouts (all row-major, every 16-bit tensor of a call has the plan's dtype):
+ *   X     T x K      activations                 (K contiguous)
+ *   W     K x N      weight                      (N contiguous)
+ *   bias  N          one value per output feature, broadcast over the T rows
+ *   Y     T x N      output
+ *   aux   T x ceil(N/32) uint32 ReLU mask words: bit (n % 32) of word
+ *         [t][n / 32] is 1 iff the pre-activation Z[t][n] > 0 (strictly),
+ *         least significant bit first; bits past N are 0.
+ *   dY2   T x K      gradient input of the backward product (K plays D2)
+ *   W2    K x N      second operand of the backward product
+ *   dZ    T x N      masked gradient
+ *   dbias N          fp32 bias gradient
+ *
+ * Arithmetic: products accumulate in fp32 (tensor cores, fp32 accumulators in
+ * tensor memory); the bias is converted to fp32 and added; outputs are rounded
+ * to the 16-bit type with round-to-nearest-even.
+ *
+ * Streams and ownership: every execute call is asynchronous on the caller's
+ * stream and never synchronises (the pages' execute is non-blocking; the
+ * caller synchronises before reading results). The caller owns every tensor.
+ * A plan owns only its workspace and host state, allocated by gemm_epi_plan
+ * and released by gemm_epi_free; execute calls allocate nothing. One plan
+ * must not run concurrently on two streams (its workspace is shared).
+ *
+ * Errors: functions return GEMM_EPI_OK (0) or a negative code; a message is
+ * kept per thread and read with gemm_epi_last_error(). Argument errors are
+ * detected before anything is launched.
+ */
+#ifndef GEMM_EPI_H
+#define GEMM_EPI_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GEMM_EPI_API __attribute__((visibility("default")))
+#else
+#define GEMM_EPI_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA runtime stream handle (same type as cuda_runtime_api.h's). */
+typedef struct CUstream_st* cudaStream_t;
+
+typedef enum { GEMM_EPI_F16 = 0, GEMM_EPI_BF16 = 1 } gemm_epi_dtype;
+
+/* The pages' epilog names ("Fusing bias addition into matrix multiplication
+ * with nvmath-python": BIAS, RELU_BIAS, RELU_AUX_BIAS; "nvmath-python fused
+ * epilogs for linear layers": DRELU_BGRAD). */
+typedef enum {
+  GEMM_EPI_BIAS = 0,          /* Y = X.W + bias                              */
+  GEMM_EPI_RELU_BIAS = 1,     /* Y = relu(X.W + bias)                        */
+  GEMM_EPI_RELU_AUX_BIAS = 2, /* Y = relu(X.W + bias), aux = mask (Z > 0)    */
+  GEMM_EPI_DRELU_BGRAD = 3    /* dZ = (dY2.W2) masked by aux, dbias = sum_t dZ */
+} gemm_epi_epilog;
+
+enum {
+  GEMM_EPI_OK = 0,
+  GEMM_EPI_ERR_INVALID_ARG = -1,     /* bad dimension, enum, NULL pointer or unknown plan */
+  GEMM_EPI_ERR_MISALIGNED = -2,      /* a pointer is not aligned as required below        */
+  GEMM_EPI_ERR_EPILOG_MISMATCH = -3, /* call does not fit the plan's epilog              */
+  GEMM_EPI_ERR_CUDA = -4,            /* CUDA runtime / driver error (message kept)        */
+  GEMM_EPI_ERR_TIMEOUT = -5,         /* a kernel's bounded wait expired (watchdog)        */
+  GEMM_EPI_ERR_UNSUPPORTED = -6      /* no device of compute capability 10.0             */
+};
+
+typedef struct gemm_epi_plan_s* gemm_epi_plan_t;
+
+/* What a plan chose, for logs and tests. */
+typedef struct {
+  int64_t T, N, K;
+  int dtype, epilog;
+  int kernel;          /* 0 = persistent tile kernel, 1 = skinny (swap-AB, split-K) kernel */
+  int tile_m, tile_n, tile_k, stages;
+  int split_k;         /* K slices per output tile (1 = none) */
+  int grid;            /* CTAs launched by the main kernel */
+  int launches;        /* kernel launches per execute call */
+  int num_sms;
+  size_t workspace_bytes;
+} gemm_epi_info;
+
+/*
+ * gemm_epi_plan: validate a problem and choose its kernel configuration.
+ *   T >= 1 rows; N >= 8 and K >= 8, both multiples of 8 (16-byte row
+ *   strides); dtype and epilog from the enums above. For DRELU_BGRAD, K is
+ *   the contraction length D2 of G = dY2 . W2 (a backward plan is separate
+ *   from the forward plan, as the pages build a separate matmul for it).
+ *   Uses the current CUDA device; allocates the plan's workspace there.
+ * Returns a plan, or NULL with gemm_epi_last_error() set.
+ */
+GEMM_EPI_API gemm_epi_plan_t gemm_epi_plan(int64_t T, int64_t N, int64_t K, gemm_epi_dtype dtype,
+                              gemm_epi_epilog epilog);
+
+/*
+ * gemm_epi_execute: the forward epilogs (BIAS, RELU_BIAS, RELU_AUX_BIAS).
+ *   X, W, Y: device pointers, 16-byte aligned. bias: device pointer, 2-byte
+ *   aligned, never NULL. aux: device pointer, 4-byte aligned, required for
+ *   RELU_AUX_BIAS and ignored (may be NULL) otherwise.
+ * Returns GEMM_EPI_OK once the work is enqueued on `stream`;
+ * GEMM_EPI_ERR_EPILOG_MISMATCH on a DRELU_BGRAD plan or a missing aux;
+ * GEMM_EPI_ERR_TIMEOUT if an earlier call on this plan reported a watchdog
+ * expiry (the report is cleared by reading it).
+ */
+GEMM_EPI_API int gemm_epi_execute(gemm_epi_plan_t plan, const void* X, const void* W, const void* bias, void* Y,
+                     uint32_t* aux, cudaStream_t stream);
+
+/*
+ * drelu_bgrad_execute: DRELU_BGRAD ("nvmath-python fused epilogs for linear
+ * layers", DRELU_BGRAD section): G = dY2 . W2, dZ = G where the mask bit of
+ * aux is set, else 0 (rounded to dtype), and dbias[n] = sum over t of the
+ * fp32 masked G, reduced in a fixed order (bitwise reproducible).
+ *   dY2 (T x K), W2 (K x N), dZ (T x N): device, 16-byte aligned.
+ *   aux: device, 4-byte aligned, the forward's relu_aux (T x ceil(N/32)).
+ *   dbias: device, 4-byte aligned, N floats.
+ * Returns as gemm_epi_execute; GEMM_EPI_ERR_EPILOG_MISMATCH on a forward plan.
+ */
+GEMM_EPI_API int drelu_bgrad_execute(gemm_epi_plan_t plan, const void* dY2, const void* W2, const uint32_t* aux,
+                        void* dZ, float* dbias, cudaStream_t stream);
+
+/* Release a plan and its workspace. NULL and already-freed plans are
+ * ignored. The caller must make sure no work of the plan is still running
+ * (synchronise its stream first). */
+GEMM_EPI_API void gemm_epi_free(gemm_epi_plan_t plan);
+
+/* The calling thread's last error message ("" if none). */
+GEMM_EPI_API const char* gemm_epi_last_error(void);
+
+/* Fill *info with the plan's choices. Returns GEMM_EPI_OK or ERR_INVALID_ARG. */
+GEMM_EPI_API int gemm_epi_query(gemm_epi_plan_t plan, gemm_epi_info* info);
+
+/* After the caller synchronised the plan's stream: GEMM_EPI_OK, or
+ * GEMM_EPI_ERR_TIMEOUT if a kernel of this plan gave up on a wait (and then
+ * left its outputs incomplete). Reading clears the report. */
+GEMM_EPI_API int gemm_epi_status(gemm_epi_plan_t plan);
+
+/*
+ * Unfused path, for measurement only (the pages' three-kernel baseline,
+ * "AI inference compiler optimisation: operator fusion", section 2.2:
+ * MatMul writes an intermediate, BiasAdd reads it and writes another, ReLU
+ * reads that and writes the output).
+ *   gemm_epi_unfused_execute: GEMM -> T1 (T x N, dtype), T1 + bias -> T2,
+ *   relu(T2) -> Y (and, for RELU_AUX_BIAS, the mask from T2 > 0 -> aux).
+ *   For BIAS the ReLU kernel is skipped and T2 is the output: pass Y as T2.
+ *   drelu_bgrad_unfused_execute: GEMM -> G (dtype), mask apply -> dZ,
+ *   column sum of dZ -> dbias (fixed order).
+ * T1, T2, G: caller-owned device scratch of T x N dtype, 16-byte aligned.
+ */
+GEMM_EPI_API int gemm_epi_unfused_execute(gemm_epi_plan_t plan, const void* X, const void* W, const void* bias,
+                             void* T1, void* T2, void* Y, uint32_t* aux, cudaStream_t stream);
+GEMM_EPI_API int drelu_bgrad_unfused_execute(gemm_epi_plan_t plan, const void* dY2, const void* W2,
+                                const uint32_t* aux, void* G, void* dZ, float* dbias,
+                                cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GEMM_EPI_H */

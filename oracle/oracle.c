@@ -90,32 +90,49 @@ typedef struct {
   double* S;             /* nr x nc */
 } job_t;
 
+#define ROWS_PER_PASS 8
+
+/* Rows are taken ROWS_PER_PASS at a time so that each decoded row of B is
+ * read once per pass instead of once per row; every output element is still
+ * its own binary64 sum, taken over k in ascending order. */
 static void* worker(void* p) {
   job_t* j = (job_t*)p;
   const int64_t nc = j->nc;
-  for (int64_t i = j->row_begin; i < j->row_end; ++i) {
-    const int64_t r = j->rows ? j->rows[i] : i;
-    double* c = j->C + i * nc;
-    double* s = j->S + i * nc;
-    for (int64_t q = 0; q < nc; ++q) {
-      c[q] = 0.0;
-      s[q] = 0.0;
-    }
-    const uint16_t* arow = j->A + r * j->K;
-    /* k ascending for every output element of this row */
-    for (int64_t k = 0; k < j->K; ++k) {
-      const double a = decode(arow[k], j->dtype);
-      const double* brow = j->Bsel + k * nc;
+  for (int64_t i0 = j->row_begin; i0 < j->row_end; i0 += ROWS_PER_PASS) {
+    const int nrow = (int)(j->row_end - i0 < ROWS_PER_PASS ? j->row_end - i0 : ROWS_PER_PASS);
+    const uint16_t* arow[ROWS_PER_PASS];
+    double* c[ROWS_PER_PASS];
+    double* s[ROWS_PER_PASS];
+    for (int r = 0; r < nrow; ++r) {
+      const int64_t i = i0 + r;
+      const int64_t row = j->rows ? j->rows[i] : i;
+      arow[r] = j->A + row * j->K;
+      c[r] = j->C + i * nc;
+      s[r] = j->S + i * nc;
       for (int64_t q = 0; q < nc; ++q) {
-        const double prod = a * brow[q];
-        c[q] += prod;
-        s[q] += fabs(prod);
+        c[r][q] = 0.0;
+        s[r][q] = 0.0;
+      }
+    }
+    for (int64_t k = 0; k < j->K; ++k) {
+      const double* brow = j->Bsel + k * nc;
+      for (int r = 0; r < nrow; ++r) {
+        const double a = decode(arow[r][k], j->dtype);
+        double* cr = c[r];
+        double* sr = s[r];
+        for (int64_t q = 0; q < nc; ++q) {
+          const double prod = a * brow[q];
+          cr[q] += prod;
+          sr[q] += fabs(prod);
+        }
       }
     }
     if (j->bsel) {
-      for (int64_t q = 0; q < nc; ++q) {
-        c[q] += j->bsel[q];
-        s[q] += fabs(j->bsel[q]);
+      for (int r = 0; r < nrow; ++r) {
+        for (int64_t q = 0; q < nc; ++q) {
+          c[r][q] += j->bsel[q];
+          s[r][q] += fabs(j->bsel[q]);
+        }
       }
     }
   }

@@ -1,0 +1,171 @@
+"""Helpers for the GPU parity tests: run the library through its C ABI and
+compare with the CPU oracle under the acceptance bounds.
+
+Bounds (per element): Y and dZ within 2e-3 * S + u * |ref|, where S is the
+oracle's sum of |products| (+ |bias|) and u the unit roundoff of the 16-bit
+output (2^-8 for bf16, 2^-11 for fp16): the 2e-3 * S term bounds the
+computation, the u * |ref| term the one final rounding to the output type,
+which 2e-3 * S alone cannot cover when |Y| is close to S (small K, bf16);
+dbias (fp32) within 1e-3 * sum_t |dZ|; relu_aux
+bit-exact wherever |Z_ref| > 2e-3 * S. For integer-valued inputs every
+result is exact, so the comparison there is equality.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from gemm_epilogues_tcgen05_b200 import Plan, synth
+
+Y_REL = 2e-3
+DBIAS_REL = 1e-3
+GUARD = 4096  # sentinel elements before and after each output
+SENTINEL16 = 0x7E5A  # a 16-bit pattern no result takes in these tests
+SENTINEL32 = 0x5A5A5A5A
+
+
+def odt(dtype: torch.dtype) -> int:
+    return oracle.BF16 if dtype == torch.bfloat16 else oracle.F16
+
+
+def guarded(shape, dtype, device):
+    """An output tensor inside a larger buffer whose margins hold a sentinel."""
+    n = int(np.prod(shape))
+    if dtype in (torch.float16, torch.bfloat16):
+        buf = torch.full((n + 2 * GUARD,), SENTINEL16, dtype=torch.int16, device=device).view(dtype)
+    elif dtype == torch.int32:
+        buf = torch.full((n + 2 * GUARD,), SENTINEL32, dtype=torch.int32, device=device)
+    else:
+        buf = torch.full((n + 2 * GUARD,), float("nan"), dtype=dtype, device=device)
+    return buf, buf[GUARD:GUARD + n].view(shape)
+
+
+def guards_intact(buf) -> bool:
+    head, tail = buf[:GUARD], buf[-GUARD:]
+    if buf.dtype in (torch.float16, torch.bfloat16):
+        h, t = head.view(torch.int16), tail.view(torch.int16)
+        return bool(torch.all(h == SENTINEL16)) and bool(torch.all(t == SENTINEL16))
+    if buf.dtype == torch.int32:
+        return bool(torch.all(head == SENTINEL32)) and bool(torch.all(tail == SENTINEL32))
+    return bool(torch.all(torch.isnan(head))) and bool(torch.all(torch.isnan(tail)))
+
+
+def run_forward(inp_cpu: dict, epilog: str, dtype, device="cuda", unfused=False):
+    X, W, b = (inp_cpu[k].to(device) for k in ("X", "W", "bias"))
+    T, K = X.shape
+    N = W.shape[1]
+    with Plan(T, N, K, dtype, epilog) as plan:
+        info = plan.info()
+        ybuf, Y = guarded((T, N), dtype, device)
+        abuf, aux = guarded((T, (N + 31) // 32), torch.int32, device)
+        aux_arg = aux if epilog == "RELU_AUX_BIAS" else None
+        if unfused:
+            T1 = torch.empty((T, N), dtype=dtype, device=device)
+            T2 = Y if epilog == "BIAS" else torch.empty((T, N), dtype=dtype, device=device)
+            plan.gemm_epi_unfused_execute(X, W, b, T1, T2, Y, aux_arg)
+        else:
+            plan.gemm_epi_execute(X, W, b, Y, aux_arg)
+        torch.cuda.synchronize()
+        assert plan.status() == 0, "watchdog fired"
+    assert guards_intact(ybuf), "Y guard region overwritten"
+    if epilog == "RELU_AUX_BIAS":
+        assert guards_intact(abuf), "aux guard region overwritten"
+    out = {"Y": Y.cpu(), "info": info}
+    if epilog == "RELU_AUX_BIAS":
+        out["aux"] = aux.cpu().numpy().view(np.uint32)
+    return out
+
+
+def run_backward(inp_cpu: dict, aux_words: np.ndarray, dtype, device="cuda", unfused=False, repeats=1):
+    dY2, W2 = inp_cpu["dY2"].to(device), inp_cpu["W2"].to(device)
+    T, D2 = dY2.shape
+    N = W2.shape[1]
+    aux = torch.from_numpy(np.ascontiguousarray(aux_words).view(np.int32)).to(device)
+    outs = []
+    with Plan(T, N, D2, dtype, "DRELU_BGRAD") as plan:
+        info = plan.info()
+        for _ in range(repeats):
+            zbuf, dZ = guarded((T, N), dtype, device)
+            bbuf, dbias = guarded((N,), torch.float32, device)
+            if unfused:
+                G = torch.empty((T, N), dtype=dtype, device=device)
+                plan.drelu_bgrad_unfused_execute(dY2, W2, aux, G, dZ, dbias)
+            else:
+                plan.drelu_bgrad_execute(dY2, W2, aux, dZ, dbias)
+            torch.cuda.synchronize()
+            assert plan.status() == 0, "watchdog fired"
+            assert guards_intact(zbuf), "dZ guard region overwritten"
+            assert guards_intact(bbuf), "dbias guard region overwritten"
+            outs.append({"dZ": dZ.cpu(), "dbias": dbias.cpu(), "info": info})
+    return outs if repeats > 1 else outs[0]
+
+
+def unit_roundoff(dtype) -> float:
+    return {torch.bfloat16: 2.0 ** -8, torch.float16: 2.0 ** -11}.get(dtype, 0.0)
+
+
+def assert_within(got: np.ndarray, ref: np.ndarray, scale: np.ndarray, rel: float, what: str, out_u: float = 0.0):
+    got = np.asarray(got, dtype=np.float64)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite values"
+    err = np.abs(got - ref)
+    bound = rel * scale + out_u * np.abs(ref)
+    bad = err > bound
+    if bad.any():
+        idx = np.argwhere(bad)[:5].tolist()
+        worst = float(np.max(err / np.maximum(bound, 1e-300)))
+        raise AssertionError(f"{what}: {int(bad.sum())} of {bad.size} outside {rel}*S; worst ratio {worst:.3g}; "
+                             f"first at {idx}")
+
+
+def check_forward(inp_cpu, epilog, dtype, gpu, rows=None, cols=None, exact=False):
+    bits = synth.bits_u16
+    ref = oracle.linear_fwd(bits(inp_cpu["X"]), bits(inp_cpu["W"]), bits(inp_cpu["bias"]), odt(dtype), epilog,
+                            rows=rows, cols=cols)
+    Y = gpu["Y"]
+    r_idx = slice(None) if rows is None else torch.tensor(rows)
+    c_idx = slice(None) if cols is None else torch.tensor(cols)
+    Ys = Y[r_idx][:, c_idx].double().numpy()
+    if exact:
+        expect = torch.from_numpy(ref["Y"]).to(dtype).double().numpy()  # exact Z rounded once
+        assert np.array_equal(Ys, expect), f"{epilog}: Y not bit-exact on integer inputs"
+    else:
+        assert_within(Ys, ref["Y"], ref["S"], Y_REL, f"{epilog} Y", unit_roundoff(dtype))
+    if epilog != "BIAS":
+        assert np.all(Ys >= 0), "ReLU output negative"
+    if epilog == "RELU_AUX_BIAS":
+        N = Y.shape[1]
+        got_bits = oracle.relu_aux_bits(gpu["aux"], N)
+        got_bits = got_bits[(slice(None) if rows is None else rows)][:, (slice(None) if cols is None else cols)]
+        if exact:
+            assert np.array_equal(got_bits, ref["bits"]), "relu_aux not bit-exact on integer inputs"
+        else:
+            sure = np.abs(ref["Z"]) > Y_REL * ref["S"]
+            mism = (got_bits != ref["bits"]) & sure
+            assert not mism.any(), f"relu_aux differs at {int(mism.sum())} decided positions"
+        # pad bits past N are zero
+        if N % 32:
+            last = gpu["aux"][:, -1]
+            assert np.all((last >> np.uint32(N % 32)) == 0), "pad bits set"
+    return ref
+
+
+def check_backward(inp_cpu, aux_words, dtype, gpu, rows=None, cols=None, exact=False):
+    bits = synth.bits_u16
+    N = inp_cpu["W2"].shape[1]
+    ref = oracle.drelu_bgrad(bits(inp_cpu["dY2"]), bits(inp_cpu["W2"]), aux_words, odt(dtype), N, rows=rows, cols=cols)
+    r_idx = slice(None) if rows is None else torch.tensor(rows)
+    c_idx = slice(None) if cols is None else torch.tensor(cols)
+    dZ = gpu["dZ"][r_idx][:, c_idx].double().numpy()
+    if exact:
+        expect = torch.from_numpy(ref["dZ"]).to(dtype).double().numpy()
+        assert np.array_equal(dZ, expect), "dZ not bit-exact on integer inputs"
+    else:
+        assert_within(dZ, ref["dZ"], ref["S"], Y_REL, "dZ", unit_roundoff(dtype))
+    if rows is None:
+        db = gpu["dbias"][c_idx].double().numpy()
+        if exact:
+            assert np.array_equal(db, ref["dbias"]), "dbias not exact on integer inputs"
+        else:
+            assert_within(db, ref["dbias"], ref["Sb"], DBIAS_REL, "dbias")
+    return ref

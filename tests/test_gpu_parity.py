@@ -1,0 +1,155 @@
+"""GPU parity of the fused kernels against the CPU oracle, element by
+element, on shapes that span several tiles and ragged tails, for every
+epilog, both 16-bit types and every tile width the planner can choose."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gemm_epilogues_tcgen05_b200 import binding, synth
+
+from _parity import check_backward, check_forward, run_backward, run_forward
+
+pytestmark = pytest.mark.gpu
+
+DT = {"fp16": torch.float16, "bf16": torch.bfloat16}
+SHAPES = [(1, 8, 8), (5, 40, 24), (130, 72, 136), (200, 264, 200), (257, 520, 328), (384, 512, 512)]
+FWD_EPILOGS = ["BIAS", "RELU_BIAS", "RELU_AUX_BIAS"]
+
+
+@pytest.fixture(autouse=True)
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+@pytest.mark.parametrize("bn", [64, 128, 256])
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+@pytest.mark.parametrize("T,N,K", SHAPES)
+def test_forward_all_epilogs(monkeypatch, T, N, K, dtype, bn):
+    monkeypatch.setenv("GEMM_EPI_FORCE_BN", str(bn))
+    inp = synth.make_shape_inputs(T, N, K, dtype, seed=T * 7 + N + K)
+    for ep in FWD_EPILOGS:
+        gpu = run_forward(inp, ep, DT[dtype])
+        assert gpu["info"]["tile_n"] == bn
+        check_forward(inp, ep, DT[dtype], gpu)
+
+
+@pytest.mark.parametrize("bn", [64, 128, 256])
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+@pytest.mark.parametrize("T,N,K", SHAPES)
+def test_backward_drelu_bgrad(monkeypatch, T, N, K, dtype, bn):
+    monkeypatch.setenv("GEMM_EPI_FORCE_BN", str(bn))
+    D2 = max(8, (K // 2) // 8 * 8)
+    inp = synth.make_shape_inputs(T, N, K, dtype, seed=T * 5 + N + K, D2=D2)
+    fwd = run_forward(inp, "RELU_AUX_BIAS", DT[dtype])
+    gpu = run_backward(inp, fwd["aux"], DT[dtype])
+    check_backward(inp, fwd["aux"], DT[dtype], gpu)
+
+
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+@pytest.mark.parametrize("T,N,K,D2", [(130, 72, 64, 40), (257, 520, 128, 96), (64, 8, 8, 8)])
+def test_integer_inputs_bit_exact(T, N, K, D2, dtype):
+    """Integer inputs: every sum is exact in fp32, so Y, aux, dZ and dbias
+    must equal the exact result rounded once (pins ties Z == 0, the mask
+    layout and the backward operand orientation)."""
+    inp = synth.make_shape_inputs(T, N, K, dtype, seed=900 + T, D2=D2, kind="int")
+    for ep in FWD_EPILOGS:
+        gpu = run_forward(inp, ep, DT[dtype])
+        check_forward(inp, ep, DT[dtype], gpu, exact=True)
+    fwd = run_forward(inp, "RELU_AUX_BIAS", DT[dtype])
+    gpu = run_backward(inp, fwd["aux"], DT[dtype])
+    check_backward(inp, fwd["aux"], DT[dtype], gpu, exact=True)
+
+
+def test_zero_bias_is_plain_gemm_relu():
+    T, N, K = 200, 136, 96
+    inp = synth.make_shape_inputs(T, N, K, "fp16", seed=77)
+    inp["bias"] = torch.zeros(N, dtype=torch.float16)
+    gpu = run_forward(inp, "RELU_BIAS", torch.float16)
+    ref = (inp["X"].double() @ inp["W"].double()).clamp_min(0)
+    S = (inp["X"].double().abs() @ inp["W"].double().abs())
+    assert torch.all((gpu["Y"].double() - ref).abs() <= 2e-3 * S)
+
+
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+def test_unfused_path_matches_oracle(dtype):
+    T, N, K, D2 = 257, 264, 200, 136
+    inp = synth.make_shape_inputs(T, N, K, dtype, seed=31, D2=D2)
+    for ep in FWD_EPILOGS:
+        gpu = run_forward(inp, ep, DT[dtype], unfused=True)
+        check_forward(inp, ep, DT[dtype], gpu)
+    fwd = run_forward(inp, "RELU_AUX_BIAS", DT[dtype])
+    gpu = run_backward(inp, fwd["aux"], DT[dtype], unfused=True)
+    check_backward(inp, fwd["aux"], DT[dtype], gpu)
+
+
+def test_dbias_bitwise_reproducible_across_runs_and_streams():
+    T, N, D2 = 1000, 520, 264
+    inp = synth.make_shape_inputs(T, N, 64, "bf16", seed=5, D2=D2)
+    fwd = run_forward(inp, "RELU_AUX_BIAS", torch.bfloat16)
+    outs = run_backward(inp, fwd["aux"], torch.bfloat16, repeats=3)
+    for o in outs[1:]:
+        assert torch.equal(o["dbias"], outs[0]["dbias"])
+        assert torch.equal(o["dZ"].view(torch.int16), outs[0]["dZ"].view(torch.int16))
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        other = run_backward(inp, fwd["aux"], torch.bfloat16)
+    s.synchronize()
+    assert torch.equal(other["dbias"], outs[0]["dbias"])
+
+
+def test_plan_reuse_many_executes():
+    """One plan, several executes with different buffers (tensor maps re-encoded)."""
+    T, N, K = 300, 264, 136
+    with binding.Plan(T, N, K, torch.float16, "RELU_AUX_BIAS") as plan:
+        for seed in (1, 2, 3):
+            inp = synth.make_shape_inputs(T, N, K, "fp16", seed=seed)
+            g = {k: v.cuda() for k, v in inp.items()}
+            Y, aux = plan.forward(g["X"], g["W"], g["bias"])
+            torch.cuda.synchronize()
+            check_forward(inp, "RELU_AUX_BIAS", torch.float16,
+                          {"Y": Y.cpu(), "aux": aux.cpu().numpy().view(np.uint32)})
+
+
+def test_error_paths_on_device():
+    T, N, K = 64, 64, 64
+    dev = "cuda"
+    X = torch.zeros(T * K + 8, dtype=torch.float16, device=dev)
+    W = torch.zeros(K, N, dtype=torch.float16, device=dev)
+    b = torch.zeros(N, dtype=torch.float16, device=dev)
+    Y = torch.zeros(T, N, dtype=torch.float16, device=dev)
+    L = binding.lib()
+    h = binding.gemm_epi_plan(T, N, K, binding.F16, binding.RELU_AUX_BIAS)
+    try:
+        s = torch.cuda.current_stream().cuda_stream
+        # misaligned X (2-byte offset)
+        rc = L.gemm_epi_execute(h, X.data_ptr() + 2, W.data_ptr(), b.data_ptr(), Y.data_ptr(), Y.data_ptr(), s)
+        assert rc == binding.ERR_MISALIGNED
+        # RELU_AUX_BIAS without aux
+        rc = L.gemm_epi_execute(h, X.data_ptr(), W.data_ptr(), b.data_ptr(), Y.data_ptr(), None, s)
+        assert rc == binding.ERR_EPILOG_MISMATCH
+        # backward call on a forward plan
+        rc = L.drelu_bgrad_execute(h, X.data_ptr(), W.data_ptr(), Y.data_ptr(), Y.data_ptr(), Y.data_ptr(), s)
+        assert rc == binding.ERR_EPILOG_MISMATCH
+        # NULL bias
+        rc = L.gemm_epi_execute(h, X.data_ptr(), W.data_ptr(), None, Y.data_ptr(), Y.data_ptr(), s)
+        assert rc == binding.ERR_INVALID_ARG
+    finally:
+        binding.gemm_epi_free(h)
+    binding.gemm_epi_free(h)  # double free is ignored
+    assert L.gemm_epi_execute(h, X.data_ptr(), W.data_ptr(), b.data_ptr(), Y.data_ptr(), Y.data_ptr(),
+                              None) == binding.ERR_INVALID_ARG
+    hb = binding.gemm_epi_plan(T, N, K, binding.F16, binding.DRELU_BGRAD)
+    try:
+        rc = L.gemm_epi_execute(hb, X.data_ptr(), W.data_ptr(), b.data_ptr(), Y.data_ptr(), Y.data_ptr(), None)
+        assert rc == binding.ERR_EPILOG_MISMATCH
+    finally:
+        binding.gemm_epi_free(hb)
+
+
+def test_injected_workspace_allocation_failure(monkeypatch):
+    monkeypatch.setenv("GEMM_EPI_INJECT_PLAN_ALLOC_FAILURE", "1")
+    with pytest.raises(binding.GemmEpiError) as e:
+        binding.gemm_epi_plan(256, 256, 256, binding.BF16, binding.DRELU_BGRAD)
+    assert "injected" in str(e.value)
