@@ -337,11 +337,16 @@ def cpu_baseline(w: synth.Workload, fwd_epi: str, has_bwd: bool, target_s: float
     oracle.build()
     threads = oracle.default_threads()
     inp = synth.make_inputs(w, device="cpu")
-    n = min(w.T, 8)
-    dt, fl = oracle_step_rows(w, inp, list(range(n)), fwd_epi, has_bwd, threads)
-    rows_target = int(min(w.T, max(n, n * target_s / max(dt, 1e-6))))
-    rows = synth.sample_indices(w.T, rows_target, seed=w.seed)
+    # grow the row sample until one run takes about target_s (each run also
+    # pays a fixed cost for decoding W, so scale from the last measurement)
+    rows = list(range(min(w.T, 8)))
     dt, fl = oracle_step_rows(w, inp, rows, fwd_epi, has_bwd, threads)
+    for _ in range(3):
+        if dt >= 0.6 * target_s or len(rows) >= w.T:
+            break
+        want = int(min(w.T, max(len(rows) + 1, len(rows) * target_s / max(dt, 1e-6))))
+        rows = synth.sample_indices(w.T, want, seed=w.seed)
+        dt, fl = oracle_step_rows(w, inp, rows, fwd_epi, has_bwd, threads)
     return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
             "sample": f"{len(rows)} of {w.T} rows (every column), forward{' + backward' if has_bwd else ''}, "
                       f"fp64, {dt:.1f} s"}
@@ -397,8 +402,8 @@ def config_of(w, fwd_epi, has_bwd, args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=400)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="ffn", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ablation", action="store_true", help="time the unfused path instead")
