@@ -28,7 +28,10 @@ ERR_UNSUPPORTED = -6
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgemm_epi.so")
 
 EXPORTED = ["gemm_epi_plan", "gemm_epi_execute", "drelu_bgrad_execute", "gemm_epi_free", "gemm_epi_last_error",
-            "gemm_epi_query", "gemm_epi_status", "gemm_epi_unfused_execute", "drelu_bgrad_unfused_execute"]
+            "gemm_epi_query", "gemm_epi_status", "gemm_epi_unfused_execute", "drelu_bgrad_unfused_execute",
+            "drelu_bgrad_execute_noalloc"]
+
+NOALLOC_SCRATCH_BYTES = 4 << 20  # GEMM_EPI_NOALLOC_SCRATCH_BYTES
 
 
 class GemmEpiError(RuntimeError):
@@ -77,6 +80,8 @@ def lib() -> ctypes.CDLL:
         L.gemm_epi_unfused_execute.argtypes = [vp] * 9
         L.drelu_bgrad_unfused_execute.restype = ci
         L.drelu_bgrad_unfused_execute.argtypes = [vp] * 8
+        L.drelu_bgrad_execute_noalloc.restype = ci
+        L.drelu_bgrad_execute_noalloc.argtypes = [i64, i64, i64, ci] + [vp] * 6
         _lib = L
     return _lib
 
@@ -126,6 +131,26 @@ def gemm_epi_plan(T: int, N: int, K: int, dtype, epilog) -> int:
 
 def gemm_epi_free(handle) -> None:
     lib().gemm_epi_free(handle)
+
+
+def drelu_bgrad_execute_noalloc(dY2, W2, aux, dZ, dbias, stream=None):
+    """DRELU_BGRAD without a plan and without any device allocation.
+
+    For callers that may not allocate device memory (a host framework that
+    owns the device's memory, or an enqueue callback that must not call
+    cudaMalloc because it can synchronise the device). The column partials
+    live in the library's fixed 4 MiB static scratch, shared by every call:
+    calls that overlap on the GPU race, so keep them on one stream. The first
+    call on a device does a one-time set-up; make it before any stream
+    capture. If the kernel's watchdog fires, dbias comes back as NaN.
+    """
+    T, K = dY2.shape
+    N = W2.shape[1]
+    dt = dY2.dtype
+    args = (_ptr(dY2, (T, K), dt, "dY2"), _ptr(W2, (K, N), dt, "W2"),
+            _ptr(aux, (T, (N + 31) // 32), torch.int32, "aux"), _ptr(dZ, (T, N), dt, "dZ"),
+            _ptr(dbias, (N,), torch.float32, "dbias"))
+    _check(lib().drelu_bgrad_execute_noalloc(T, N, K, DTYPES[dt], *args, _stream_ptr(stream)))
 
 
 class Plan:

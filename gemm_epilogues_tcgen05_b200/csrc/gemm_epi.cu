@@ -480,3 +480,147 @@ int drelu_bgrad_unfused_execute(gemm_epi_plan_t plan, const void* dY2, const voi
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free DRELU_BGRAD (drelu_bgrad_execute_noalloc).
+//
+// For callers that may not allocate device memory: the column partials and
+// the watchdog word live in this fixed, file-scope device array instead of a
+// plan's workspace. In host code `g_noalloc_scratch` only names the symbol;
+// its device address comes from cudaGetSymbolAddress, looked up once per
+// device (with that device current) on the first call there.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocStatusBytes = 256;  // status word, padded to keep the partials 256-byte aligned
+constexpr size_t kNoAllocPartialBytes = GEMM_EPI_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocStatusBytes + kNoAllocPartialBytes];
+
+constexpr int kNoAllocMaxDevices = 64;
+
+struct NoAllocDevice {
+  std::once_flag once;
+  cudaError_t err = cudaSuccess;
+  const char* what = "";
+  unsigned char* scratch = nullptr;  // device address of g_noalloc_scratch on this device
+};
+NoAllocDevice g_noalloc_dev[kNoAllocMaxDevices];
+
+// dbias[n] = sum of partials over row tiles, ascending; NaN everywhere if
+// the tile kernel's watchdog fired during this call.
+__global__ void noalloc_dbias_finish_kernel(const float* __restrict__ partials, int m_tiles, int N,
+                                            float* __restrict__ dbias, const int* __restrict__ status) {
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  if (n >= N) return;
+  if (*reinterpret_cast<const volatile int*>(status) != 0) {
+    dbias[n] = __int_as_float(0x7fc00000);
+    return;
+  }
+  float s = 0.f;
+  for (int m = 0; m < m_tiles; ++m) s += partials[static_cast<int64_t>(m) * N + n];
+  dbias[n] = s;
+}
+
+int noalloc_setup(int dev, NoAllocDevice*& out) {
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return fail(GEMM_EPI_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  NoAllocDevice& d = g_noalloc_dev[dev];
+  std::call_once(d.once, [&d] {
+    void* p = nullptr;
+    d.err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (d.err != cudaSuccess) {
+      d.what = "cudaGetSymbolAddress(scratch)";
+      return;
+    }
+    d.scratch = static_cast<unsigned char*>(p);
+    for (int bn : {64, 128, 256}) {
+      for (bool bf16 : {false, true}) {
+        TileCfg c = tile_cfg(bn, ge::EPI_DRELU_BGRAD, bf16);
+        d.err = cudaFuncSetAttribute(c.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)c.smem);
+        if (d.err != cudaSuccess) {
+          d.what = "cudaFuncSetAttribute(max dynamic shared memory)";
+          return;
+        }
+      }
+    }
+  });
+  if (d.err != cudaSuccess) return cuda_fail(d.err, d.what);
+  out = &d;
+  return GEMM_EPI_OK;
+}
+
+}  // namespace
+
+extern "C" int drelu_bgrad_execute_noalloc(int64_t T, int64_t N, int64_t K, gemm_epi_dtype dtype, const void* dY2,
+                                           const void* W2, const uint32_t* aux, void* dZ, float* dbias,
+                                           cudaStream_t stream) {
+  if (T < 1 || N < 8 || K < 8 || (N % 8) != 0 || (K % 8) != 0 || T > ((int64_t)1 << 30) || N > ((int64_t)1 << 24) ||
+      K > ((int64_t)1 << 24))
+    return fail(GEMM_EPI_ERR_INVALID_ARG, "bad shape T=%lld N=%lld K=%lld (need T>=1, N,K>=8 and multiples of 8)",
+                (long long)T, (long long)N, (long long)K);
+  if (dtype != GEMM_EPI_F16 && dtype != GEMM_EPI_BF16)
+    return fail(GEMM_EPI_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+  const int64_t m_tiles = (T + ge::kBM - 1) / ge::kBM;
+  const uint64_t need = (uint64_t)m_tiles * (uint64_t)N * sizeof(float);
+  if (need > kNoAllocPartialBytes)
+    return fail(GEMM_EPI_ERR_INVALID_ARG,
+                "drelu_bgrad_execute_noalloc: T=%lld, N=%lld needs %llu bytes of column partials, more than its "
+                "fixed %u-byte scratch (ceil(T/128) * N * 4 must fit); use a plan instead",
+                (long long)T, (long long)N, (unsigned long long)need, (unsigned)kNoAllocPartialBytes);
+  if (!dY2 || !W2 || !aux || !dZ || !dbias)
+    return fail(GEMM_EPI_ERR_INVALID_ARG, "drelu_bgrad_execute_noalloc: NULL dY2, W2, aux, dZ or dbias");
+  if (!aligned(dY2, 16) || !aligned(W2, 16) || !aligned(dZ, 16) || !aligned(aux, 4) || !aligned(dbias, 4))
+    return fail(GEMM_EPI_ERR_MISALIGNED,
+                "drelu_bgrad_execute_noalloc: dY2, W2, dZ need 16-byte, aux and dbias 4-byte alignment");
+
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  int major = 0, minor = 0, sms = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (major != 10 || minor != 0)
+    return fail(GEMM_EPI_ERR_UNSUPPORTED, "device %d has compute capability %d.%d; this library needs 10.0", dev,
+                major, minor);
+  NoAllocDevice* nd = nullptr;
+  int rc = noalloc_setup(dev, nd);
+  if (rc) return rc;
+  int* status = reinterpret_cast<int*>(nd->scratch);
+  float* partials = reinterpret_cast<float*>(nd->scratch + kNoAllocStatusBytes);
+
+  const int bn = choose_bn(T, N, sms);
+  const TileCfg cfg = tile_cfg(bn, ge::EPI_DRELU_BGRAD, dtype == GEMM_EPI_BF16);
+  CUtensorMap tmA, tmB;
+  rc = encode_2d(&tmA, dY2, (uint64_t)K, (uint64_t)T, ge::kBK, ge::kBM, "dY2");
+  if (rc) return rc;
+  rc = encode_2d(&tmB, W2, (uint64_t)N, (uint64_t)K, 64, ge::kBK, "W2");
+  if (rc) return rc;
+
+  ge::TileParams k{};
+  k.T = (int32_t)T;
+  k.N = (int32_t)N;
+  k.K = (int32_t)K;
+  k.m_tiles = (int32_t)m_tiles;
+  k.n_tiles = ceil_div(N, bn);
+  k.k_blocks = ceil_div(K, ge::kBK);
+  k.num_tiles = k.m_tiles * k.n_tiles;
+  k.aux_words = ceil_div(N, 32);
+  k.out = dZ;
+  k.aux_in = aux;
+  k.partials = partials;
+  k.status = status;
+  k.timeout_ns = 2000000000ull;
+  const int grid = k.num_tiles < sms ? k.num_tiles : sms;
+
+  // the status word must start each call at zero; the partials are fully
+  // rewritten by the tile kernel before the finishing kernel reads them
+  e = cudaMemsetAsync(status, 0, sizeof(int), stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
+  cfg.fn<<<grid, ge::kThreads, cfg.smem, stream>>>(tmA, tmB, k);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "tile kernel launch");
+  noalloc_dbias_finish_kernel<<<ceil_div(N, 256), 256, 0, stream>>>(partials, k.m_tiles, (int)N, dbias, status);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "dbias finish launch");
+  return GEMM_EPI_OK;
+}

@@ -165,6 +165,49 @@ GEMM_EPI_API int drelu_bgrad_unfused_execute(gemm_epi_plan_t plan, const void* d
                                 const uint32_t* aux, void* G, void* dZ, float* dbias,
                                 cudaStream_t stream);
 
+/* Capacity of the fixed scratch used by drelu_bgrad_execute_noalloc: the
+ * backward needs ceil(T/128) * N floats of column partials. */
+#define GEMM_EPI_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+/*
+ * drelu_bgrad_execute_noalloc: the same DRELU_BGRAD computation as
+ * drelu_bgrad_execute, for callers that must not allocate device memory.
+ * (The pages have no counterpart: this is a deployment variant, not part of
+ * the method.)
+ *
+ * Who needs it: code that runs inside a host that owns all device memory --
+ * a framework's caching allocator or an inference engine with a fixed,
+ * pre-reserved budget -- where a raw cudaMalloc would bypass its accounting
+ * or fail once the pool has claimed the device; and enqueue-time plugin
+ * callbacks, which must not call cudaMalloc/cudaFree because those can
+ * synchronise the device and stall every other stream. Such callers cannot
+ * create a plan (gemm_epi_plan allocates its workspace), so this entry point
+ * takes the shape directly and allocates nothing: no cudaMalloc, no
+ * cudaFree, no allocating library call.
+ *
+ * Scratch: the column partial sums live in one fixed array of
+ * GEMM_EPI_NOALLOC_SCRATCH_BYTES (4 MiB) plus a 256-byte status block, in
+ * static device memory of this library; every GPU that loads the library
+ * keeps it until the process exits. Shapes whose partials exceed it
+ * (ceil(T/128) * N * 4 bytes > 4 MiB, e.g. T = 4096 needs N <= 32768) are
+ * rejected with GEMM_EPI_ERR_INVALID_ARG and a message, before any work.
+ * All calls share that array: two calls that overlap on the GPU (other
+ * streams, other host threads, same device) race on it and corrupt each
+ * other's dbias. Serialise them, e.g. on one stream.
+ *
+ * Arguments: T, N, K (K is D2) and dtype as for gemm_epi_plan with epilog
+ * DRELU_BGRAD; the pointers, alignment and layouts as drelu_bgrad_execute.
+ * First call on a device: it looks up the scratch array's device address
+ * and sets the kernel's shared-memory limit for that device, once; make
+ * that first call before any stream capture begins. Each call clears the
+ * status block, then launches two kernels on `stream` and returns without
+ * synchronising. If a kernel wait expires (the watchdog), every dbias entry
+ * is written as NaN instead of a sum.
+ */
+GEMM_EPI_API int drelu_bgrad_execute_noalloc(int64_t T, int64_t N, int64_t K, gemm_epi_dtype dtype,
+                                             const void* dY2, const void* W2, const uint32_t* aux, void* dZ,
+                                             float* dbias, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
