@@ -40,6 +40,8 @@ from gemm_epilogues_tcgen05_b200 import synth  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
+QUEUE_CHUNK = 32                 # steps queued behind one GPU sleep
+QUEUE_SLEEP_CYCLES = 3_000_000   # ~1.5 ms at 2 GHz: longer than the host needs to queue a chunk
 
 
 # ------------------------------------------------------------------ setup
@@ -159,7 +161,7 @@ class ClockSampler:
 
 # ----------------------------------------------------------------- our arm
 def run_ours(args, w: synth.Workload, rank: int, world: int, dev: torch.device):
-    from gemm_epilogues_tcgen05_b200 import Plan
+    from gemm_epilogues_tcgen05_b200 import Plan, binding
 
     fwd_epi, has_bwd = step_spec(w)
     dt = w.torch_dtype
@@ -186,26 +188,41 @@ def run_ours(args, w: synth.Workload, rank: int, world: int, dev: torch.device):
     stream = torch.cuda.current_stream(dev)
     fwd_aux = aux if fwd_epi == "RELU_AUX_BIAS" else None
 
+    # prebuilt C calls: the timed loop does no per-call argument checking
+    if args.ablation:
+        fcall = fplan.unfused_call(X, W, b, T1, T2 if fwd_epi != "BIAS" else Y, Y, fwd_aux, stream)
+        bcall = bplan.drelu_bgrad_unfused_call(dY2, W2, aux, G, dZ, dbias, stream) if bplan is not None else None
+    else:
+        fcall = fplan.execute_call(X, W, b, Y, fwd_aux, stream)
+        bcall = bplan.drelu_bgrad_call(dY2, W2, aux, dZ, dbias, stream) if bplan is not None else None
+
+    def call(c):
+        rc = c[0](*c[1])
+        if rc != 0:
+            raise RuntimeError(f"library call failed ({rc}): {binding.gemm_epi_last_error()}")
+
     def step(ev):
         ev[0].record(stream)
-        if args.ablation:
-            fplan.gemm_epi_unfused_execute(X, W, b, T1, T2 if fwd_epi != "BIAS" else Y, Y, fwd_aux, stream)
-        else:
-            fplan.gemm_epi_execute(X, W, b, Y, fwd_aux, stream)
+        call(fcall)
         ev[1].record(stream)
-        if bplan is not None:
-            if args.ablation:
-                bplan.drelu_bgrad_unfused_execute(dY2, W2, aux, G, dZ, dbias, stream)
-            else:
-                bplan.drelu_bgrad_execute(dY2, W2, aux, dZ, dbias, stream)
+        if bcall is not None:
+            call(bcall)
         ev[2].record(stream)
 
     def new_events():
         return [torch.cuda.Event(enable_timing=True) for _ in range(3)]
 
-    for _ in range(args.warmup):
-        flush.zero_()
-        step(new_events())
+    def run_steps(evlist):
+        # Steps are queued in chunks behind a short GPU sleep, so that the host
+        # is ahead of the device and the events time the kernels, not the
+        # host's launch latency (the e2e figure includes that).
+        for c0 in range(0, len(evlist), QUEUE_CHUNK):
+            torch.cuda._sleep(QUEUE_SLEEP_CYCLES)
+            for ev in evlist[c0:c0 + QUEUE_CHUNK]:
+                flush.zero_()
+                step(ev)
+
+    run_steps([new_events() for _ in range(args.warmup)])
     torch.cuda.synchronize(dev)
     for p in (fplan, bplan):
         if p is not None and p.status() != 0:
@@ -225,9 +242,7 @@ def run_ours(args, w: synth.Workload, rank: int, world: int, dev: torch.device):
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
     wall0 = time.time()
-    for i in range(args.steps):
-        flush.zero_()
-        step(evs[i])
+    run_steps(evs)
     torch.cuda.synchronize(dev)
     wall1 = time.time()
     if world > 1:
@@ -247,17 +262,21 @@ def run_ours(args, w: synth.Workload, rank: int, world: int, dev: torch.device):
 
     alg = algorithmic(w, fwd_epi, bplan is not None)
     flops_step = sum(v["flops"] for v in alg.values())
-    launches_per_step = 1 + (2 if bplan is not None else 0)
-    if args.ablation:
+    # our kernels per step, as the plans report them (the L2 flush between
+    # steps is torch's and sits outside the timed events)
+    launches_per_step = fplan.info()["launches"] + (bplan.info()["launches"] if bplan is not None else 0)
+    if args.ablation:  # GEMM + bias + ReLU kernels; GEMM + mask + two column-sum kernels
         launches_per_step = (2 if fwd_epi == "BIAS" else 3) + (4 if bplan is not None else 0)
 
     # e2e: host buffers (pinned), H2D of the step's inputs, both calls, D2H of every output
     e2e = run_e2e(args, w, fwd_epi, fplan, bplan, inp, dev, stream) if not args.ablation else None
 
+    kernel = fplan.info()["kernel"]
     fplan.free()
     if bplan is not None:
         bplan.free()
     return {"step_ms": step_ms, "fwd_ms": fwd_avg, "bwd_ms": bwd_avg, "alg": alg, "flops_step": flops_step,
+            "kernel": kernel,
             "launches": launches_per_step * args.steps, "clocks": clocks, "e2e": e2e,
             "wall_s": wall1 - wall0}
 
@@ -453,10 +472,19 @@ def main():
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak}
     else:
         achieved = alg[part]["flops"] / (part_ms / 1e3) / 1e12
-        peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))  # fp16 dense = bf16 dense
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak}
-    roof["kernel"] = f"{part} ({'tile_kernel ' + (fwd_epi if part == 'fwd' else 'DRELU_BGRAD + dbias finish')})"
-    roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json burst)" if peak_src == "measured" else "fallback"
+        # fp16 dense peak = bf16 dense peak. The burst figure applies to a kernel
+        # timed alone; when the power cap engaged during the timed region the
+        # kernel ran as a sustained load, so the sustained figure applies.
+        burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+        capped = bool(res["clocks"]) and "sw_power_cap" in (res["clocks"].get("reasons") or [])
+        peak = sustained if capped else burst
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "frac_of_burst": achieved / burst, "peak_kind": "sustained (sw_power_cap active)" if capped else "burst"}
+    kname = ("skinny_kernel" if res["kernel"] == 1 else "tile_kernel")
+    roof["kernel"] = f"{part}: {kname} " + (fwd_epi if part == "fwd" else "DRELU_BGRAD" +
+                                              (" + dbias finish" if res["kernel"] == 0 else ""))
+    roof["peak_source"] = "measured (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
     roof["traffic"] = measured_traffic(w, part)
     # roofline time of the whole step: slower of FLOPs at the tensor peak and bytes at HBM
     t_roof = sum(max(v["flops"] / (float(peaks.get("bf16_tflops", 1590.0)) * 1e12),

@@ -218,6 +218,35 @@ class Plan:
                 _ptr(dZ, (T, N), dt, "dZ"), _ptr(dbias, (N,), torch.float32, "dbias"))
         _check(lib().drelu_bgrad_unfused_execute(self.handle, *args, _stream_ptr(stream)))
 
+    # prebuilt calls: (fn, args) so that fn(*args) enqueues the C call with no
+    # per-call argument checking (for tight launch loops; check rc yourself)
+    def execute_call(self, X, W, bias, Y, aux=None, stream=None):
+        T, N, K, dt = self.T, self.N, self.K, self.dtype
+        args = (self.handle, _ptr(X, (T, K), dt, "X"), _ptr(W, (K, N), dt, "W"), _ptr(bias, (N,), dt, "bias"),
+                _ptr(Y, (T, N), dt, "Y"), _ptr(aux, (T, self.aux_words), torch.int32, "aux"), _stream_ptr(stream))
+        return lib().gemm_epi_execute, args
+
+    def drelu_bgrad_call(self, dY2, W2, aux, dZ, dbias, stream=None):
+        T, N, K, dt = self.T, self.N, self.K, self.dtype
+        args = (self.handle, _ptr(dY2, (T, K), dt, "dY2"), _ptr(W2, (K, N), dt, "W2"),
+                _ptr(aux, (T, self.aux_words), torch.int32, "aux"), _ptr(dZ, (T, N), dt, "dZ"),
+                _ptr(dbias, (N,), torch.float32, "dbias"), _stream_ptr(stream))
+        return lib().drelu_bgrad_execute, args
+
+    def unfused_call(self, X, W, bias, T1, T2, Y, aux=None, stream=None):
+        T, N, K, dt = self.T, self.N, self.K, self.dtype
+        args = (self.handle, _ptr(X, (T, K), dt, "X"), _ptr(W, (K, N), dt, "W"), _ptr(bias, (N,), dt, "bias"),
+                _ptr(T1, (T, N), dt, "T1"), _ptr(T2, (T, N), dt, "T2"), _ptr(Y, (T, N), dt, "Y"),
+                _ptr(aux, (T, self.aux_words), torch.int32, "aux"), _stream_ptr(stream))
+        return lib().gemm_epi_unfused_execute, args
+
+    def drelu_bgrad_unfused_call(self, dY2, W2, aux, G, dZ, dbias, stream=None):
+        T, N, K, dt = self.T, self.N, self.K, self.dtype
+        args = (self.handle, _ptr(dY2, (T, K), dt, "dY2"), _ptr(W2, (K, N), dt, "W2"),
+                _ptr(aux, (T, self.aux_words), torch.int32, "aux"), _ptr(G, (T, N), dt, "G"),
+                _ptr(dZ, (T, N), dt, "dZ"), _ptr(dbias, (N,), torch.float32, "dbias"), _stream_ptr(stream))
+        return lib().drelu_bgrad_unfused_execute, args
+
     # conveniences that allocate their outputs (allocation happens in torch,
     # outside the library; the library call itself allocates nothing)
     def forward(self, X, W, bias, stream=None):

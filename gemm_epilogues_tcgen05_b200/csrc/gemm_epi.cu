@@ -14,6 +14,7 @@
 
 #include "../../include/gemm_epi.h"
 #include "aux_kernels.cuh"
+#include "skinny_kernel.cuh"
 #include "tile_kernel.cuh"
 
 namespace {
@@ -117,13 +118,60 @@ TileCfg tile_cfg(int BN, int epi, bool bf16) {
 
 int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
 
+using SkinnyKernelFn = void (*)(CUtensorMap, CUtensorMap, ge::SkinnyParams);
+
+template <int TP, bool BF>
+SkinnyKernelFn pick_skinny_epi(int epi) {
+  switch (epi) {
+    case ge::EPI_BIAS: return ge::skinny_kernel<TP, ge::EPI_BIAS, BF>;
+    case ge::EPI_RELU_BIAS: return ge::skinny_kernel<TP, ge::EPI_RELU_BIAS, BF>;
+    case ge::EPI_RELU_AUX_BIAS: return ge::skinny_kernel<TP, ge::EPI_RELU_AUX_BIAS, BF>;
+    default: return ge::skinny_kernel<TP, ge::EPI_DRELU_BGRAD, BF>;
+  }
+}
+
+struct SkinnyCfg {
+  int TP = 16;
+  SkinnyKernelFn fn = nullptr;
+  uint32_t smem = 0;
+  int stages = 0;
+};
+
+template <int TP>
+SkinnyCfg skinny_cfg_tp(int epi, bool bf16) {
+  SkinnyCfg c;
+  c.TP = TP;
+  c.fn = bf16 ? pick_skinny_epi<TP, true>(epi) : pick_skinny_epi<TP, false>(epi);
+  c.smem = ge::SkinnySmem<TP>::BYTES;
+  c.stages = ge::SkinnySmem<TP>::STAGES;
+  return c;
+}
+
+SkinnyCfg skinny_cfg(int64_t T, int epi, bool bf16) {
+  if (T <= 16) return skinny_cfg_tp<16>(epi, bf16);
+  if (T <= 32) return skinny_cfg_tp<32>(epi, bf16);
+  if (T <= 64) return skinny_cfg_tp<64>(epi, bf16);
+  if (T <= 128) return skinny_cfg_tp<128>(epi, bf16);
+  return skinny_cfg_tp<256>(epi, bf16);
+}
+
+// Few-row problems (T <= 256) use the swap-AB stream-K kernel unless
+// GEMM_EPI_FORCE_KERNEL says otherwise ("tile" or "skinny").
+bool use_skinny(int64_t T) {
+  if (const char* f = getenv("GEMM_EPI_FORCE_KERNEL")) {
+    if (!strcmp(f, "tile")) return false;
+    if (!strcmp(f, "skinny")) return T <= 256;
+  }
+  return T <= 256;
+}
+
 }  // namespace
 
 struct gemm_epi_plan_s {
   int64_t T, N, K;
   int dtype, epilog;
   int device, num_sms;
-  int m_tiles, n_tiles, k_blocks, num_tiles, aux_words, grid;
+  int m_tiles, n_tiles, k_blocks, num_tiles, aux_words, grid, group_m;
   TileCfg cfg;       // fused kernel
   TileCfg cfg_store; // unfused GEMM (plain store)
   float* partials = nullptr;  // DRELU_BGRAD: m_tiles x N
@@ -135,6 +183,15 @@ struct gemm_epi_plan_s {
   const void* a_ptr = nullptr;
   const void* b_ptr = nullptr;
   CUtensorMap tmA, tmB;
+  // few-row kernel (kernel == 1)
+  int kernel = 0;
+  SkinnyCfg sk;
+  int sk_grid = 0, sk_kbt = 0, sk_total = 0, sk_max_segs = 1, sk_prefetch = 0;
+  float* sk_partials = nullptr;
+  int* sk_tickets = nullptr;
+  size_t sk_bytes = 0;
+  const void* xs_ptr = nullptr;
+  CUtensorMap tmXs;  // the row operand with a TP-row box
 };
 
 namespace {
@@ -151,6 +208,8 @@ int take_status(gemm_epi_plan_s* p) {
   const int v = *s;
   if (v != 0) {
     *s = 0;
+    // an interrupted launch may have left split-tile tickets counted
+    if (p->sk_tickets) cudaMemset(p->sk_tickets, 0, sizeof(int) * (size_t)ceil_div(p->N, 128));
     return fail(GEMM_EPI_ERR_TIMEOUT, "a kernel of this plan gave up waiting (watchdog code 0x%x)", v);
   }
   return GEMM_EPI_OK;
@@ -180,6 +239,7 @@ ge::TileParams base_params(const gemm_epi_plan_s* p) {
   k.k_blocks = p->k_blocks;
   k.num_tiles = p->num_tiles;
   k.aux_words = p->aux_words;
+  k.group_m = p->group_m;
   k.status = p->status_dev;
   k.timeout_ns = p->timeout_ns;
   return k;
@@ -189,6 +249,53 @@ int launch_tile(const gemm_epi_plan_s* p, const TileCfg& c, const ge::TileParams
   c.fn<<<p->grid, ge::kThreads, c.smem, s>>>(p->tmA, p->tmB, k);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "tile kernel launch");
+  return GEMM_EPI_OK;
+}
+
+// Raster group: when the row operand (T x K) fits comfortably in L2, one
+// group spans every row tile, so each column block of W is streamed from
+// HBM once while X stays resident; otherwise 16 row tiles per group.
+int choose_group_m(int64_t T, int64_t K, int m_tiles) {
+  const int64_t a_bytes = T * K * 2;
+  return a_bytes <= (int64_t)40 << 20 ? m_tiles : (m_tiles < 16 ? m_tiles : 16);
+}
+
+int prepare_skinny_maps(gemm_epi_plan_s* p, const void* A, const void* B) {
+  if (A != p->xs_ptr) {
+    int rc = encode_2d(&p->tmXs, A, (uint64_t)p->K, (uint64_t)p->T, ge::kBK, (uint32_t)p->sk.TP, "the row operand");
+    if (rc) return rc;
+    p->xs_ptr = A;
+  }
+  if (B != p->b_ptr) {
+    int rc = encode_2d(&p->tmB, B, (uint64_t)p->N, (uint64_t)p->K, 64, ge::kBK, "the weight operand");
+    if (rc) return rc;
+    p->b_ptr = B;
+  }
+  return GEMM_EPI_OK;
+}
+
+ge::SkinnyParams skinny_params(const gemm_epi_plan_s* p) {
+  ge::SkinnyParams k{};
+  k.T = (int32_t)p->T;
+  k.N = (int32_t)p->N;
+  k.K = (int32_t)p->K;
+  k.n_tiles = ceil_div(p->N, 128);
+  k.kbt = p->sk_kbt;
+  k.total_kb = p->sk_total;
+  k.aux_words = p->aux_words;
+  k.max_segs = p->sk_max_segs;
+  k.prefetch = p->sk_prefetch;
+  k.partials = p->sk_partials;
+  k.tickets = p->sk_tickets;
+  k.status = p->status_dev;
+  k.timeout_ns = p->timeout_ns;
+  return k;
+}
+
+int launch_skinny(const gemm_epi_plan_s* p, const ge::SkinnyParams& k, cudaStream_t s) {
+  p->sk.fn<<<p->sk_grid, ge::kThreads, p->sk.smem, s>>>(p->tmB, p->tmXs, k);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "few-row kernel launch");
   return GEMM_EPI_OK;
 }
 
@@ -261,6 +368,7 @@ gemm_epi_plan_t gemm_epi_plan(int64_t T, int64_t N, int64_t K, gemm_epi_dtype dt
   p->k_blocks = ceil_div(K, ge::kBK);
   p->num_tiles = p->m_tiles * p->n_tiles;
   p->aux_words = ceil_div(N, 32);
+  p->group_m = choose_group_m(T, K, p->m_tiles);
   p->grid = p->num_tiles < sms ? p->num_tiles : sms;
   p->timeout_ns = 2000000000ull;  // 2 s per wait
   if (const char* t = getenv("GEMM_EPI_WAIT_TIMEOUT_MS")) {
@@ -269,6 +377,8 @@ gemm_epi_plan_t gemm_epi_plan(int64_t T, int64_t N, int64_t K, gemm_epi_dtype dt
   }
 
   auto cleanup = [&](int rc) {
+    if (p->sk_partials) cudaFree(p->sk_partials);
+    if (p->sk_tickets) cudaFree(p->sk_tickets);
     if (p->partials) cudaFree(p->partials);
     if (p->status_host) cudaFreeHost(p->status_host);
     delete p;
@@ -279,6 +389,48 @@ gemm_epi_plan_t gemm_epi_plan(int64_t T, int64_t N, int64_t K, gemm_epi_dtype dt
   for (const TileCfg* c : {&p->cfg, &p->cfg_store}) {
     e = cudaFuncSetAttribute(c->fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)c->smem);
     if (e != cudaSuccess) return cleanup(cuda_fail(e, "cudaFuncSetAttribute(max dynamic shared memory)"));
+  }
+  if (use_skinny(T)) {
+    p->kernel = 1;
+    p->sk = skinny_cfg(T, (int)epilog, bf16);
+    const int n_tiles = ceil_div(N, 128);
+    p->sk_kbt = ceil_div(K, ge::kBK);
+    p->sk_total = n_tiles * p->sk_kbt;
+    // every CTA gets at least 8 k-blocks, so a tile is shared by few CTAs
+    // With at least half as many feature tiles as SMs (and no more than
+    // SMs), every CTA takes whole tiles: no split-tile partials or fixups,
+    // whose dependent round trips cost more than the idle SMs would give.
+    // Otherwise stream-K over up to one CTA per SM, at least 8 k-blocks each.
+    if (n_tiles * 2 >= sms && n_tiles <= sms) {
+      p->sk_grid = n_tiles;
+    } else {
+      int g = p->sk_total / 8;
+      g = g < 1 ? 1 : g;
+      p->sk_grid = g < sms ? g : sms;
+    }
+    if (const char* f = getenv("GEMM_EPI_SKINNY_GRID")) {  // tuning override
+      const int v = atoi(f);
+      if (v >= 1 && v <= p->sk_total) p->sk_grid = v;
+    }
+    if (const char* f = getenv("GEMM_EPI_SKINNY_PREFETCH")) p->sk_prefetch = atoi(f) > 0 ? atoi(f) : 0;
+    p->sk_max_segs = 1;
+    for (int t = 0; t < n_tiles; ++t) {
+      const int64_t first = ge::skinny_owner((int64_t)t * p->sk_kbt, p->sk_grid, p->sk_total);
+      const int64_t last = ge::skinny_owner((int64_t)(t + 1) * p->sk_kbt - 1, p->sk_grid, p->sk_total);
+      if (last - first + 1 > p->sk_max_segs) p->sk_max_segs = (int)(last - first + 1);
+    }
+    e = cudaFuncSetAttribute(p->sk.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p->sk.smem);
+    if (e != cudaSuccess) return cleanup(cuda_fail(e, "cudaFuncSetAttribute(max dynamic shared memory)"));
+    if (p->sk_max_segs > 1) {
+      p->sk_bytes = (size_t)n_tiles * p->sk_max_segs * p->sk.TP * 128 * sizeof(float);
+      e = cudaMalloc((void**)&p->sk_partials, p->sk_bytes);
+      if (e != cudaSuccess) return cleanup(cuda_fail(e, "cudaMalloc(split-tile partials)"));
+      e = cudaMalloc((void**)&p->sk_tickets, sizeof(int) * (size_t)n_tiles);
+      if (e != cudaSuccess) return cleanup(cuda_fail(e, "cudaMalloc(tickets)"));
+      e = cudaMemset(p->sk_tickets, 0, sizeof(int) * (size_t)n_tiles);
+      if (e != cudaSuccess) return cleanup(cuda_fail(e, "cudaMemset(tickets)"));
+      p->sk_bytes += sizeof(int) * (size_t)n_tiles;
+    }
   }
   e = cudaHostAlloc((void**)&p->status_host, sizeof(int), cudaHostAllocMapped);
   if (e != cudaSuccess) return cleanup(cuda_fail(e, "cudaHostAlloc(status word)"));
@@ -311,6 +463,8 @@ void gemm_epi_free(gemm_epi_plan_t plan) {
     }
   }
   if (plan->partials) cudaFree(plan->partials);
+  if (plan->sk_partials) cudaFree(plan->sk_partials);
+  if (plan->sk_tickets) cudaFree(plan->sk_tickets);
   if (plan->status_host) cudaFreeHost(plan->status_host);
   delete plan;
 }
@@ -326,16 +480,27 @@ int gemm_epi_query(gemm_epi_plan_t plan, gemm_epi_info* info) {
   info->K = p->K;
   info->dtype = p->dtype;
   info->epilog = p->epilog;
-  info->kernel = 0;
-  info->tile_m = ge::kBM;
-  info->tile_n = p->cfg.BN;
-  info->tile_k = ge::kBK;
-  info->stages = p->cfg.stages;
-  info->split_k = 1;
-  info->grid = p->grid;
-  info->launches = p->epilog == GEMM_EPI_DRELU_BGRAD ? 2 : 1;
+  info->kernel = p->kernel;
   info->num_sms = p->num_sms;
-  info->workspace_bytes = p->epilog == GEMM_EPI_DRELU_BGRAD ? p->partial_bytes : 0;
+  if (p->kernel == 1) {
+    info->tile_m = 128;  // features per tile (the MMA's M)
+    info->tile_n = p->sk.TP;  // padded rows (the MMA's N)
+    info->tile_k = ge::kBK;
+    info->stages = p->sk.stages;
+    info->split_k = p->sk_max_segs;
+    info->grid = p->sk_grid;
+    info->launches = 1;
+    info->workspace_bytes = p->sk_bytes + (p->epilog == GEMM_EPI_DRELU_BGRAD ? p->partial_bytes : 0);
+  } else {
+    info->tile_m = ge::kBM;
+    info->tile_n = p->cfg.BN;
+    info->tile_k = ge::kBK;
+    info->stages = p->cfg.stages;
+    info->split_k = 1;
+    info->grid = p->grid;
+    info->launches = p->epilog == GEMM_EPI_DRELU_BGRAD ? 2 : 1;
+    info->workspace_bytes = p->epilog == GEMM_EPI_DRELU_BGRAD ? p->partial_bytes : 0;
+  }
   return GEMM_EPI_OK;
 }
 
@@ -359,6 +524,15 @@ int gemm_epi_execute(gemm_epi_plan_t plan, const void* X, const void* W, const v
     return fail(GEMM_EPI_ERR_MISALIGNED, "gemm_epi_execute: X, W, Y need 16-byte, bias 2-byte, aux 4-byte alignment");
   int rc = take_status(p);
   if (rc) return rc;
+  if (p->kernel == 1) {
+    rc = prepare_skinny_maps(p, X, W);
+    if (rc) return rc;
+    ge::SkinnyParams k = skinny_params(p);
+    k.bias = bias;
+    k.out = Y;
+    k.aux_out = aux;
+    return launch_skinny(p, k, stream);
+  }
   rc = prepare_maps(p, X, W);
   if (rc) return rc;
   ge::TileParams k = base_params(p);
@@ -381,6 +555,15 @@ int drelu_bgrad_execute(gemm_epi_plan_t plan, const void* dY2, const void* W2, c
                 "drelu_bgrad_execute: dY2, W2, dZ need 16-byte, aux and dbias 4-byte alignment");
   int rc = take_status(p);
   if (rc) return rc;
+  if (p->kernel == 1) {
+    rc = prepare_skinny_maps(p, dY2, W2);
+    if (rc) return rc;
+    ge::SkinnyParams k = skinny_params(p);
+    k.out = dZ;
+    k.aux_in = aux;
+    k.dbias = dbias;
+    return launch_skinny(p, k, stream);
+  }
   rc = prepare_maps(p, dY2, W2);
   if (rc) return rc;
   ge::TileParams k = base_params(p);
@@ -605,6 +788,7 @@ extern "C" int drelu_bgrad_execute_noalloc(int64_t T, int64_t N, int64_t K, gemm
   k.k_blocks = ceil_div(K, ge::kBK);
   k.num_tiles = k.m_tiles * k.n_tiles;
   k.aux_words = ceil_div(N, 32);
+  k.group_m = choose_group_m(T, K, k.m_tiles);
   k.out = dZ;
   k.aux_in = aux;
   k.partials = partials;

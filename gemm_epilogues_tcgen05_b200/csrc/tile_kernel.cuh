@@ -32,6 +32,7 @@ struct TileParams {
   int32_t T, N, K;
   int32_t m_tiles, n_tiles, k_blocks, num_tiles;
   int32_t aux_words;        // ceil(N / 32)
+  int32_t group_m;          // row tiles per raster group (see tile_coords)
   const void* bias;         // N values of the 16-bit type (forward)
   void* out;                // T x N, 16-bit: Y, dZ, or the unfused intermediate
   uint32_t* aux_out;        // RELU_AUX_BIAS mask words
@@ -44,7 +45,6 @@ struct TileParams {
 constexpr int kBM = 128;
 constexpr int kBK = 64;
 constexpr int kThreads = 192;
-constexpr int kGroupM = 8;
 
 template <int BN, int STAGES>
 struct TileSmem {
@@ -62,11 +62,15 @@ struct TileSmem {
   static constexpr uint32_t BYTES = END + 1024;               // + alignment slack
 };
 
-__device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, int& mb, int& nb) {
-  const int per_group = kGroupM * n_tiles;
+// Tile order: groups of `group_m` row tiles; inside a group the row tile
+// varies fastest, then the column tile. Consecutive CTAs therefore share
+// W's column block and the group's rows of X stay in L2 while the group
+// sweeps all column blocks.
+__device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, int group_m, int& mb, int& nb) {
+  const int per_group = group_m * n_tiles;
   const int g = tile / per_group;
-  const int first_m = g * kGroupM;
-  const int gsize = min(m_tiles - first_m, kGroupM);
+  const int first_m = g * group_m;
+  const int gsize = min(m_tiles - first_m, group_m);
   const int r = tile - g * per_group;
   mb = first_m + r % gsize;
   nb = r / gsize;
@@ -196,7 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
         int mb, nb;
-        tile_coords(tile, p.m_tiles, p.n_tiles, mb, nb);
+        tile_coords(tile, p.m_tiles, p.n_tiles, p.group_m, mb, nb);
         const int m0 = mb * kBM, n0 = nb * BN;
         for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
           const uint32_t s = it % STAGES;
@@ -267,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tcount) {
       int mb, nb;
-      tile_coords(tile, p.m_tiles, p.n_tiles, mb, nb);
+      tile_coords(tile, p.m_tiles, p.n_tiles, p.group_m, mb, nb);
       const int m0 = mb * kBM, n0 = nb * BN;
       const uint32_t buf = tcount & 1u;
       const uint32_t tph = (tcount >> 1) & 1u;
@@ -287,7 +291,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int row = m0 + static_cast<int>(ew * 32 + lane);
         const bool row_ok = row < p.T;
         const uint32_t tbase = tmem_base + ((ew * 32u) << 16) + buf * BN;
-#pragma unroll 1
+        // DRELU: this row's mask words for the whole tile, loaded before any
+        // store (a load after a store could not be moved above it)
+        uint32_t mwords[EPI == EPI_DRELU_BGRAD ? BN / 32 : 1];
+        if constexpr (EPI == EPI_DRELU_BGRAD) {
+#pragma unroll
+          for (int c = 0; c < BN / 32; ++c) {
+            const int nc0 = n0 + c * 32;
+            mwords[c] = (row_ok && nc0 < p.N) ? __ldg(p.aux_in + static_cast<int64_t>(row) * p.aux_words + (nc0 >> 5)) : 0u;
+          }
+        }
+#pragma unroll
         for (int c = 0; c < BN / 32; ++c) {
           const int nc0 = n0 + c * 32;
           if (nc0 >= p.N) break;  // warp-uniform
@@ -298,7 +312,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
           if constexpr (EPI == EPI_DRELU_BGRAD) {
-            const uint32_t m = row_ok ? __ldg(p.aux_in + static_cast<int64_t>(row) * p.aux_words + (nc0 >> 5)) : 0u;
+            const uint32_t m = mwords[c];
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = ((m >> j) & 1u) ? v[j] : 0.f;
           } else if constexpr (EPI != EPI_STORE) {

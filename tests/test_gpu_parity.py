@@ -14,7 +14,30 @@ pytestmark = pytest.mark.gpu
 
 DT = {"fp16": torch.float16, "bf16": torch.bfloat16}
 SHAPES = [(1, 8, 8), (5, 40, 24), (130, 72, 136), (200, 264, 200), (257, 520, 328), (384, 512, 512)]
+# few-row shapes whose feature tiles are split over several CTAs (stream-K
+# segments), with ragged K and N, and one where every CTA owns whole tiles
+SKINNY_SHAPES = [(16, 1032, 2048), (100, 264, 1000), (256, 4104, 520), (40, 2056, 64), (1, 11008, 4096)]
 FWD_EPILOGS = ["BIAS", "RELU_BIAS", "RELU_AUX_BIAS"]
+# kernel variants: the tile kernel at each width, and the few-row kernel
+VARIANTS = ["tile64", "tile128", "tile256", "skinny"]
+
+
+def _force(monkeypatch, variant):
+    if variant == "skinny":
+        monkeypatch.setenv("GEMM_EPI_FORCE_KERNEL", "skinny")
+        monkeypatch.delenv("GEMM_EPI_FORCE_BN", raising=False)
+    else:
+        monkeypatch.setenv("GEMM_EPI_FORCE_KERNEL", "tile")
+        monkeypatch.setenv("GEMM_EPI_FORCE_BN", variant[4:])
+
+
+def _expect_variant(info, variant, T):
+    if variant == "skinny" and T <= 256:
+        assert info["kernel"] == 1
+    else:
+        assert info["kernel"] == 0
+        if variant != "skinny":
+            assert info["tile_n"] == int(variant[4:])
 
 
 @pytest.fixture(autouse=True)
@@ -23,32 +46,52 @@ def _need_gpu():
         pytest.skip("no CUDA device")
 
 
-@pytest.mark.parametrize("bn", [64, 128, 256])
+@pytest.mark.parametrize("variant", VARIANTS)
 @pytest.mark.parametrize("dtype", ["fp16", "bf16"])
 @pytest.mark.parametrize("T,N,K", SHAPES)
-def test_forward_all_epilogs(monkeypatch, T, N, K, dtype, bn):
-    monkeypatch.setenv("GEMM_EPI_FORCE_BN", str(bn))
+def test_forward_all_epilogs(monkeypatch, T, N, K, dtype, variant):
+    _force(monkeypatch, variant)
     inp = synth.make_shape_inputs(T, N, K, dtype, seed=T * 7 + N + K)
     for ep in FWD_EPILOGS:
         gpu = run_forward(inp, ep, DT[dtype])
-        assert gpu["info"]["tile_n"] == bn
+        _expect_variant(gpu["info"], variant, T)
         check_forward(inp, ep, DT[dtype], gpu)
 
 
-@pytest.mark.parametrize("bn", [64, 128, 256])
+@pytest.mark.parametrize("variant", VARIANTS)
 @pytest.mark.parametrize("dtype", ["fp16", "bf16"])
 @pytest.mark.parametrize("T,N,K", SHAPES)
-def test_backward_drelu_bgrad(monkeypatch, T, N, K, dtype, bn):
-    monkeypatch.setenv("GEMM_EPI_FORCE_BN", str(bn))
+def test_backward_drelu_bgrad(monkeypatch, T, N, K, dtype, variant):
+    _force(monkeypatch, variant)
     D2 = max(8, (K // 2) // 8 * 8)
     inp = synth.make_shape_inputs(T, N, K, dtype, seed=T * 5 + N + K, D2=D2)
     fwd = run_forward(inp, "RELU_AUX_BIAS", DT[dtype])
     gpu = run_backward(inp, fwd["aux"], DT[dtype])
+    _expect_variant(gpu["info"], variant, T)
     check_backward(inp, fwd["aux"], DT[dtype], gpu)
 
 
 @pytest.mark.parametrize("dtype", ["fp16", "bf16"])
-@pytest.mark.parametrize("T,N,K,D2", [(130, 72, 64, 40), (257, 520, 128, 96), (64, 8, 8, 8)])
+@pytest.mark.parametrize("T,N,K", SKINNY_SHAPES)
+def test_skinny_split_tiles(monkeypatch, T, N, K, dtype):
+    """Few-row kernel on shapes whose tiles are shared by several CTAs."""
+    monkeypatch.delenv("GEMM_EPI_FORCE_KERNEL", raising=False)
+    D2 = K
+    inp = synth.make_shape_inputs(T, N, K, dtype, seed=T + N + K, D2=D2)
+    for ep in FWD_EPILOGS:
+        gpu = run_forward(inp, ep, DT[dtype])
+        assert gpu["info"]["kernel"] == 1
+        check_forward(inp, ep, DT[dtype], gpu)
+    fwd = run_forward(inp, "RELU_AUX_BIAS", DT[dtype])
+    outs = run_backward(inp, fwd["aux"], DT[dtype], repeats=2)  # tickets reset between launches
+    for gpu in outs:
+        assert gpu["info"]["kernel"] == 1
+        check_backward(inp, fwd["aux"], DT[dtype], gpu)
+    assert torch.equal(outs[0]["dbias"], outs[1]["dbias"])
+
+
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+@pytest.mark.parametrize("T,N,K,D2", [(130, 72, 64, 40), (257, 520, 128, 96), (64, 8, 8, 8), (16, 1032, 1024, 512)])
 def test_integer_inputs_bit_exact(T, N, K, D2, dtype):
     """Integer inputs: every sum is exact in fp32, so Y, aux, dZ and dbias
     must equal the exact result rounded once (pins ties Z == 0, the mask
