@@ -15,6 +15,7 @@
 #include "../../include/gemm_epi.h"
 #include "aux_kernels.cuh"
 #include "skinny_kernel.cuh"
+#include "tile2_kernel.cuh"
 #include "tile_kernel.cuh"
 
 namespace {
@@ -94,7 +95,29 @@ struct TileCfg {
   int BN = 256, stages = 4;
   TileKernelFn fn = nullptr;
   uint32_t smem = 0;
+  bool pair = false;  // CTA-pair kernel, launched in clusters of 2
 };
+
+template <bool BF>
+TileKernelFn pick_pair_epi(int epi) {
+  switch (epi) {
+    case ge::EPI_BIAS: return ge::tile2_kernel<256, 6, ge::EPI_BIAS, BF>;
+    case ge::EPI_RELU_BIAS: return ge::tile2_kernel<256, 6, ge::EPI_RELU_BIAS, BF>;
+    case ge::EPI_RELU_AUX_BIAS: return ge::tile2_kernel<256, 6, ge::EPI_RELU_AUX_BIAS, BF>;
+    case ge::EPI_DRELU_BGRAD: return ge::tile2_kernel<256, 6, ge::EPI_DRELU_BGRAD, BF>;
+    default: return ge::tile2_kernel<256, 6, ge::EPI_STORE, BF>;
+  }
+}
+
+TileCfg pair_cfg(int epi, bool bf16) {
+  TileCfg c;
+  c.BN = 256;
+  c.stages = 6;
+  c.smem = ge::Tile2Smem<256, 6>::BYTES;
+  c.fn = bf16 ? pick_pair_epi<true>(epi) : pick_pair_epi<false>(epi);
+  c.pair = true;
+  return c;
+}
 
 TileCfg tile_cfg(int BN, int epi, bool bf16) {
   TileCfg c;
@@ -157,6 +180,17 @@ SkinnyCfg skinny_cfg(int64_t T, int epi, bool bf16) {
 
 // Few-row problems (T <= 256) use the swap-AB stream-K kernel unless
 // GEMM_EPI_FORCE_KERNEL says otherwise ("tile" or "skinny").
+// CTA pairs (256 x 256 tiles) when there is at least one full wave of pair
+// tiles; GEMM_EPI_FORCE_KERNEL=tile / pair overrides.
+bool use_pair(int64_t T, int64_t N, int num_sms) {
+  const int64_t pair_tiles = ((T + 255) / 256) * ((N + 255) / 256);
+  if (const char* f = getenv("GEMM_EPI_FORCE_KERNEL")) {
+    if (!strcmp(f, "tile")) return false;
+    if (!strcmp(f, "pair")) return T > 256;
+  }
+  return T > 256 && pair_tiles >= num_sms / 2;
+}
+
 bool use_skinny(int64_t T) {
   if (const char* f = getenv("GEMM_EPI_FORCE_KERNEL")) {
     if (!strcmp(f, "tile")) return false;
@@ -246,18 +280,44 @@ ge::TileParams base_params(const gemm_epi_plan_s* p) {
 }
 
 int launch_tile(const gemm_epi_plan_s* p, const TileCfg& c, const ge::TileParams& k, cudaStream_t s) {
+  if (c.pair) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)p->grid, 1, 1);
+    cfg.blockDim = dim3(ge::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = c.smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, c.fn, p->tmA, p->tmB, k);
+    if (e != cudaSuccess) return cuda_fail(e, "pair kernel launch");
+    return GEMM_EPI_OK;
+  }
   c.fn<<<p->grid, ge::kThreads, c.smem, s>>>(p->tmA, p->tmB, k);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "tile kernel launch");
   return GEMM_EPI_OK;
 }
 
-// Raster group: when the row operand (T x K) fits comfortably in L2, one
-// group spans every row tile, so each column block of W is streamed from
-// HBM once while X stays resident; otherwise 16 row tiles per group.
-int choose_group_m(int64_t T, int64_t K, int m_tiles) {
-  const int64_t a_bytes = T * K * 2;
-  return a_bytes <= (int64_t)40 << 20 ? m_tiles : (m_tiles < 16 ? m_tiles : 16);
+// Raster group (in row tiles of `tile_rows`): the group's block of X --
+// group rows x K x 2 bytes -- is kept to about 48 MB, a little under half of
+// the 126 MB L2, so it stays resident while the group sweeps every column
+// block of W. When all of X fits, one group spans every row tile and each
+// column block of W is streamed from HBM once.
+int choose_group_m(int64_t T, int64_t K, int tile_rows) {
+  const int m_tiles = (int)((T + tile_rows - 1) / tile_rows);
+  const int64_t block = (int64_t)tile_rows * K * 2;
+  int64_t g = ((int64_t)48 << 20) / block;
+  if (const char* f = getenv("GEMM_EPI_GROUP_M")) {  // tuning override
+    const int v = atoi(f);
+    if (v >= 1) g = v;
+  }
+  if (g < 1) g = 1;
+  return g >= m_tiles ? m_tiles : (int)g;
 }
 
 int prepare_skinny_maps(gemm_epi_plan_s* p, const void* A, const void* B) {
@@ -360,16 +420,23 @@ gemm_epi_plan_t gemm_epi_plan(int64_t T, int64_t N, int64_t K, gemm_epi_dtype dt
   p->device = dev;
   p->num_sms = sms;
   const bool bf16 = dtype == GEMM_EPI_BF16;
-  const int bn = choose_bn(T, N, sms);
-  p->cfg = tile_cfg(bn, (int)epilog, bf16);
-  p->cfg_store = tile_cfg(bn, ge::EPI_STORE, bf16);
+  const bool pair = use_pair(T, N, sms);
+  const int bn = pair ? 256 : choose_bn(T, N, sms);
+  p->cfg = pair ? pair_cfg((int)epilog, bf16) : tile_cfg(bn, (int)epilog, bf16);
+  p->cfg_store = pair ? pair_cfg(ge::EPI_STORE, bf16) : tile_cfg(bn, ge::EPI_STORE, bf16);
+  p->kernel = pair ? 2 : 0;
   p->m_tiles = ceil_div(T, ge::kBM);
   p->n_tiles = ceil_div(N, bn);
   p->k_blocks = ceil_div(K, ge::kBK);
   p->num_tiles = p->m_tiles * p->n_tiles;
   p->aux_words = ceil_div(N, 32);
-  p->group_m = choose_group_m(T, K, p->m_tiles);
+  p->group_m = choose_group_m(T, K, pair ? 2 * ge::kBM : ge::kBM);
   p->grid = p->num_tiles < sms ? p->num_tiles : sms;
+  if (pair) {  // one cluster of two CTAs per 256-row x 256-column tile, up to one CTA per SM
+    const int pair_tiles = ceil_div(T, 256) * p->n_tiles;
+    const int pairs = pair_tiles < sms / 2 ? pair_tiles : sms / 2;
+    p->grid = 2 * pairs;
+  }
   p->timeout_ns = 2000000000ull;  // 2 s per wait
   if (const char* t = getenv("GEMM_EPI_WAIT_TIMEOUT_MS")) {
     long long ms = atoll(t);
@@ -492,7 +559,7 @@ int gemm_epi_query(gemm_epi_plan_t plan, gemm_epi_info* info) {
     info->launches = 1;
     info->workspace_bytes = p->sk_bytes + (p->epilog == GEMM_EPI_DRELU_BGRAD ? p->partial_bytes : 0);
   } else {
-    info->tile_m = ge::kBM;
+    info->tile_m = p->kernel == 2 ? 2 * ge::kBM : ge::kBM;
     info->tile_n = p->cfg.BN;
     info->tile_k = ge::kBK;
     info->stages = p->cfg.stages;
@@ -788,7 +855,7 @@ extern "C" int drelu_bgrad_execute_noalloc(int64_t T, int64_t N, int64_t K, gemm
   k.k_blocks = ceil_div(K, ge::kBK);
   k.num_tiles = k.m_tiles * k.n_tiles;
   k.aux_words = ceil_div(N, 32);
-  k.group_m = choose_group_m(T, K, k.m_tiles);
+  k.group_m = choose_group_m(T, K, ge::kBM);
   k.out = dZ;
   k.aux_in = aux;
   k.partials = partials;

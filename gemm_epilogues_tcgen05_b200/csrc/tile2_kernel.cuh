@@ -1,0 +1,216 @@
+// tile2_kernel.cuh -- the CTA-pair (cluster of 2, tcgen05 cta_group::2)
+// variant of the persistent tile kernel, for large problems.
+//
+// A pair computes a 256 x BN output tile with one MMA stream: the leader CTA
+// (rank 0) issues tcgen05.mma.cta_group::2 with M = 256, reading rows 0..127
+// of the X tile and columns 0..BN/2-1 of the W tile from its own shared
+// memory and rows 128..255 / columns BN/2..BN-1 from its peer's (same
+// offsets); each CTA's TMEM receives its 128 rows of the accumulator, all BN
+// columns. Per CTA and k-block that is 16 KB of X and BN/2 x 64 of W instead
+// of the single-CTA kernel's 16 KB + BN x 64, so each SM needs two thirds of
+// the operand traffic per FLOP and the ring can be deeper.
+//
+// Synchronisation across the pair:
+//   full[s]   (leader's) one arrival -- the leader's expect_tx for both CTAs'
+//             bytes -- plus both CTAs' TMA transaction bytes (the peer's loads
+//             name the leader's barrier)
+//   empty[s]  (each CTA's) one arrival from the leader's MMA commit,
+//             multicast to both CTAs
+//   tfull[b]  (each CTA's) the leader's commit after a tile, multicast
+//   tempty[b] (leader's) eight arrivals: four epilogue warps of each CTA,
+//             the peer's through its shared::cluster address
+// No load uses TMA multicast. Every wait is bounded as in the 1-CTA kernel.
+#pragma once
+
+#include "tile_kernel.cuh"
+
+namespace ge {
+
+template <int BN, int STAGES>
+struct Tile2Smem {
+  static constexpr uint32_t A_BYTES = kBM * kBK * 2;          // this CTA's 128 rows x 64 k
+  static constexpr uint32_t B_CHUNK = kBK * 64 * 2;           // 64 k x 64 n
+  static constexpr uint32_t B_BYTES = (BN / 128) * B_CHUNK;   // this CTA's BN/2 columns
+  static constexpr uint32_t OFF_A = 0;
+  static constexpr uint32_t OFF_B = OFF_A + STAGES * A_BYTES;
+  static constexpr uint32_t OFF_BAR = OFF_B + STAGES * B_BYTES;
+  static constexpr uint32_t N_BARS = 2 * STAGES + 5;
+  static constexpr uint32_t OFF_MISC = OFF_BAR + N_BARS * 8;
+  static constexpr uint32_t OFF_BIAS = (OFF_MISC + 16 + 15) / 16 * 16;
+  static constexpr uint32_t OFF_COLP = OFF_BIAS + 2 * BN * 4;
+  static constexpr uint32_t END = OFF_COLP + 2 * 4 * BN * 4;
+  static constexpr uint32_t BYTES = END + 1024;
+};
+
+template <int BN, int STAGES, int EPI, bool BF16>
+__global__ void __launch_bounds__(kThreads, 1)
+    tile2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                 const TileParams p) {
+  using L = Tile2Smem<BN, STAGES>;
+  static_assert(BN == 128 || BN == 256, "the pair kernel splits BN in 64-column chunks per CTA");
+  constexpr uint32_t TMEM_COLS = 2 * BN;
+  constexpr uint32_t IDESC = idesc_f16(BF16, /*A MN-major*/ false, /*B MN-major*/ true, 2 * kBM, BN);
+  constexpr uint32_t PAIR_TX = 2 * (L::A_BYTES + L::B_BYTES);
+  constexpr uint16_t BOTH = 0x3;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem + L::OFF_A;
+  uint8_t* sB = smem + L::OFF_B;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+  float* bias_s = reinterpret_cast<float*>(smem + L::OFF_BIAS);  // [2][BN]
+  float* colp_s = reinterpret_cast<float*>(smem + L::OFF_COLP);  // [2][4][BN]
+
+  const uint32_t warp = threadIdx.x >> 5;
+  const uint32_t lane = lane_id();
+  const uint32_t rank = cluster_ctarank();  // 0 = leader
+  const int pair = static_cast<int>(blockIdx.x >> 1);
+  const int npairs = static_cast<int>(gridDim.x >> 1);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 8);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();  // both CTAs' barriers exist before either side signals the other
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int m2_tiles = (p.m_tiles + 1) / 2;  // 256-row tiles
+  const int num_tiles = m2_tiles * p.n_tiles;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      const uint32_t full0 = mapa_shared(smem_u32(&full[0]), 0);
+      for (int tile = pair; ok && tile < num_tiles; tile += npairs) {
+        int mb, nb;
+        tile_coords(tile, m2_tiles, p.n_tiles, p.group_m, mb, nb);
+        const int m0 = mb * 2 * kBM + static_cast<int>(rank) * kBM;
+        const int nh0 = nb * BN + static_cast<int>(rank) * (BN / 2);
+        for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+          const uint32_t s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1u;
+          if (!wait_bounded(&empty[s], ph ^ 1u, p, abort_flag, 1)) {
+            ok = false;
+            break;
+          }
+          if (rank == 0) mbar_arrive_expect_tx(&full[s], PAIR_TX);
+          const uint32_t fbar = full0 + s * 8;  // the leader's full[s]
+          tma_load_2d_pair(sA + s * L::A_BYTES, &tmA, fbar, kb * kBK, m0);
+#pragma unroll
+          for (int j = 0; j < BN / 128; ++j)
+            tma_load_2d_pair(sB + s * L::B_BYTES + j * L::B_CHUNK, &tmB, fbar, nh0 + j * 64, kb * kBK);
+        }
+      }
+      // the last fills have landed once the MMA has released them
+      const uint32_t inflight = it < STAGES ? it : STAGES;
+      for (uint32_t i = it - inflight; i < it; ++i)
+        wait_bounded(&empty[i % STAGES], ((i / STAGES) & 1u), p, abort_flag, 2, /*honour_abort=*/false);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA
+    if (lane == 0) {
+      if (rank == 0) {
+        uint32_t it = 0, tcount = 0;
+        bool ok = true;
+        for (int tile = pair; ok && tile < num_tiles; tile += npairs, ++tcount) {
+          const uint32_t buf = tcount & 1u;
+          const uint32_t tph = (tcount >> 1) & 1u;
+          if (!wait_bounded(&tempty[buf], tph ^ 1u, p, abort_flag, 3)) break;
+          tc_fence_after();
+          const uint32_t d_tmem = tmem_base + buf * BN;
+          for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+            const uint32_t s = it % STAGES;
+            const uint32_t ph = (it / STAGES) & 1u;
+            if (!wait_bounded(&full[s], ph, p, abort_flag, 4)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a0 = smem_u32(sA + s * L::A_BYTES);
+            const uint32_t b0 = smem_u32(sB + s * L::B_BYTES);
+#pragma unroll
+            for (int kk = 0; kk < kBK / 16; ++kk) {
+              const uint64_t adesc = smem_desc_sw128(a0 + kk * 32, 16, 1024);
+              const uint64_t bdesc = smem_desc_sw128(b0 + kk * 2048, L::B_CHUNK, 1024);
+              umma_f16_pair(d_tmem, adesc, bdesc, IDESC, (kb | kk) != 0 ? 1u : 0u);
+            }
+            umma_commit_pair(&empty[s], BOTH);
+          }
+          if (!ok) break;
+          umma_commit_pair(&tfull[buf], BOTH);
+        }
+        umma_commit_pair(drain, BOTH);
+      }
+      // both CTAs: the leader's MMAs write this CTA's TMEM; they must be done
+      wait_bounded(drain, 0, p, abort_flag, 5, /*honour_abort=*/false);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const uint32_t ew = warp & 3u;
+    const uint32_t et = threadIdx.x - 64;
+    uint32_t tcount = 0;
+    bool ok = true;
+    const uint32_t tempty0 = mapa_shared(smem_u32(&tempty[0]), 0);
+    for (int tile = pair; tile < num_tiles; tile += npairs, ++tcount) {
+      int mb, nb;
+      tile_coords(tile, m2_tiles, p.n_tiles, p.group_m, mb, nb);
+      const int prow = mb * 2 + static_cast<int>(rank);  // this CTA's 128-row block
+      const int m0 = prow * kBM, n0 = nb * BN;
+      const uint32_t buf = tcount & 1u;
+      const uint32_t tph = (tcount >> 1) & 1u;
+      float* bs = bias_s + buf * BN;
+      float* cp = colp_s + buf * 4 * BN;
+      epi_stage_bias<BN, EPI, BF16>(p, n0, bs, et);
+      named_bar_sync(1, 128);
+      if (ok) ok = wait_bounded(&tfull[buf], tph, p, abort_flag, 6);
+      ok = __all_sync(0xffffffffu, ok);
+      if (ok) {
+        tc_fence_after();
+        epi_rows<BN, EPI, BF16>(p, tmem_base + ((ew * 32u) << 16) + buf * BN, m0 + static_cast<int>(ew * 32 + lane), n0,
+                                bs, cp + ew * BN);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(tempty0 + buf * 8);
+      }
+      if constexpr (EPI == EPI_DRELU_BGRAD) {
+        named_bar_sync(1, 128);
+        if (ok && prow < p.m_tiles) epi_write_partials<BN>(p, prow, n0, cp, et);
+      }
+    }
+  }
+
+  tc_fence_before();
+  cluster_sync();  // neither CTA leaves while the other may still signal it
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem_base, TMEM_COLS);
+}
+
+}  // namespace ge

@@ -139,6 +139,104 @@ __device__ __forceinline__ void warp_transpose_reduce32(float (&v)[32]) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// Epilogue pieces shared by the one-CTA and the CTA-pair tile kernels. One
+// epilogue thread owns one accumulator row (its TMEM lane) of a 128-row block.
+
+// Stage the tile's bias values (fp32) in shared memory.
+template <int BN, int EPI, bool BF16>
+__device__ __forceinline__ void epi_stage_bias(const TileParams& p, int n0, float* bs, uint32_t et) {
+  if constexpr (EPI == EPI_BIAS || EPI == EPI_RELU_BIAS || EPI == EPI_RELU_AUX_BIAS) {
+    for (int c = et; c < BN; c += 128) {
+      const int n = n0 + c;
+      bs[c] = n < p.N ? load_16<BF16>(p.bias, n) : 0.f;
+    }
+  }
+}
+
+// Drain row `row` (columns n0 .. n0+BN) of the accumulator at TMEM address
+// `tbase` (this warp's lane quarter, the buffer's first column) through the
+// epilogue: bias, ReLU, mask word, 16-bit stores; for DRELU_BGRAD the mask
+// select and this warp's column sums into cpw[0..BN).
+template <int BN, int EPI, bool BF16>
+__device__ __forceinline__ void epi_rows(const TileParams& p, uint32_t tbase, int row, int n0, const float* bs,
+                                         float* cpw) {
+  const uint32_t lane = lane_id();
+  const bool row_ok = row < p.T;
+  // DRELU: this row's mask words for the whole tile, loaded before any store
+  // (a load after a store could not be moved above it)
+  uint32_t mwords[EPI == EPI_DRELU_BGRAD ? BN / 32 : 1];
+  if constexpr (EPI == EPI_DRELU_BGRAD) {
+#pragma unroll
+    for (int c = 0; c < BN / 32; ++c) {
+      const int nc0 = n0 + c * 32;
+      mwords[c] = (row_ok && nc0 < p.N) ? __ldg(p.aux_in + static_cast<int64_t>(row) * p.aux_words + (nc0 >> 5)) : 0u;
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < BN / 32; ++c) {
+    const int nc0 = n0 + c * 32;
+    if (nc0 >= p.N) break;  // warp-uniform
+    uint32_t r[32];
+    tmem_ld_32x32b_x32(tbase + c * 32, r);
+    tmem_wait_ld();
+    float v[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+    if constexpr (EPI == EPI_DRELU_BGRAD) {
+      const uint32_t m = mwords[c];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = ((m >> j) & 1u) ? v[j] : 0.f;
+    } else if constexpr (EPI != EPI_STORE) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] += bs[c * 32 + j];
+      if constexpr (EPI == EPI_RELU_BIAS || EPI == EPI_RELU_AUX_BIAS) {
+        uint32_t m = 0;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const bool pos = v[j] > 0.f;
+          m |= (pos ? 1u : 0u) << j;
+          v[j] = pos ? v[j] : 0.f;
+        }
+        if constexpr (EPI == EPI_RELU_AUX_BIAS) {
+          const int valid = p.N - nc0;
+          if (valid < 32) m &= (1u << valid) - 1u;
+          if (row_ok) p.aux_out[static_cast<int64_t>(row) * p.aux_words + (nc0 >> 5)] = m;
+        }
+      }
+    }
+    if (row_ok) {
+      uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.out) + static_cast<int64_t>(row) * p.N + nc0);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (nc0 + 8 * q < p.N) {
+          uint4 w;
+          w.x = pack2<BF16>(v[8 * q + 0], v[8 * q + 1]);
+          w.y = pack2<BF16>(v[8 * q + 2], v[8 * q + 3]);
+          w.z = pack2<BF16>(v[8 * q + 4], v[8 * q + 5]);
+          w.w = pack2<BF16>(v[8 * q + 6], v[8 * q + 7]);
+          dst[q] = w;
+        }
+      }
+    }
+    if constexpr (EPI == EPI_DRELU_BGRAD) {
+      warp_transpose_reduce32(v);
+      cpw[c * 32 + lane] = v[0];
+    }
+  }
+}
+
+// DRELU_BGRAD: combine the four warps' column sums (rows in lane-quarter
+// order) into the partial row `prow` of the workspace.
+template <int BN>
+__device__ __forceinline__ void epi_write_partials(const TileParams& p, int prow, int n0, const float* cp, uint32_t et) {
+  for (int c = et; c < BN; c += 128) {
+    const int n = n0 + c;
+    if (n < p.N)
+      p.partials[static_cast<int64_t>(prow) * p.N + n] = ((cp[0 * BN + c] + cp[1 * BN + c]) + cp[2 * BN + c]) + cp[3 * BN + c];
+  }
+}
+
 template <int BN, int STAGES, int EPI, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
     tile_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -277,96 +375,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t tph = (tcount >> 1) & 1u;
       float* bs = bias_s + buf * BN;
       float* cp = colp_s + buf * 4 * BN;
-      if constexpr (EPI == EPI_BIAS || EPI == EPI_RELU_BIAS || EPI == EPI_RELU_AUX_BIAS) {
-        for (int c = et; c < BN; c += 128) {
-          const int n = n0 + c;
-          bs[c] = n < p.N ? load_16<BF16>(p.bias, n) : 0.f;
-        }
-      }
+      epi_stage_bias<BN, EPI, BF16>(p, n0, bs, et);
       named_bar_sync(1, 128);
       if (ok) ok = wait_bounded(&tfull[buf], tph, p, abort_flag, 6);
       ok = __all_sync(0xffffffffu, ok);
       if (ok) {
         tc_fence_after();
-        const int row = m0 + static_cast<int>(ew * 32 + lane);
-        const bool row_ok = row < p.T;
-        const uint32_t tbase = tmem_base + ((ew * 32u) << 16) + buf * BN;
-        // DRELU: this row's mask words for the whole tile, loaded before any
-        // store (a load after a store could not be moved above it)
-        uint32_t mwords[EPI == EPI_DRELU_BGRAD ? BN / 32 : 1];
-        if constexpr (EPI == EPI_DRELU_BGRAD) {
-#pragma unroll
-          for (int c = 0; c < BN / 32; ++c) {
-            const int nc0 = n0 + c * 32;
-            mwords[c] = (row_ok && nc0 < p.N) ? __ldg(p.aux_in + static_cast<int64_t>(row) * p.aux_words + (nc0 >> 5)) : 0u;
-          }
-        }
-#pragma unroll
-        for (int c = 0; c < BN / 32; ++c) {
-          const int nc0 = n0 + c * 32;
-          if (nc0 >= p.N) break;  // warp-uniform
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(tbase + c * 32, r);
-          tmem_wait_ld();
-          float v[32];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-          if constexpr (EPI == EPI_DRELU_BGRAD) {
-            const uint32_t m = mwords[c];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = ((m >> j) & 1u) ? v[j] : 0.f;
-          } else if constexpr (EPI != EPI_STORE) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] += bs[c * 32 + j];
-            if constexpr (EPI == EPI_RELU_BIAS || EPI == EPI_RELU_AUX_BIAS) {
-              uint32_t m = 0;
-#pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                const bool pos = v[j] > 0.f;
-                m |= (pos ? 1u : 0u) << j;
-                v[j] = pos ? v[j] : 0.f;
-              }
-              if constexpr (EPI == EPI_RELU_AUX_BIAS) {
-                const int valid = p.N - nc0;
-                if (valid < 32) m &= (1u << valid) - 1u;
-                if (row_ok) p.aux_out[static_cast<int64_t>(row) * p.aux_words + (nc0 >> 5)] = m;
-              }
-            }
-          }
-          if (row_ok) {
-            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.out) +
-                                                  static_cast<int64_t>(row) * p.N + nc0);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              if (nc0 + 8 * q < p.N) {
-                uint4 w;
-                w.x = pack2<BF16>(v[8 * q + 0], v[8 * q + 1]);
-                w.y = pack2<BF16>(v[8 * q + 2], v[8 * q + 3]);
-                w.z = pack2<BF16>(v[8 * q + 4], v[8 * q + 5]);
-                w.w = pack2<BF16>(v[8 * q + 6], v[8 * q + 7]);
-                dst[q] = w;
-              }
-            }
-          }
-          if constexpr (EPI == EPI_DRELU_BGRAD) {
-            warp_transpose_reduce32(v);
-            cp[ew * BN + c * 32 + lane] = v[0];
-          }
-        }
+        epi_rows<BN, EPI, BF16>(p, tmem_base + ((ew * 32u) << 16) + buf * BN, m0 + static_cast<int>(ew * 32 + lane), n0,
+                                bs, cp + ew * BN);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[buf]);
       }
       if constexpr (EPI == EPI_DRELU_BGRAD) {
         named_bar_sync(1, 128);
-        if (ok) {
-          for (int c = et; c < BN; c += 128) {
-            const int n = n0 + c;
-            if (n < p.N)
-              p.partials[static_cast<int64_t>(mb) * p.N + n] = ((cp[0 * BN + c] + cp[1 * BN + c]) + cp[2 * BN + c]) +
-                                                               cp[3 * BN + c];
-          }
-        }
+        if (ok) epi_write_partials<BN>(p, mb, n0, cp, et);
       }
     }
   }

@@ -84,7 +84,8 @@ typedef struct gemm_epi_plan_s* gemm_epi_plan_t;
 typedef struct {
   int64_t T, N, K;
   int dtype, epilog;
-  int kernel;          /* 0 = persistent tile kernel, 1 = skinny (swap-AB, split-K) kernel */
+  int kernel;          /* 0 = tile kernel (one CTA per tile), 1 = few-row kernel (swap-AB,
+                          stream-K), 2 = tile kernel on CTA pairs (256-row tiles) */
   int tile_m, tile_n, tile_k, stages;
   int split_k;         /* K slices per output tile (1 = none) */
   int grid;            /* CTAs launched by the main kernel */

@@ -18,13 +18,17 @@ SHAPES = [(1, 8, 8), (5, 40, 24), (130, 72, 136), (200, 264, 200), (257, 520, 32
 # segments), with ragged K and N, and one where every CTA owns whole tiles
 SKINNY_SHAPES = [(16, 1032, 2048), (100, 264, 1000), (256, 4104, 520), (40, 2056, 64), (1, 11008, 4096)]
 FWD_EPILOGS = ["BIAS", "RELU_BIAS", "RELU_AUX_BIAS"]
-# kernel variants: the tile kernel at each width, and the few-row kernel
-VARIANTS = ["tile64", "tile128", "tile256", "skinny"]
+# CTA-pair shapes: T not a multiple of 256 (the peer CTA's rows partly or
+# wholly past T), N not a multiple of 256 (the peer's columns past N)
+PAIR_SHAPES = [(300, 264, 136), (600, 520, 328), (1000, 1032, 264), (257, 8, 64)]
+# kernel variants: the tile kernel at each width, the few-row kernel and the
+# CTA-pair tile kernel
+VARIANTS = ["tile64", "tile128", "tile256", "skinny", "pair"]
 
 
 def _force(monkeypatch, variant):
-    if variant == "skinny":
-        monkeypatch.setenv("GEMM_EPI_FORCE_KERNEL", "skinny")
+    if variant in ("skinny", "pair"):
+        monkeypatch.setenv("GEMM_EPI_FORCE_KERNEL", variant)
         monkeypatch.delenv("GEMM_EPI_FORCE_BN", raising=False)
     else:
         monkeypatch.setenv("GEMM_EPI_FORCE_KERNEL", "tile")
@@ -32,8 +36,10 @@ def _force(monkeypatch, variant):
 
 
 def _expect_variant(info, variant, T):
-    if variant == "skinny" and T <= 256:
+    if variant in ("skinny", "pair") and T <= 256:
         assert info["kernel"] == 1
+    elif variant == "pair":
+        assert info["kernel"] == 2
     else:
         assert info["kernel"] == 0
         if variant != "skinny":
@@ -72,6 +78,27 @@ def test_backward_drelu_bgrad(monkeypatch, T, N, K, dtype, variant):
 
 
 @pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+@pytest.mark.parametrize("T,N,K", PAIR_SHAPES)
+def test_pair_kernel_ragged(monkeypatch, T, N, K, dtype):
+    """CTA-pair kernel on ragged shapes, every epilog, and DRELU_BGRAD twice."""
+    _force(monkeypatch, "pair")
+    D2 = max(8, (K // 2) // 8 * 8)
+    inp = synth.make_shape_inputs(T, N, K, dtype, seed=T + 3 * N + K, D2=D2)
+    for ep in FWD_EPILOGS:
+        gpu = run_forward(inp, ep, DT[dtype])
+        _expect_variant(gpu["info"], "pair", T)
+        check_forward(inp, ep, DT[dtype], gpu)
+    fwd = run_forward(inp, "RELU_AUX_BIAS", DT[dtype])
+    outs = run_backward(inp, fwd["aux"], DT[dtype], repeats=2)
+    for gpu in outs:
+        _expect_variant(gpu["info"], "pair", T)
+        check_backward(inp, fwd["aux"], DT[dtype], gpu)
+    assert torch.equal(outs[0]["dbias"], outs[1]["dbias"])
+    for ep in FWD_EPILOGS:
+        check_forward(inp, ep, DT[dtype], run_forward(inp, ep, DT[dtype], unfused=True))
+
+
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
 @pytest.mark.parametrize("T,N,K", SKINNY_SHAPES)
 def test_skinny_split_tiles(monkeypatch, T, N, K, dtype):
     """Few-row kernel on shapes whose tiles are shared by several CTAs."""
@@ -92,10 +119,13 @@ def test_skinny_split_tiles(monkeypatch, T, N, K, dtype):
 
 @pytest.mark.parametrize("dtype", ["fp16", "bf16"])
 @pytest.mark.parametrize("T,N,K,D2", [(130, 72, 64, 40), (257, 520, 128, 96), (64, 8, 8, 8), (16, 1032, 1024, 512)])
-def test_integer_inputs_bit_exact(T, N, K, D2, dtype):
+@pytest.mark.parametrize("variant", ["auto", "pair"])
+def test_integer_inputs_bit_exact(monkeypatch, T, N, K, D2, dtype, variant):
     """Integer inputs: every sum is exact in fp32, so Y, aux, dZ and dbias
     must equal the exact result rounded once (pins ties Z == 0, the mask
     layout and the backward operand orientation)."""
+    if variant == "pair":
+        _force(monkeypatch, "pair")
     inp = synth.make_shape_inputs(T, N, K, dtype, seed=900 + T, D2=D2, kind="int")
     for ep in FWD_EPILOGS:
         gpu = run_forward(inp, ep, DT[dtype])
