@@ -518,10 +518,12 @@ def measured_traffic(w, part):
             d = json.load(f)
     except Exception:
         return None
-    entry = d.get(f"{w.name}:{part}")
-    if not entry or entry.get("source_hash") != kernel_source_hash():
-        return None
-    return entry.get("dram_bytes_per_launch")
+    current = kernel_source_hash()
+    for key, entry in d.items():
+        if key.split("#")[0] == f"{w.name}:{part}" and isinstance(entry, dict) \
+                and entry.get("source_hash") == current:
+            return entry.get("dram_bytes_per_launch")
+    return None
 
 
 if __name__ == "__main__":

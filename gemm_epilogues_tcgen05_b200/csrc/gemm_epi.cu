@@ -62,9 +62,11 @@ EncodeTiledFn encode_fn() {
 }
 
 // 2-D row-major tensor of 16-bit elements: `inner` contiguous columns,
-// `outer` rows; box of box_inner x box_outer with 128-byte swizzle.
+// `outer` rows; box of box_inner x box_outer with 128-byte swizzle (operand
+// tiles) or 64-byte swizzle (32 x 32 output staging blocks).
 int encode_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
-              uint32_t box_outer, const char* name) {
+              uint32_t box_outer, const char* name,
+              CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(GEMM_EPI_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   const cuuint64_t dims[2] = {inner, outer};
@@ -72,13 +74,19 @@ int encode_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(GEMM_EPI_ERR_CUDA, "tensor map encode for %s failed (CUresult %d)", name, (int)r);
   return GEMM_EPI_OK;
 }
 
-using TileKernelFn = void (*)(CUtensorMap, CUtensorMap, ge::TileParams);
+using TileKernelFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, ge::TileParams);
+
+// the output (Y, dZ or an unfused intermediate) as the tile kernels' TMA
+// stores see it: 32 x 32 blocks, 64-byte swizzle
+int encode_out(CUtensorMap* map, const void* out, int64_t T, int64_t N) {
+  return encode_2d(map, out, (uint64_t)N, (uint64_t)T, 32, 32, "the output", CU_TENSOR_MAP_SWIZZLE_64B);
+}
 
 template <int BN, int ST, bool BF>
 TileKernelFn pick_epi(int epi) {
@@ -181,14 +189,19 @@ SkinnyCfg skinny_cfg(int64_t T, int epi, bool bf16) {
 // Few-row problems (T <= 256) use the swap-AB stream-K kernel unless
 // GEMM_EPI_FORCE_KERNEL says otherwise ("tile" or "skinny").
 // CTA pairs (256 x 256 tiles) when there is at least one full wave of pair
-// tiles; GEMM_EPI_FORCE_KERNEL=tile / pair overrides.
-bool use_pair(int64_t T, int64_t N, int num_sms) {
+// tiles and the row operand X is at most 1 GiB. The size limit is measured,
+// not derived: under the 1 kW power cap the pair kernel ran the
+// 65536 x 16384 x 8192 fp16 problem (X = 2 GiB) at ~860 MHz and 908 TFLOP/s
+// against the one-CTA kernel's ~1100 MHz and 1106 TFLOP/s, while at
+// T = 16384 (X = 512 MiB) and below the pair kernel was as fast or up to 6 %
+// faster. GEMM_EPI_FORCE_KERNEL=tile / pair overrides.
+bool use_pair(int64_t T, int64_t N, int64_t K, int num_sms) {
   const int64_t pair_tiles = ((T + 255) / 256) * ((N + 255) / 256);
   if (const char* f = getenv("GEMM_EPI_FORCE_KERNEL")) {
     if (!strcmp(f, "tile")) return false;
     if (!strcmp(f, "pair")) return T > 256;
   }
-  return T > 256 && pair_tiles >= num_sms / 2;
+  return T > 256 && pair_tiles >= num_sms / 2 && T * K * 2 <= ((int64_t)1 << 30);
 }
 
 bool use_skinny(int64_t T) {
@@ -216,7 +229,8 @@ struct gemm_epi_plan_s {
   // tensor-map cache
   const void* a_ptr = nullptr;
   const void* b_ptr = nullptr;
-  CUtensorMap tmA, tmB;
+  const void* y_ptr = nullptr;
+  CUtensorMap tmA, tmB, tmY;
   // few-row kernel (kernel == 1)
   int kernel = 0;
   SkinnyCfg sk;
@@ -279,7 +293,18 @@ ge::TileParams base_params(const gemm_epi_plan_s* p) {
   return k;
 }
 
-int launch_tile(const gemm_epi_plan_s* p, const TileCfg& c, const ge::TileParams& k, cudaStream_t s) {
+int prepare_out_map(gemm_epi_plan_s* p, const void* out) {
+  if (out != p->y_ptr) {
+    int rc = encode_out(&p->tmY, out, p->T, p->N);
+    if (rc) return rc;
+    p->y_ptr = out;
+  }
+  return GEMM_EPI_OK;
+}
+
+int launch_tile(gemm_epi_plan_s* p, const TileCfg& c, const ge::TileParams& k, cudaStream_t s) {
+  int rc = prepare_out_map(p, k.out);
+  if (rc) return rc;
   if (c.pair) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)p->grid, 1, 1);
@@ -293,11 +318,11 @@ int launch_tile(const gemm_epi_plan_s* p, const TileCfg& c, const ge::TileParams
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, c.fn, p->tmA, p->tmB, k);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, c.fn, p->tmA, p->tmB, p->tmY, k);
     if (e != cudaSuccess) return cuda_fail(e, "pair kernel launch");
     return GEMM_EPI_OK;
   }
-  c.fn<<<p->grid, ge::kThreads, c.smem, s>>>(p->tmA, p->tmB, k);
+  c.fn<<<p->grid, ge::kThreads, c.smem, s>>>(p->tmA, p->tmB, p->tmY, k);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "tile kernel launch");
   return GEMM_EPI_OK;
@@ -420,7 +445,7 @@ gemm_epi_plan_t gemm_epi_plan(int64_t T, int64_t N, int64_t K, gemm_epi_dtype dt
   p->device = dev;
   p->num_sms = sms;
   const bool bf16 = dtype == GEMM_EPI_BF16;
-  const bool pair = use_pair(T, N, sms);
+  const bool pair = use_pair(T, N, K, sms);
   const int bn = pair ? 256 : choose_bn(T, N, sms);
   p->cfg = pair ? pair_cfg((int)epilog, bf16) : tile_cfg(bn, (int)epilog, bf16);
   p->cfg_store = pair ? pair_cfg(ge::EPI_STORE, bf16) : tile_cfg(bn, ge::EPI_STORE, bf16);
@@ -840,10 +865,12 @@ extern "C" int drelu_bgrad_execute_noalloc(int64_t T, int64_t N, int64_t K, gemm
 
   const int bn = choose_bn(T, N, sms);
   const TileCfg cfg = tile_cfg(bn, ge::EPI_DRELU_BGRAD, dtype == GEMM_EPI_BF16);
-  CUtensorMap tmA, tmB;
+  CUtensorMap tmA, tmB, tmY;
   rc = encode_2d(&tmA, dY2, (uint64_t)K, (uint64_t)T, ge::kBK, ge::kBM, "dY2");
   if (rc) return rc;
   rc = encode_2d(&tmB, W2, (uint64_t)N, (uint64_t)K, 64, ge::kBK, "W2");
+  if (rc) return rc;
+  rc = encode_out(&tmY, dZ, T, N);
   if (rc) return rc;
 
   ge::TileParams k{};
@@ -867,7 +894,7 @@ extern "C" int drelu_bgrad_execute_noalloc(int64_t T, int64_t N, int64_t K, gemm
   // rewritten by the tile kernel before the finishing kernel reads them
   e = cudaMemsetAsync(status, 0, sizeof(int), stream);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
-  cfg.fn<<<grid, ge::kThreads, cfg.smem, stream>>>(tmA, tmB, k);
+  cfg.fn<<<grid, ge::kThreads, cfg.smem, stream>>>(tmA, tmB, tmY, k);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "tile kernel launch");
   noalloc_dbias_finish_kernel<<<ceil_div(N, 256), 256, 0, stream>>>(partials, k.m_tiles, (int)N, dbias, status);

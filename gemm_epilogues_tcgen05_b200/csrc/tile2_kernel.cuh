@@ -38,14 +38,15 @@ struct Tile2Smem {
   static constexpr uint32_t OFF_MISC = OFF_BAR + N_BARS * 8;
   static constexpr uint32_t OFF_BIAS = (OFF_MISC + 16 + 15) / 16 * 16;
   static constexpr uint32_t OFF_COLP = OFF_BIAS + 2 * BN * 4;
-  static constexpr uint32_t END = OFF_COLP + 2 * 4 * BN * 4;
+  static constexpr uint32_t OFF_STG = (OFF_COLP + 2 * 4 * BN * 4 + 1023) / 1024 * 1024;
+  static constexpr uint32_t END = OFF_STG + kStageBytesPerWarp * 4;
   static constexpr uint32_t BYTES = END + 1024;
 };
 
 template <int BN, int STAGES, int EPI, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
     tile2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                 const TileParams p) {
+                 const __grid_constant__ CUtensorMap tmY, const TileParams p) {
   using L = Tile2Smem<BN, STAGES>;
   static_assert(BN == 128 || BN == 256, "the pair kernel splits BN in 64-column chunks per CTA");
   constexpr uint32_t TMEM_COLS = 2 * BN;
@@ -66,6 +67,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
   float* bias_s = reinterpret_cast<float*>(smem + L::OFF_BIAS);  // [2][BN]
   float* colp_s = reinterpret_cast<float*>(smem + L::OFF_COLP);  // [2][4][BN]
+  uint8_t* stg_s = smem + L::OFF_STG;                             // [4 warps][2][2 KB]
 
   const uint32_t warp = threadIdx.x >> 5;
   const uint32_t lane = lane_id();
@@ -89,6 +91,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
+    prefetch_tensormap(&tmY);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, TMEM_COLS);
@@ -176,6 +179,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ epilogue
     const uint32_t ew = warp & 3u;
     const uint32_t et = threadIdx.x - 64;
+    uint8_t* stg = stg_s + ew * kStageBytesPerWarp;
+    uint32_t scount = 0;
     uint32_t tcount = 0;
     bool ok = true;
     const uint32_t tempty0 = mapa_shared(smem_u32(&tempty[0]), 0);
@@ -195,7 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) {
         tc_fence_after();
         epi_rows<BN, EPI, BF16>(p, tmem_base + ((ew * 32u) << 16) + buf * BN, m0 + static_cast<int>(ew * 32 + lane), n0,
-                                bs, cp + ew * BN);
+                                bs, cp + ew * BN, &tmY, stg, scount, m0 + static_cast<int>(ew * 32));
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(tempty0 + buf * 8);
@@ -205,6 +210,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok && prow < p.m_tiles) epi_write_partials<BN>(p, prow, n0, cp, et);
       }
     }
+    if (lane == 0) bulk_wait_group_all();  // this warp's output stores are complete
+    __syncwarp();
   }
 
   tc_fence_before();

@@ -45,6 +45,9 @@ struct TileParams {
 constexpr int kBM = 128;
 constexpr int kBK = 64;
 constexpr int kThreads = 192;
+// output staging: each epilogue warp owns two 32 x 32 16-bit blocks (2 KB
+// each), written to global memory by TMA stores
+constexpr uint32_t kStageBytesPerWarp = 2 * 2048;
 
 template <int BN, int STAGES>
 struct TileSmem {
@@ -58,7 +61,8 @@ struct TileSmem {
   static constexpr uint32_t OFF_MISC = OFF_BAR + N_BARS * 8;  // tmem slot, abort flag
   static constexpr uint32_t OFF_BIAS = (OFF_MISC + 16 + 15) / 16 * 16;
   static constexpr uint32_t OFF_COLP = OFF_BIAS + 2 * BN * 4;
-  static constexpr uint32_t END = OFF_COLP + 2 * 4 * BN * 4;
+  static constexpr uint32_t OFF_STG = (OFF_COLP + 2 * 4 * BN * 4 + 1023) / 1024 * 1024;
+  static constexpr uint32_t END = OFF_STG + kStageBytesPerWarp * 4;
   static constexpr uint32_t BYTES = END + 1024;               // + alignment slack
 };
 
@@ -160,7 +164,8 @@ __device__ __forceinline__ void epi_stage_bias(const TileParams& p, int n0, floa
 // select and this warp's column sums into cpw[0..BN).
 template <int BN, int EPI, bool BF16>
 __device__ __forceinline__ void epi_rows(const TileParams& p, uint32_t tbase, int row, int n0, const float* bs,
-                                         float* cpw) {
+                                         float* cpw, const CUtensorMap* tmY, uint8_t* stg, uint32_t& scount,
+                                         int wrow0) {
   const uint32_t lane = lane_id();
   const bool row_ok = row < p.T;
   // DRELU: this row's mask words for the whole tile, loaded before any store
@@ -205,19 +210,33 @@ __device__ __forceinline__ void epi_rows(const TileParams& p, uint32_t tbase, in
         }
       }
     }
-    if (row_ok) {
-      uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.out) + static_cast<int64_t>(row) * p.N + nc0);
+    {
+      // Stage this warp's 32 x 32 block (row = lane, 64 bytes) with the
+      // 64-byte swizzle -- 16-byte chunk q of row r at chunk q ^ ((r >> 1) & 3)
+      // -- so the 16-byte shared stores are conflict-free, then one lane
+      // writes the block with a TMA store (rows and columns past T and N are
+      // clipped by the tensor map). The buffer used two blocks ago must have
+      // been read by its store before it is overwritten.
+      uint8_t* buf = stg + (scount & 1u) * 2048;
+      if (lane == 0) bulk_wait_group_read<1>();
+      __syncwarp();
+      const uint32_t rbase = smem_u32(buf) + lane * 64;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        if (nc0 + 8 * q < p.N) {
-          uint4 w;
-          w.x = pack2<BF16>(v[8 * q + 0], v[8 * q + 1]);
-          w.y = pack2<BF16>(v[8 * q + 2], v[8 * q + 3]);
-          w.z = pack2<BF16>(v[8 * q + 4], v[8 * q + 5]);
-          w.w = pack2<BF16>(v[8 * q + 6], v[8 * q + 7]);
-          dst[q] = w;
-        }
+        uint4 w;
+        w.x = pack2<BF16>(v[8 * q + 0], v[8 * q + 1]);
+        w.y = pack2<BF16>(v[8 * q + 2], v[8 * q + 3]);
+        w.z = pack2<BF16>(v[8 * q + 4], v[8 * q + 5]);
+        w.w = pack2<BF16>(v[8 * q + 6], v[8 * q + 7]);
+        st_shared_v4(rbase + ((q ^ ((lane >> 1) & 3u)) * 16), w);
       }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(tmY, buf, nc0, wrow0);
+        bulk_commit_group();
+      }
+      ++scount;
     }
     if constexpr (EPI == EPI_DRELU_BGRAD) {
       warp_transpose_reduce32(v);
@@ -240,7 +259,7 @@ __device__ __forceinline__ void epi_write_partials(const TileParams& p, int prow
 template <int BN, int STAGES, int EPI, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
     tile_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const TileParams p) {
+                const __grid_constant__ CUtensorMap tmY, const TileParams p) {
   using L = TileSmem<BN, STAGES>;
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN must be 64, 128, 192 or 256");
   constexpr uint32_t TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
@@ -261,6 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
   float* bias_s = reinterpret_cast<float*>(smem + L::OFF_BIAS);  // [2][BN]
   float* colp_s = reinterpret_cast<float*>(smem + L::OFF_COLP);  // [2][4][BN]
+  uint8_t* stg_s = smem + L::OFF_STG;                             // [4 warps][2][2 KB]
 
   const uint32_t warp = threadIdx.x >> 5;
   const uint32_t lane = lane_id();
@@ -281,6 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
+    prefetch_tensormap(&tmY);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, TMEM_COLS);
@@ -365,6 +386,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ epilogue
     const uint32_t ew = warp & 3u;        // TMEM lane quarter this warp may access
     const uint32_t et = threadIdx.x - 64;  // 0..127
+    uint8_t* stg = stg_s + ew * kStageBytesPerWarp;
+    uint32_t scount = 0;
     uint32_t tcount = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tcount) {
@@ -382,7 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) {
         tc_fence_after();
         epi_rows<BN, EPI, BF16>(p, tmem_base + ((ew * 32u) << 16) + buf * BN, m0 + static_cast<int>(ew * 32 + lane), n0,
-                                bs, cp + ew * BN);
+                                bs, cp + ew * BN, &tmY, stg, scount, m0 + static_cast<int>(ew * 32));
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[buf]);
@@ -392,6 +415,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) epi_write_partials<BN>(p, mb, n0, cp, et);
       }
     }
+    if (lane == 0) bulk_wait_group_all();  // this warp's output stores are complete
+    __syncwarp();
   }
 
   tc_fence_before();
