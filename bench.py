@@ -482,9 +482,9 @@ def main():
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "frac_of_burst": achieved / burst,
                 "peak_kind": "sustained (launch >= 1 ms)" if long_launch else "burst (launch < 1 ms)"}
-    kname = ("skinny_kernel" if res["kernel"] == 1 else "tile_kernel")
+    kname = {0: "tile_kernel", 1: "skinny_kernel", 2: "tile2_kernel (CTA pair)"}[res["kernel"]]
     roof["kernel"] = f"{part}: {kname} " + (fwd_epi if part == "fwd" else "DRELU_BGRAD" +
-                                              (" + dbias finish" if res["kernel"] == 0 else ""))
+                                              (" + dbias finish" if res["kernel"] != 1 else ""))
     roof["peak_source"] = "measured (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
     roof["traffic"] = measured_traffic(w, part)
     # roofline time of the whole step: slower of FLOPs at the tensor peak and bytes at HBM
