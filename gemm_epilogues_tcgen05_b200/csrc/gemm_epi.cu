@@ -226,6 +226,7 @@ struct gemm_epi_plan_s {
   int* status_host = nullptr;
   int* status_dev = nullptr;
   uint64_t timeout_ns = 0;
+  int inject_stall = 0;  // GEMM_EPI_INJECT_STALL at plan time (watchdog tests)
   // tensor-map cache
   const void* a_ptr = nullptr;
   const void* b_ptr = nullptr;
@@ -290,6 +291,7 @@ ge::TileParams base_params(const gemm_epi_plan_s* p) {
   k.group_m = p->group_m;
   k.status = p->status_dev;
   k.timeout_ns = p->timeout_ns;
+  k.inject_stall = p->inject_stall;
   return k;
 }
 
@@ -467,6 +469,10 @@ gemm_epi_plan_t gemm_epi_plan(int64_t T, int64_t N, int64_t K, gemm_epi_dtype dt
     long long ms = atoll(t);
     if (ms > 0) p->timeout_ns = (uint64_t)ms * 1000000ull;
   }
+  // Fault injection for the watchdog tests (one-CTA tile kernel only): the
+  // MMA warp withholds its first tile's completion signal, so the epilogue's
+  // bounded wait runs out and the kernel reports ERR_TIMEOUT.
+  if (const char* f = getenv("GEMM_EPI_INJECT_STALL")) p->inject_stall = atoi(f) != 0;
 
   auto cleanup = [&](int rc) {
     if (p->sk_partials) cudaFree(p->sk_partials);

@@ -40,6 +40,7 @@ struct TileParams {
   float* partials;          // DRELU_BGRAD: m_tiles x N column partial sums
   int* status;              // watchdog report (host-visible)
   uint64_t timeout_ns;
+  int32_t inject_stall;     // fault injection for tests: withhold the first tile's tmem_full commit
 };
 
 constexpr int kBM = 128;
@@ -375,7 +376,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_commit(&empty[s]);
         }
         if (!ok) break;
-        umma_commit(&tfull[buf]);
+        // (fault injection: the epilogue then waits on a barrier nothing arrives on)
+        if (!(p.inject_stall && tcount == 0)) umma_commit(&tfull[buf]);
       }
       // every MMA issued above must finish before tensor memory is freed
       umma_commit(drain);

@@ -226,3 +226,34 @@ def test_injected_workspace_allocation_failure(monkeypatch):
     with pytest.raises(binding.GemmEpiError) as e:
         binding.gemm_epi_plan(256, 256, 256, binding.BF16, binding.DRELU_BGRAD)
     assert "injected" in str(e.value)
+
+
+@pytest.mark.parametrize("epilog", ["RELU_AUX_BIAS", "DRELU_BGRAD"])
+def test_watchdog_reports_timeout_and_context_stays_usable(monkeypatch, epilog):
+    """Fault injection without a GPU fault: the MMA warp withholds the first
+    tile's completion signal, the epilogue's bounded wait (200 ms here) runs
+    out, the kernel frees its tensor memory and returns, and the host reads
+    ERR_TIMEOUT. A fresh plan afterwards must compute correctly."""
+    T, N, K = 512, 512, 256
+    monkeypatch.setenv("GEMM_EPI_FORCE_KERNEL", "tile")
+    monkeypatch.setenv("GEMM_EPI_FORCE_BN", "64")
+    monkeypatch.setenv("GEMM_EPI_WAIT_TIMEOUT_MS", "200")
+    monkeypatch.setenv("GEMM_EPI_INJECT_STALL", "1")
+    inp = synth.make_shape_inputs(T, N, K, "bf16", seed=17, D2=K)
+    g = {k: v.cuda() for k, v in inp.items()}
+    dt = torch.bfloat16
+    aux = torch.zeros((T, (N + 31) // 32), dtype=torch.int32, device="cuda")
+    with binding.Plan(T, N, K, dt, epilog) as plan:
+        if epilog == "DRELU_BGRAD":
+            plan.backward(g["dY2"], g["W2"], aux)
+        else:
+            plan.forward(g["X"], g["W"], g["bias"])
+        torch.cuda.synchronize()  # returns: the kernel gave up and exited
+        assert plan.status() == binding.ERR_TIMEOUT
+        assert "watchdog" in binding.gemm_epi_last_error()
+        assert plan.status() == binding.OK  # the report is cleared by reading it
+    monkeypatch.delenv("GEMM_EPI_INJECT_STALL")
+    gpu = run_forward(inp, "RELU_AUX_BIAS", dt)
+    check_forward(inp, "RELU_AUX_BIAS", dt, gpu)
+    out = run_backward(inp, gpu["aux"], dt)
+    check_backward(inp, gpu["aux"], dt, out)
