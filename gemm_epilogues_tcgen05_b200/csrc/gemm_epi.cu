@@ -80,12 +80,36 @@ int encode_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer
   return GEMM_EPI_OK;
 }
 
-using TileKernelFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, ge::TileParams);
+using TileKernelFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, ge::TileParams);
 
 // the output (Y, dZ or an unfused intermediate) as the tile kernels' TMA
 // stores see it: 32 x 32 blocks, 64-byte swizzle
 int encode_out(CUtensorMap* map, const void* out, int64_t T, int64_t N) {
   return encode_2d(map, out, (uint64_t)N, (uint64_t)T, 32, 32, "the output", CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
+// the mask words as the tile kernels' TMA stores see them: per warp and tile
+// a block of BN/32 words x 32 rows. Usable when a row of words is a multiple
+// of 16 bytes and the pointer is 16-byte aligned; otherwise the kernels store
+// the words directly.
+bool aux_tma_ok(const void* aux, int64_t N, int bn) {
+  const int64_t words = (N + 31) / 32;
+  return bn >= 128 && (words % 4) == 0 && (reinterpret_cast<uintptr_t>(aux) & 15) == 0;
+}
+
+int encode_aux(CUtensorMap* map, const void* aux, int64_t T, int64_t N, int bn) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(GEMM_EPI_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const uint64_t words = (uint64_t)((N + 31) / 32);
+  const cuuint64_t dims[2] = {words, (uint64_t)T};
+  const cuuint64_t strides[1] = {words * 4};
+  const cuuint32_t box[2] = {(cuuint32_t)(bn / 32), 32};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(aux), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(GEMM_EPI_ERR_CUDA, "tensor map encode for the mask words failed (CUresult %d)", (int)r);
+  return GEMM_EPI_OK;
 }
 
 template <int BN, int ST, bool BF>
@@ -231,7 +255,8 @@ struct gemm_epi_plan_s {
   const void* a_ptr = nullptr;
   const void* b_ptr = nullptr;
   const void* y_ptr = nullptr;
-  CUtensorMap tmA, tmB, tmY;
+  const void* aux_ptr = nullptr;
+  CUtensorMap tmA, tmB, tmY, tmAux;
   // few-row kernel (kernel == 1)
   int kernel = 0;
   SkinnyCfg sk;
@@ -304,9 +329,20 @@ int prepare_out_map(gemm_epi_plan_s* p, const void* out) {
   return GEMM_EPI_OK;
 }
 
-int launch_tile(gemm_epi_plan_s* p, const TileCfg& c, const ge::TileParams& k, cudaStream_t s) {
+int launch_tile(gemm_epi_plan_s* p, const TileCfg& c, const ge::TileParams& k_in, cudaStream_t s) {
+  ge::TileParams k = k_in;
   int rc = prepare_out_map(p, k.out);
   if (rc) return rc;
+  k.aux_tma = 0;
+  if (k.aux_out && aux_tma_ok(k.aux_out, p->N, c.BN)) {
+    if (k.aux_out != p->aux_ptr) {
+      rc = encode_aux(&p->tmAux, k.aux_out, p->T, p->N, c.BN);
+      if (rc) return rc;
+      p->aux_ptr = k.aux_out;
+    }
+    k.aux_tma = 1;
+  }
+  const CUtensorMap& tmAux = k.aux_tma ? p->tmAux : p->tmY;  // unused by the kernel unless aux_tma
   if (c.pair) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)p->grid, 1, 1);
@@ -320,11 +356,11 @@ int launch_tile(gemm_epi_plan_s* p, const TileCfg& c, const ge::TileParams& k, c
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, c.fn, p->tmA, p->tmB, p->tmY, k);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, c.fn, p->tmA, p->tmB, p->tmY, tmAux, k);
     if (e != cudaSuccess) return cuda_fail(e, "pair kernel launch");
     return GEMM_EPI_OK;
   }
-  c.fn<<<p->grid, ge::kThreads, c.smem, s>>>(p->tmA, p->tmB, p->tmY, k);
+  c.fn<<<p->grid, ge::kThreads, c.smem, s>>>(p->tmA, p->tmB, p->tmY, tmAux, k);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "tile kernel launch");
   return GEMM_EPI_OK;
@@ -900,7 +936,7 @@ extern "C" int drelu_bgrad_execute_noalloc(int64_t T, int64_t N, int64_t K, gemm
   // rewritten by the tile kernel before the finishing kernel reads them
   e = cudaMemsetAsync(status, 0, sizeof(int), stream);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
-  cfg.fn<<<grid, ge::kThreads, cfg.smem, stream>>>(tmA, tmB, tmY, k);
+  cfg.fn<<<grid, ge::kThreads, cfg.smem, stream>>>(tmA, tmB, tmY, tmY, k);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "tile kernel launch");
   noalloc_dbias_finish_kernel<<<ceil_div(N, 256), 256, 0, stream>>>(partials, k.m_tiles, (int)N, dbias, status);

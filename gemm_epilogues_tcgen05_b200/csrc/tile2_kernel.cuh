@@ -39,14 +39,16 @@ struct Tile2Smem {
   static constexpr uint32_t OFF_BIAS = (OFF_MISC + 16 + 15) / 16 * 16;
   static constexpr uint32_t OFF_COLP = OFF_BIAS + 2 * BN * 4;
   static constexpr uint32_t OFF_STG = (OFF_COLP + 2 * 4 * BN * 4 + 1023) / 1024 * 1024;
-  static constexpr uint32_t END = OFF_STG + kStageBytesPerWarp * 4;
+  static constexpr uint32_t OFF_AUXSTG = OFF_STG + kStageBytesPerWarp * 4;
+  static constexpr uint32_t END = OFF_AUXSTG + kAuxStageBytesPerWarp * 4;
   static constexpr uint32_t BYTES = END + 1024;
 };
 
 template <int BN, int STAGES, int EPI, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
     tile2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                 const __grid_constant__ CUtensorMap tmY, const TileParams p) {
+                 const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmAux,
+                 const TileParams p) {
   using L = Tile2Smem<BN, STAGES>;
   static_assert(BN == 128 || BN == 256, "the pair kernel splits BN in 64-column chunks per CTA");
   constexpr uint32_t TMEM_COLS = 2 * BN;
@@ -68,6 +70,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* bias_s = reinterpret_cast<float*>(smem + L::OFF_BIAS);  // [2][BN]
   float* colp_s = reinterpret_cast<float*>(smem + L::OFF_COLP);  // [2][4][BN]
   uint8_t* stg_s = smem + L::OFF_STG;                             // [4 warps][2][2 KB]
+  uint8_t* auxstg_s = smem + L::OFF_AUXSTG;                       // [4 warps][1 KB]
 
   const uint32_t warp = threadIdx.x >> 5;
   const uint32_t lane = lane_id();
@@ -200,7 +203,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) {
         tc_fence_after();
         epi_rows<BN, EPI, BF16>(p, tmem_base + ((ew * 32u) << 16) + buf * BN, m0 + static_cast<int>(ew * 32 + lane), n0,
-                                bs, cp + ew * BN, &tmY, stg, scount, m0 + static_cast<int>(ew * 32));
+                                bs, cp + ew * BN, &tmY, stg, scount, m0 + static_cast<int>(ew * 32), &tmAux,
+                                auxstg_s + ew * kAuxStageBytesPerWarp);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(tempty0 + buf * 8);

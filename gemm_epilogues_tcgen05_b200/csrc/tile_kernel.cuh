@@ -41,6 +41,7 @@ struct TileParams {
   int* status;              // watchdog report (host-visible)
   uint64_t timeout_ns;
   int32_t inject_stall;     // fault injection for tests: withhold the first tile's tmem_full commit
+  int32_t aux_tma;          // RELU_AUX_BIAS: mask words go out by TMA store (see AuxByTma)
 };
 
 constexpr int kBM = 128;
@@ -49,6 +50,8 @@ constexpr int kThreads = 192;
 // output staging: each epilogue warp owns two 32 x 32 16-bit blocks (2 KB
 // each), written to global memory by TMA stores
 constexpr uint32_t kStageBytesPerWarp = 2 * 2048;
+// mask-word staging: each epilogue warp's 32 rows x (BN / 32) words of a tile
+constexpr uint32_t kAuxStageBytesPerWarp = 1024;
 
 template <int BN, int STAGES>
 struct TileSmem {
@@ -63,7 +66,8 @@ struct TileSmem {
   static constexpr uint32_t OFF_BIAS = (OFF_MISC + 16 + 15) / 16 * 16;
   static constexpr uint32_t OFF_COLP = OFF_BIAS + 2 * BN * 4;
   static constexpr uint32_t OFF_STG = (OFF_COLP + 2 * 4 * BN * 4 + 1023) / 1024 * 1024;
-  static constexpr uint32_t END = OFF_STG + kStageBytesPerWarp * 4;
+  static constexpr uint32_t OFF_AUXSTG = OFF_STG + kStageBytesPerWarp * 4;
+  static constexpr uint32_t END = OFF_AUXSTG + kAuxStageBytesPerWarp * 4;
   static constexpr uint32_t BYTES = END + 1024;               // + alignment slack
 };
 
@@ -163,12 +167,26 @@ __device__ __forceinline__ void epi_stage_bias(const TileParams& p, int n0, floa
 // `tbase` (this warp's lane quarter, the buffer's first column) through the
 // epilogue: bias, ReLU, mask word, 16-bit stores; for DRELU_BGRAD the mask
 // select and this warp's column sums into cpw[0..BN).
+// Mask words go out through shared memory and one TMA store per warp and
+// tile when a row's words span at least 16 bytes (BN >= 128); with BN = 64
+// (8 bytes) they are stored directly.
+template <int BN>
+struct AuxByTma {
+  static constexpr bool value = BN >= 128;
+};
+
 template <int BN, int EPI, bool BF16>
 __device__ __forceinline__ void epi_rows(const TileParams& p, uint32_t tbase, int row, int n0, const float* bs,
                                          float* cpw, const CUtensorMap* tmY, uint8_t* stg, uint32_t& scount,
-                                         int wrow0) {
+                                         int wrow0, const CUtensorMap* tmAux, uint8_t* auxstg) {
   const uint32_t lane = lane_id();
   const bool row_ok = row < p.T;
+  constexpr bool kAuxTma = EPI == EPI_RELU_AUX_BIAS && AuxByTma<BN>::value;
+  uint32_t auxw[kAuxTma ? BN / 32 : 1];
+  if constexpr (kAuxTma) {
+#pragma unroll
+    for (int c = 0; c < BN / 32; ++c) auxw[c] = 0u;
+  }
   // DRELU: this row's mask words for the whole tile, loaded before any store
   // (a load after a store could not be moved above it)
   uint32_t mwords[EPI == EPI_DRELU_BGRAD ? BN / 32 : 1];
@@ -207,7 +225,10 @@ __device__ __forceinline__ void epi_rows(const TileParams& p, uint32_t tbase, in
         if constexpr (EPI == EPI_RELU_AUX_BIAS) {
           const int valid = p.N - nc0;
           if (valid < 32) m &= (1u << valid) - 1u;
-          if (row_ok) p.aux_out[static_cast<int64_t>(row) * p.aux_words + (nc0 >> 5)] = m;
+          if (kAuxTma && p.aux_tma)
+            auxw[kAuxTma ? c : 0] = m;
+          else if (row_ok)
+            p.aux_out[static_cast<int64_t>(row) * p.aux_words + (nc0 >> 5)] = m;
         }
       }
     }
@@ -244,6 +265,20 @@ __device__ __forceinline__ void epi_rows(const TileParams& p, uint32_t tbase, in
       cpw[c * 32 + lane] = v[0];
     }
   }
+  if (kAuxTma && p.aux_tma) {
+    // row `lane` of the warp's [32][BN/32] word block; the previous tile's
+    // block was read by its store before any later chunk's wait returned
+    constexpr int WB = BN / 32 * 4;  // bytes per row
+    const uint32_t rb = smem_u32(auxstg) + lane * WB;
+#pragma unroll
+    for (int q = 0; q < WB / 16; ++q) st_shared_v4(rb + q * 16, make_uint4(auxw[4 * q], auxw[4 * q + 1], auxw[4 * q + 2], auxw[4 * q + 3]));
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(tmAux, auxstg, n0 >> 5, wrow0);
+      bulk_commit_group();
+    }
+  }
 }
 
 // DRELU_BGRAD: combine the four warps' column sums (rows in lane-quarter
@@ -260,7 +295,8 @@ __device__ __forceinline__ void epi_write_partials(const TileParams& p, int prow
 template <int BN, int STAGES, int EPI, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
     tile_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const __grid_constant__ CUtensorMap tmY, const TileParams p) {
+                const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmAux,
+                const TileParams p) {
   using L = TileSmem<BN, STAGES>;
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN must be 64, 128, 192 or 256");
   constexpr uint32_t TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
@@ -282,6 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* bias_s = reinterpret_cast<float*>(smem + L::OFF_BIAS);  // [2][BN]
   float* colp_s = reinterpret_cast<float*>(smem + L::OFF_COLP);  // [2][4][BN]
   uint8_t* stg_s = smem + L::OFF_STG;                             // [4 warps][2][2 KB]
+  uint8_t* auxstg_s = smem + L::OFF_AUXSTG;                       // [4 warps][1 KB]
 
   const uint32_t warp = threadIdx.x >> 5;
   const uint32_t lane = lane_id();
@@ -407,7 +444,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) {
         tc_fence_after();
         epi_rows<BN, EPI, BF16>(p, tmem_base + ((ew * 32u) << 16) + buf * BN, m0 + static_cast<int>(ew * 32 + lane), n0,
-                                bs, cp + ew * BN, &tmY, stg, scount, m0 + static_cast<int>(ew * 32));
+                                bs, cp + ew * BN, &tmY, stg, scount, m0 + static_cast<int>(ew * 32), &tmAux,
+                                auxstg_s + ew * kAuxStageBytesPerWarp);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[buf]);

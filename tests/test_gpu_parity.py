@@ -13,14 +13,15 @@ from _parity import check_backward, check_forward, run_backward, run_forward
 pytestmark = pytest.mark.gpu
 
 DT = {"fp16": torch.float16, "bf16": torch.bfloat16}
-SHAPES = [(1, 8, 8), (5, 40, 24), (130, 72, 136), (200, 264, 200), (257, 520, 328), (384, 512, 512)]
+SHAPES = [(1, 8, 8), (5, 40, 24), (130, 72, 136), (200, 264, 200), (257, 520, 328), (384, 512, 512),
+          (300, 640, 136)]  # the last two: ceil(N/32) % 4 == 0, so mask words go out by TMA store
 # few-row shapes whose feature tiles are split over several CTAs (stream-K
 # segments), with ragged K and N, and one where every CTA owns whole tiles
 SKINNY_SHAPES = [(16, 1032, 2048), (100, 264, 1000), (256, 4104, 520), (40, 2056, 64), (1, 11008, 4096)]
 FWD_EPILOGS = ["BIAS", "RELU_BIAS", "RELU_AUX_BIAS"]
 # CTA-pair shapes: T not a multiple of 256 (the peer CTA's rows partly or
 # wholly past T), N not a multiple of 256 (the peer's columns past N)
-PAIR_SHAPES = [(300, 264, 136), (600, 520, 328), (1000, 1032, 264), (257, 8, 64)]
+PAIR_SHAPES = [(300, 264, 136), (600, 520, 328), (1000, 1032, 264), (257, 8, 64), (600, 1024, 328)]
 # kernel variants: the tile kernel at each width, the few-row kernel and the
 # CTA-pair tile kernel
 VARIANTS = ["tile64", "tile128", "tile256", "skinny", "pair"]
@@ -118,7 +119,8 @@ def test_skinny_split_tiles(monkeypatch, T, N, K, dtype):
 
 
 @pytest.mark.parametrize("dtype", ["fp16", "bf16"])
-@pytest.mark.parametrize("T,N,K,D2", [(130, 72, 64, 40), (257, 520, 128, 96), (64, 8, 8, 8), (16, 1032, 1024, 512)])
+@pytest.mark.parametrize("T,N,K,D2", [(130, 72, 64, 40), (257, 520, 128, 96), (64, 8, 8, 8), (16, 1032, 1024, 512),
+                                      (300, 1024, 64, 40)])
 @pytest.mark.parametrize("variant", ["auto", "pair"])
 def test_integer_inputs_bit_exact(monkeypatch, T, N, K, D2, dtype, variant):
     """Integer inputs: every sum is exact in fp32, so Y, aux, dZ and dbias
