@@ -222,16 +222,22 @@ SkinnyCfg skinny_cfg(int64_t T, int epi, bool bf16) {
 bool use_pair(int64_t T, int64_t N, int64_t K, int num_sms) {
   const int64_t pair_tiles = ((T + 255) / 256) * ((N + 255) / 256);
   if (const char* f = getenv("GEMM_EPI_FORCE_KERNEL")) {
-    if (!strcmp(f, "tile")) return false;
-    if (!strcmp(f, "pair")) return T > 256;
+    if (!strcmp(f, "tile") || !strcmp(f, "skinny")) return false;
+    if (!strcmp(f, "pair")) return T >= 256;
   }
-  return T > 256 && pair_tiles >= num_sms / 2 && T * K * 2 <= ((int64_t)1 << 30);
+  if (T * K * 2 > ((int64_t)1 << 30)) return false;
+  // 192..256 rows: one pair tile row halves each CTA's operand feed against
+  // the few-row kernel's (measured at T = 256, N = 11008: 38.0 / 40.3 us
+  // forward / backward against 50.1 / 60.8 us), given a quarter wave of tiles
+  if (T >= 192 && T <= 256) return pair_tiles >= num_sms / 4;
+  return T > 256 && pair_tiles >= num_sms / 2;
 }
 
 bool use_skinny(int64_t T) {
   if (const char* f = getenv("GEMM_EPI_FORCE_KERNEL")) {
     if (!strcmp(f, "tile")) return false;
     if (!strcmp(f, "skinny")) return T <= 256;
+    if (!strcmp(f, "pair")) return T < 256;
   }
   return T <= 256;
 }
@@ -524,7 +530,7 @@ gemm_epi_plan_t gemm_epi_plan(int64_t T, int64_t N, int64_t K, gemm_epi_dtype dt
     e = cudaFuncSetAttribute(c->fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)c->smem);
     if (e != cudaSuccess) return cleanup(cuda_fail(e, "cudaFuncSetAttribute(max dynamic shared memory)"));
   }
-  if (use_skinny(T)) {
+  if (!pair && use_skinny(T)) {
     p->kernel = 1;
     p->sk = skinny_cfg(T, (int)epilog, bf16);
     const int n_tiles = ceil_div(N, 128);
