@@ -253,6 +253,7 @@ struct gemm_epi_plan_s {
   TileCfg cfg_store; // unfused GEMM (plain store)
   float* partials = nullptr;  // DRELU_BGRAD: m_tiles x N
   size_t partial_bytes = 0;
+  int* col_tickets = nullptr;  // DRELU_BGRAD on the tile kernels: n_tiles counters
   int* status_host = nullptr;
   int* status_dev = nullptr;
   uint64_t timeout_ns = 0;
@@ -290,6 +291,7 @@ int take_status(gemm_epi_plan_s* p) {
     *s = 0;
     // an interrupted launch may have left split-tile tickets counted
     if (p->sk_tickets) cudaMemset(p->sk_tickets, 0, sizeof(int) * (size_t)ceil_div(p->N, 128));
+    if (p->col_tickets) cudaMemset(p->col_tickets, 0, sizeof(int) * (size_t)p->n_tiles);
     return fail(GEMM_EPI_ERR_TIMEOUT, "a kernel of this plan gave up waiting (watchdog code 0x%x)", v);
   }
   return GEMM_EPI_OK;
@@ -517,6 +519,7 @@ gemm_epi_plan_t gemm_epi_plan(int64_t T, int64_t N, int64_t K, gemm_epi_dtype dt
   if (const char* f = getenv("GEMM_EPI_INJECT_STALL")) p->inject_stall = atoi(f) != 0;
 
   auto cleanup = [&](int rc) {
+    if (p->col_tickets) cudaFree(p->col_tickets);
     if (p->sk_partials) cudaFree(p->sk_partials);
     if (p->sk_tickets) cudaFree(p->sk_tickets);
     if (p->partials) cudaFree(p->partials);
@@ -584,6 +587,12 @@ gemm_epi_plan_t gemm_epi_plan(int64_t T, int64_t N, int64_t K, gemm_epi_dtype dt
       return cleanup(fail(GEMM_EPI_ERR_CUDA, "injected workspace allocation failure"));
     e = cudaMalloc((void**)&p->partials, p->partial_bytes);
     if (e != cudaSuccess) return cleanup(cuda_fail(e, "cudaMalloc(workspace)"));
+    if (p->kernel != 1) {  // the tile kernels finish dbias themselves (last ticket per column block)
+      e = cudaMalloc((void**)&p->col_tickets, sizeof(int) * (size_t)p->n_tiles);
+      if (e != cudaSuccess) return cleanup(cuda_fail(e, "cudaMalloc(column tickets)"));
+      e = cudaMemset(p->col_tickets, 0, sizeof(int) * (size_t)p->n_tiles);
+      if (e != cudaSuccess) return cleanup(cuda_fail(e, "cudaMemset(column tickets)"));
+    }
   }
   {
     std::lock_guard<std::mutex> g(g_mu);
@@ -603,6 +612,7 @@ void gemm_epi_free(gemm_epi_plan_t plan) {
     }
   }
   if (plan->partials) cudaFree(plan->partials);
+  if (plan->col_tickets) cudaFree(plan->col_tickets);
   if (plan->sk_partials) cudaFree(plan->sk_partials);
   if (plan->sk_tickets) cudaFree(plan->sk_tickets);
   if (plan->status_host) cudaFreeHost(plan->status_host);
@@ -638,8 +648,8 @@ int gemm_epi_query(gemm_epi_plan_t plan, gemm_epi_info* info) {
     info->stages = p->cfg.stages;
     info->split_k = 1;
     info->grid = p->grid;
-    info->launches = p->epilog == GEMM_EPI_DRELU_BGRAD ? 2 : 1;
-    info->workspace_bytes = p->epilog == GEMM_EPI_DRELU_BGRAD ? p->partial_bytes : 0;
+    info->launches = 1;
+    info->workspace_bytes = p->epilog == GEMM_EPI_DRELU_BGRAD ? p->partial_bytes + sizeof(int) * (size_t)p->n_tiles : 0;
   }
   return GEMM_EPI_OK;
 }
@@ -710,12 +720,9 @@ int drelu_bgrad_execute(gemm_epi_plan_t plan, const void* dY2, const void* W2, c
   k.out = dZ;
   k.aux_in = aux;
   k.partials = p->partials;
-  rc = launch_tile(p, p->cfg, k, stream);
-  if (rc) return rc;
-  ge::dbias_finish_kernel<<<ceil_div(p->N, 256), 256, 0, stream>>>(p->partials, p->m_tiles, (int)p->N, dbias);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "dbias finish launch");
-  return GEMM_EPI_OK;
+  k.col_tickets = p->col_tickets;
+  k.dbias = dbias;
+  return launch_tile(p, p->cfg, k, stream);
 }
 
 int gemm_epi_unfused_execute(gemm_epi_plan_t plan, const void* X, const void* W, const void* bias, void* T1, void* T2,

@@ -71,6 +71,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* colp_s = reinterpret_cast<float*>(smem + L::OFF_COLP);  // [2][4][BN]
   uint8_t* stg_s = smem + L::OFF_STG;                             // [4 warps][2][2 KB]
   uint8_t* auxstg_s = smem + L::OFF_AUXSTG;                       // [4 warps][1 KB]
+  volatile int* dflag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 8);
 
   const uint32_t warp = threadIdx.x >> 5;
   const uint32_t lane = lane_id();
@@ -211,7 +212,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if constexpr (EPI == EPI_DRELU_BGRAD) {
         named_bar_sync(1, 128);
-        if (ok && prow < p.m_tiles) epi_write_partials<BN>(p, prow, n0, cp, et);
+        const bool has_row = prow < p.m_tiles;
+        if (ok && has_row) epi_write_partials<BN>(p, prow, n0, cp, et);
+        if (p.col_tickets) epi_finish_dbias<BN>(p, nb, n0, (ok && has_row) ? 1 : 0, et, dflag);
       }
     }
     if (lane == 0) bulk_wait_group_all();  // this warp's output stores are complete

@@ -42,6 +42,8 @@ struct TileParams {
   uint64_t timeout_ns;
   int32_t inject_stall;     // fault injection for tests: withhold the first tile's tmem_full commit
   int32_t aux_tma;          // RELU_AUX_BIAS: mask words go out by TMA store (see AuxByTma)
+  int* col_tickets;         // DRELU_BGRAD: per column block, zero between launches; null = no in-kernel finish
+  float* dbias;             // DRELU_BGRAD: written by the tile that takes a column block's last ticket
 };
 
 constexpr int kBM = 128;
@@ -292,6 +294,38 @@ __device__ __forceinline__ void epi_write_partials(const TileParams& p, int prow
   }
 }
 
+// DRELU_BGRAD, second pass inside the kernel: after its partial rows are
+// written, a tile takes `rows` tickets on its column block; the tile that
+// takes the block's last ticket sums every partial row of the block in
+// ascending row order -- the same order whichever tile is last -- writes
+// dbias and resets the counter for the next launch. Called by the 128
+// epilogue threads; `flag` is a shared-memory word.
+template <int BN>
+__device__ __forceinline__ void epi_finish_dbias(const TileParams& p, int nb, int n0, int rows, uint32_t et,
+                                                 volatile int* flag) {
+  __threadfence();
+  named_bar_sync(1, 128);
+  if (et == 0) {
+    const int prev = atomicAdd(p.col_tickets + nb, rows);
+    const int last = prev + rows == p.m_tiles;
+    if (last) p.col_tickets[nb] = 0;
+    *flag = last;
+  }
+  named_bar_sync(1, 128);
+  if (*flag) {
+    __threadfence();
+    for (int c = et; c < BN; c += 128) {
+      const int n = n0 + c;
+      if (n < p.N) {
+        float s = 0.f;
+        for (int m = 0; m < p.m_tiles; ++m) s += __ldcg(p.partials + static_cast<int64_t>(m) * p.N + n);
+        p.dbias[n] = s;
+      }
+    }
+  }
+  named_bar_sync(1, 128);  // the flag word is reused by the next tile
+}
+
 template <int BN, int STAGES, int EPI, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
     tile_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -319,6 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* colp_s = reinterpret_cast<float*>(smem + L::OFF_COLP);  // [2][4][BN]
   uint8_t* stg_s = smem + L::OFF_STG;                             // [4 warps][2][2 KB]
   uint8_t* auxstg_s = smem + L::OFF_AUXSTG;                       // [4 warps][1 KB]
+  volatile int* dflag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 8);
 
   const uint32_t warp = threadIdx.x >> 5;
   const uint32_t lane = lane_id();
@@ -453,6 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if constexpr (EPI == EPI_DRELU_BGRAD) {
         named_bar_sync(1, 128);
         if (ok) epi_write_partials<BN>(p, mb, n0, cp, et);
+        if (p.col_tickets) epi_finish_dbias<BN>(p, nb, n0, ok ? 1 : 0, et, dflag);
       }
     }
     if (lane == 0) bulk_wait_group_all();  // this warp's output stores are complete
