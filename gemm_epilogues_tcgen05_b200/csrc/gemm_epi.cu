@@ -223,13 +223,15 @@ bool use_pair(int64_t T, int64_t N, int64_t K, int num_sms) {
   const int64_t pair_tiles = ((T + 255) / 256) * ((N + 255) / 256);
   if (const char* f = getenv("GEMM_EPI_FORCE_KERNEL")) {
     if (!strcmp(f, "tile") || !strcmp(f, "skinny")) return false;
-    if (!strcmp(f, "pair")) return T >= 256;
+    if (!strcmp(f, "pair")) return T > 128;
   }
   if (T * K * 2 > ((int64_t)1 << 30)) return false;
-  // 192..256 rows: one pair tile row halves each CTA's operand feed against
-  // the few-row kernel's (measured at T = 256, N = 11008: 38.0 / 40.3 us
-  // forward / backward against 50.1 / 60.8 us), given a quarter wave of tiles
-  if (T >= 192 && T <= 256) return pair_tiles >= num_sms / 4;
+  // 129..256 rows: one pair tile row halves each CTA's operand feed against
+  // the few-row kernel's (measured at N = 11008, K = 4096, forward / backward:
+  // T = 256 38.0 / 40.3 us against 50.1 / 60.8; T = 192 39.4 / 41.5 against
+  // 50.3 / 53.8), given a quarter wave of tiles; at T = 128 the few-row kernel
+  // is as fast and wastes no rows
+  if (T > 128 && T <= 256) return pair_tiles >= num_sms / 4;
   return T > 256 && pair_tiles >= num_sms / 2;
 }
 
@@ -237,7 +239,7 @@ bool use_skinny(int64_t T) {
   if (const char* f = getenv("GEMM_EPI_FORCE_KERNEL")) {
     if (!strcmp(f, "tile")) return false;
     if (!strcmp(f, "skinny")) return T <= 256;
-    if (!strcmp(f, "pair")) return T < 256;
+    if (!strcmp(f, "pair")) return T <= 128;
   }
   return T <= 256;
 }

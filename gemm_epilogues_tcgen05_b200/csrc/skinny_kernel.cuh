@@ -103,20 +103,31 @@ __device__ __forceinline__ void store_16(void* base, int64_t i, float v) {
     reinterpret_cast<__half*>(base)[i] = __float2half_rn(v);
 }
 
+// DRELU_BGRAD: the mask words of rows t0 .. t0+15 for this warp's 32
+// features (one word per row). Callers load them ahead of use -- before the
+// accumulator wait, or before the previous rows' stores -- so the loads are
+// in flight while other work proceeds.
+struct Mask16 {
+  uint32_t m[16];
+};
+
+__device__ __forceinline__ Mask16 skinny_mask16(const SkinnyParams& p, int t0, int word) {
+  Mask16 r;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const int t = t0 + j;
+    r.m[j] = (t < p.T && word < p.aux_words) ? __ldg(p.aux_in + static_cast<int64_t>(t) * p.aux_words + word) : 0u;
+  }
+  return r;
+}
+
 // Epilogue of 16 rows t = t0 .. t0+15 of one feature n (this thread).
 template <int EPI, bool BF16>
 __device__ __forceinline__ void skinny_finish16(const SkinnyParams& p, float (&v)[16], int t0, int n, bool n_ok,
-                                                int word, float bias_n, float& dbias_acc) {
+                                                int word, float bias_n, float& dbias_acc, const Mask16& mk) {
   const uint32_t lane = lane_id();
   if constexpr (EPI == EPI_DRELU_BGRAD) {
-    // all 16 mask words first: loads placed after a store could not be
-    // moved above it (the pointers might alias), each would cost a round trip
-    uint32_t m[16];
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const int t = t0 + j;
-      m[j] = (t < p.T && word < p.aux_words) ? __ldg(p.aux_in + static_cast<int64_t>(t) * p.aux_words + word) : 0u;
-    }
+    const uint32_t* m = mk.m;
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       const int t = t0 + j;
@@ -161,6 +172,11 @@ __device__ __forceinline__ void skinny_fixup(const SkinnyParams& p, const float*
 #pragma unroll 1
   for (int t0 = 0; t0 < TP; t0 += RB) {
     if (t0 >= p.T) break;
+    Mask16 mk[RB / 16];
+    if constexpr (EPI == EPI_DRELU_BGRAD) {
+#pragma unroll
+      for (int h = 0; h < RB / 16; ++h) mk[h] = skinny_mask16(p, t0 + h * 16, word);
+    }
     float v[RB];
 #pragma unroll
     for (int j = 0; j < RB; ++j) v[j] = 0.f;
@@ -188,7 +204,7 @@ __device__ __forceinline__ void skinny_fixup(const SkinnyParams& p, const float*
       float w[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) w[j] = v[h * 16 + j];
-      skinny_finish16<EPI, BF16>(p, w, t0 + h * 16, n, n_ok, word, bias_n, dbias_acc);
+      skinny_finish16<EPI, BF16>(p, w, t0 + h * 16, n, n_ok, word, bias_n, dbias_acc, mk[h]);
     }
   }
 }
@@ -355,6 +371,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         bias_n = n_ok ? load_16<BF16>(p.bias, n) : 0.f;
       float dbias_acc = 0.f;
       const bool whole = s.kb0 == 0 && s.kb1 == p.kbt;
+      Mask16 mk{};
+      if constexpr (EPI == EPI_DRELU_BGRAD)
+        if (whole) mk = skinny_mask16(p, 0, word);  // in flight during the accumulator wait
       if (ok) ok = wait_bounded(&tfull[buf], tph, wp, abort_flag, 6);
       ok = __all_sync(0xffffffffu, ok);
       const uint32_t tbase = tmem_base + ((ew * 32u) << 16) + buf * TP;
@@ -364,6 +383,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
         for (int c = 0; c < TP / 16; ++c) {
           if (c * 16 >= p.T) break;  // warp-uniform
+          Mask16 mk_next{};
+          if constexpr (EPI == EPI_DRELU_BGRAD)
+            if (whole && (c + 1) * 16 < p.T) mk_next = skinny_mask16(p, (c + 1) * 16, word);
           uint32_t r[16];
           tmem_ld_32x32b_x16(tbase + c * 16, r);
           tmem_wait_ld();
@@ -371,7 +393,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
           if (whole) {
-            skinny_finish16<EPI, BF16>(p, v, c * 16, n, n_ok, word, bias_n, dbias_acc);
+            skinny_finish16<EPI, BF16>(p, v, c * 16, n, n_ok, word, bias_n, dbias_acc, mk);
+            mk = mk_next;
           } else {
 #pragma unroll
             for (int j = 0; j < 16; ++j)

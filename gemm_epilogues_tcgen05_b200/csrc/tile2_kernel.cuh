@@ -198,6 +198,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       float* bs = bias_s + buf * BN;
       float* cp = colp_s + buf * 4 * BN;
       epi_stage_bias<BN, EPI, BF16>(p, n0, bs, et);
+      MaskWords<BN> mw{};
+      if constexpr (EPI == EPI_DRELU_BGRAD) mw = load_mask_words<BN>(p, m0 + static_cast<int>(ew * 32 + lane), n0);
       named_bar_sync(1, 128);
       if (ok) ok = wait_bounded(&tfull[buf], tph, p, abort_flag, 6);
       ok = __all_sync(0xffffffffu, ok);
@@ -205,7 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         epi_rows<BN, EPI, BF16>(p, tmem_base + ((ew * 32u) << 16) + buf * BN, m0 + static_cast<int>(ew * 32 + lane), n0,
                                 bs, cp + ew * BN, &tmY, stg, scount, m0 + static_cast<int>(ew * 32), &tmAux,
-                                auxstg_s + ew * kAuxStageBytesPerWarp);
+                                auxstg_s + ew * kAuxStageBytesPerWarp, mw);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(tempty0 + buf * 8);

@@ -177,10 +177,31 @@ struct AuxByTma {
   static constexpr bool value = BN >= 128;
 };
 
+// DRELU_BGRAD: this row's mask words for a tile. The epilogue loads them
+// before it waits for the tile's accumulator, so the loads overlap the MMAs
+// (and no load follows a store it could not be moved above).
+template <int BN>
+struct MaskWords {
+  uint32_t w[BN / 32];
+};
+
+template <int BN>
+__device__ __forceinline__ MaskWords<BN> load_mask_words(const TileParams& p, int row, int n0) {
+  MaskWords<BN> m;
+  const bool row_ok = row < p.T;
+#pragma unroll
+  for (int c = 0; c < BN / 32; ++c) {
+    const int nc0 = n0 + c * 32;
+    m.w[c] = (row_ok && nc0 < p.N) ? __ldg(p.aux_in + static_cast<int64_t>(row) * p.aux_words + (nc0 >> 5)) : 0u;
+  }
+  return m;
+}
+
 template <int BN, int EPI, bool BF16>
 __device__ __forceinline__ void epi_rows(const TileParams& p, uint32_t tbase, int row, int n0, const float* bs,
                                          float* cpw, const CUtensorMap* tmY, uint8_t* stg, uint32_t& scount,
-                                         int wrow0, const CUtensorMap* tmAux, uint8_t* auxstg) {
+                                         int wrow0, const CUtensorMap* tmAux, uint8_t* auxstg,
+                                         const MaskWords<BN>& mw) {
   const uint32_t lane = lane_id();
   const bool row_ok = row < p.T;
   constexpr bool kAuxTma = EPI == EPI_RELU_AUX_BIAS && AuxByTma<BN>::value;
@@ -188,16 +209,6 @@ __device__ __forceinline__ void epi_rows(const TileParams& p, uint32_t tbase, in
   if constexpr (kAuxTma) {
 #pragma unroll
     for (int c = 0; c < BN / 32; ++c) auxw[c] = 0u;
-  }
-  // DRELU: this row's mask words for the whole tile, loaded before any store
-  // (a load after a store could not be moved above it)
-  uint32_t mwords[EPI == EPI_DRELU_BGRAD ? BN / 32 : 1];
-  if constexpr (EPI == EPI_DRELU_BGRAD) {
-#pragma unroll
-    for (int c = 0; c < BN / 32; ++c) {
-      const int nc0 = n0 + c * 32;
-      mwords[c] = (row_ok && nc0 < p.N) ? __ldg(p.aux_in + static_cast<int64_t>(row) * p.aux_words + (nc0 >> 5)) : 0u;
-    }
   }
 #pragma unroll
   for (int c = 0; c < BN / 32; ++c) {
@@ -210,7 +221,7 @@ __device__ __forceinline__ void epi_rows(const TileParams& p, uint32_t tbase, in
 #pragma unroll
     for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
     if constexpr (EPI == EPI_DRELU_BGRAD) {
-      const uint32_t m = mwords[c];
+      const uint32_t m = mw.w[c];
 #pragma unroll
       for (int j = 0; j < 32; ++j) v[j] = ((m >> j) & 1u) ? v[j] : 0.f;
     } else if constexpr (EPI != EPI_STORE) {
@@ -473,6 +484,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       float* bs = bias_s + buf * BN;
       float* cp = colp_s + buf * 4 * BN;
       epi_stage_bias<BN, EPI, BF16>(p, n0, bs, et);
+      MaskWords<BN> mw{};
+      if constexpr (EPI == EPI_DRELU_BGRAD) mw = load_mask_words<BN>(p, m0 + static_cast<int>(ew * 32 + lane), n0);
       named_bar_sync(1, 128);
       if (ok) ok = wait_bounded(&tfull[buf], tph, p, abort_flag, 6);
       ok = __all_sync(0xffffffffu, ok);
@@ -480,7 +493,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         epi_rows<BN, EPI, BF16>(p, tmem_base + ((ew * 32u) << 16) + buf * BN, m0 + static_cast<int>(ew * 32 + lane), n0,
                                 bs, cp + ew * BN, &tmY, stg, scount, m0 + static_cast<int>(ew * 32), &tmAux,
-                                auxstg_s + ew * kAuxStageBytesPerWarp);
+                                auxstg_s + ew * kAuxStageBytesPerWarp, mw);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[buf]);

@@ -37,7 +37,7 @@ def _force(monkeypatch, variant):
 
 
 def _expect_variant(info, variant, T):
-    if (variant == "skinny" and T <= 256) or (variant == "pair" and T < 256):
+    if (variant == "skinny" and T <= 256) or (variant == "pair" and T <= 128):
         assert info["kernel"] == 1
     elif variant == "pair":
         assert info["kernel"] == 2
