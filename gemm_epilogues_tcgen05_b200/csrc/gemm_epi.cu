@@ -255,11 +255,13 @@ struct gemm_epi_plan_s {
   TileCfg cfg_store; // unfused GEMM (plain store)
   float* partials = nullptr;  // DRELU_BGRAD: m_tiles x N
   size_t partial_bytes = 0;
-  int* col_tickets = nullptr;  // DRELU_BGRAD on the tile kernels: n_tiles counters
+  int* col_tickets = nullptr;  // DRELU_BGRAD on the tile kernels: n_tickets counters
+  int n_tickets = 0;
   int* status_host = nullptr;
   int* status_dev = nullptr;
   uint64_t timeout_ns = 0;
   int inject_stall = 0;  // GEMM_EPI_INJECT_STALL at plan time (watchdog tests)
+  int tail_split = 1;    // GEMM_EPI_TAIL_SPLIT=0 keeps whole tiles in the pair kernel's last round
   // tensor-map cache
   const void* a_ptr = nullptr;
   const void* b_ptr = nullptr;
@@ -293,7 +295,7 @@ int take_status(gemm_epi_plan_s* p) {
     *s = 0;
     // an interrupted launch may have left split-tile tickets counted
     if (p->sk_tickets) cudaMemset(p->sk_tickets, 0, sizeof(int) * (size_t)ceil_div(p->N, 128));
-    if (p->col_tickets) cudaMemset(p->col_tickets, 0, sizeof(int) * (size_t)p->n_tiles);
+    if (p->col_tickets) cudaMemset(p->col_tickets, 0, sizeof(int) * (size_t)p->n_tickets);
     return fail(GEMM_EPI_ERR_TIMEOUT, "a kernel of this plan gave up waiting (watchdog code 0x%x)", v);
   }
   return GEMM_EPI_OK;
@@ -327,6 +329,7 @@ ge::TileParams base_params(const gemm_epi_plan_s* p) {
   k.status = p->status_dev;
   k.timeout_ns = p->timeout_ns;
   k.inject_stall = p->inject_stall;
+  k.tail_split = p->tail_split;
   return k;
 }
 
@@ -519,6 +522,7 @@ gemm_epi_plan_t gemm_epi_plan(int64_t T, int64_t N, int64_t K, gemm_epi_dtype dt
   // MMA warp withholds its first tile's completion signal, so the epilogue's
   // bounded wait runs out and the kernel reports ERR_TIMEOUT.
   if (const char* f = getenv("GEMM_EPI_INJECT_STALL")) p->inject_stall = atoi(f) != 0;
+  if (const char* f = getenv("GEMM_EPI_TAIL_SPLIT")) p->tail_split = atoi(f) != 0;
 
   auto cleanup = [&](int rc) {
     if (p->col_tickets) cudaFree(p->col_tickets);
@@ -590,9 +594,10 @@ gemm_epi_plan_t gemm_epi_plan(int64_t T, int64_t N, int64_t K, gemm_epi_dtype dt
     e = cudaMalloc((void**)&p->partials, p->partial_bytes);
     if (e != cudaSuccess) return cleanup(cuda_fail(e, "cudaMalloc(workspace)"));
     if (p->kernel != 1) {  // the tile kernels finish dbias themselves (last ticket per column block)
-      e = cudaMalloc((void**)&p->col_tickets, sizeof(int) * (size_t)p->n_tiles);
+      p->n_tickets = p->kernel == 2 ? 2 * p->n_tiles : p->n_tiles;  // pair kernel: 128-column half blocks
+      e = cudaMalloc((void**)&p->col_tickets, sizeof(int) * (size_t)p->n_tickets);
       if (e != cudaSuccess) return cleanup(cuda_fail(e, "cudaMalloc(column tickets)"));
-      e = cudaMemset(p->col_tickets, 0, sizeof(int) * (size_t)p->n_tiles);
+      e = cudaMemset(p->col_tickets, 0, sizeof(int) * (size_t)p->n_tickets);
       if (e != cudaSuccess) return cleanup(cuda_fail(e, "cudaMemset(column tickets)"));
     }
   }
@@ -651,7 +656,7 @@ int gemm_epi_query(gemm_epi_plan_t plan, gemm_epi_info* info) {
     info->split_k = 1;
     info->grid = p->grid;
     info->launches = 1;
-    info->workspace_bytes = p->epilog == GEMM_EPI_DRELU_BGRAD ? p->partial_bytes + sizeof(int) * (size_t)p->n_tiles : 0;
+    info->workspace_bytes = p->epilog == GEMM_EPI_DRELU_BGRAD ? p->partial_bytes + sizeof(int) * (size_t)p->n_tickets : 0;
   }
   return GEMM_EPI_OK;
 }

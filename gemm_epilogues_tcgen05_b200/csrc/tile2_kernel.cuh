@@ -20,6 +20,10 @@
 //   tempty[b] (leader's) eight arrivals: four epilogue warps of each CTA,
 //             the peer's through its shared::cluster address
 // No load uses TMA multicast. Every wait is bounded as in the 1-CTA kernel.
+//
+// Tail split: when the tiles left for the last round fill at most half of
+// the pairs, each of them is processed as two 128-column halves (MMA N =
+// 128), so the last round takes half a tile's time instead of a whole one.
 #pragma once
 
 #include "tile_kernel.cuh"
@@ -44,6 +48,35 @@ struct Tile2Smem {
   static constexpr uint32_t BYTES = END + 1024;
 };
 
+// Work unit u of the pair schedule: a whole tile, or (in the split tail) one
+// column half of a tile.
+struct PairUnit {
+  int mb, nb;
+  int half;  // -1 for a whole tile, else 0 or 1
+};
+
+struct PairSchedule {
+  int num_tiles, full_units, num_units;
+  __device__ __forceinline__ PairSchedule(int tiles, int npairs, bool allow_split) {
+    num_tiles = tiles;
+    const int tail = tiles % npairs;
+    const bool split = allow_split && tail > 0 && 2 * tail <= npairs;
+    full_units = split ? tiles - tail : tiles;
+    num_units = split ? tiles + tail : tiles;
+  }
+  __device__ __forceinline__ PairUnit unit(int u, int m2_tiles, int n_tiles, int group_m) const {
+    PairUnit r;
+    int t = u;
+    r.half = -1;
+    if (u >= full_units) {
+      t = full_units + (u - full_units) / 2;
+      r.half = (u - full_units) & 1;
+    }
+    tile_coords(t, m2_tiles, n_tiles, group_m, r.mb, r.nb);
+    return r;
+  }
+};
+
 template <int BN, int STAGES, int EPI, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
     tile2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -52,8 +85,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   using L = Tile2Smem<BN, STAGES>;
   static_assert(BN == 128 || BN == 256, "the pair kernel splits BN in 64-column chunks per CTA");
   constexpr uint32_t TMEM_COLS = 2 * BN;
+  static_assert(BN == 256, "the tail split halves 256-column tiles");
   constexpr uint32_t IDESC = idesc_f16(BF16, /*A MN-major*/ false, /*B MN-major*/ true, 2 * kBM, BN);
+  constexpr uint32_t IDESC_HALF = idesc_f16(BF16, false, true, 2 * kBM, BN / 2);
   constexpr uint32_t PAIR_TX = 2 * (L::A_BYTES + L::B_BYTES);
+  constexpr uint32_t PAIR_TX_HALF = 2 * (L::A_BYTES + L::B_CHUNK);
   constexpr uint16_t BOTH = 0x3;
 
   extern __shared__ uint8_t smem_raw[];
@@ -106,7 +142,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int m2_tiles = (p.m_tiles + 1) / 2;  // 256-row tiles
-  const int num_tiles = m2_tiles * p.n_tiles;
+  const PairSchedule sched(m2_tiles * p.n_tiles, npairs, p.tail_split != 0);
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -114,11 +150,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t it = 0;
       bool ok = true;
       const uint32_t full0 = mapa_shared(smem_u32(&full[0]), 0);
-      for (int tile = pair; ok && tile < num_tiles; tile += npairs) {
-        int mb, nb;
-        tile_coords(tile, m2_tiles, p.n_tiles, p.group_m, mb, nb);
-        const int m0 = mb * 2 * kBM + static_cast<int>(rank) * kBM;
-        const int nh0 = nb * BN + static_cast<int>(rank) * (BN / 2);
+      for (int u = pair; ok && u < sched.num_units; u += npairs) {
+        const PairUnit w = sched.unit(u, m2_tiles, p.n_tiles, p.group_m);
+        const int m0 = w.mb * 2 * kBM + static_cast<int>(rank) * kBM;
+        // this CTA's columns: half of the tile (two 64-wide chunks), or half of a half (one chunk)
+        const int nchunks = w.half < 0 ? BN / 128 : 1;
+        const int nh0 = w.nb * BN + (w.half < 0 ? 0 : w.half * (BN / 2)) + static_cast<int>(rank) * nchunks * 64;
         for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
           const uint32_t s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
@@ -126,11 +163,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          if (rank == 0) mbar_arrive_expect_tx(&full[s], PAIR_TX);
+          if (rank == 0) mbar_arrive_expect_tx(&full[s], w.half < 0 ? PAIR_TX : PAIR_TX_HALF);
           const uint32_t fbar = full0 + s * 8;  // the leader's full[s]
           tma_load_2d_pair(sA + s * L::A_BYTES, &tmA, fbar, kb * kBK, m0);
-#pragma unroll
-          for (int j = 0; j < BN / 128; ++j)
+          for (int j = 0; j < nchunks; ++j)
             tma_load_2d_pair(sB + s * L::B_BYTES + j * L::B_CHUNK, &tmB, fbar, nh0 + j * 64, kb * kBK);
         }
       }
@@ -146,7 +182,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (rank == 0) {
         uint32_t it = 0, tcount = 0;
         bool ok = true;
-        for (int tile = pair; ok && tile < num_tiles; tile += npairs, ++tcount) {
+        for (int u = pair; ok && u < sched.num_units; u += npairs, ++tcount) {
+          const PairUnit w = sched.unit(u, m2_tiles, p.n_tiles, p.group_m);
+          const uint32_t idesc = w.half < 0 ? IDESC : IDESC_HALF;
           const uint32_t buf = tcount & 1u;
           const uint32_t tph = (tcount >> 1) & 1u;
           if (!wait_bounded(&tempty[buf], tph ^ 1u, p, abort_flag, 3)) break;
@@ -166,7 +204,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kk = 0; kk < kBK / 16; ++kk) {
               const uint64_t adesc = smem_desc_sw128(a0 + kk * 32, 16, 1024);
               const uint64_t bdesc = smem_desc_sw128(b0 + kk * 2048, L::B_CHUNK, 1024);
-              umma_f16_pair(d_tmem, adesc, bdesc, IDESC, (kb | kk) != 0 ? 1u : 0u);
+              umma_f16_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
             }
             umma_commit_pair(&empty[s], BOTH);
           }
@@ -188,16 +226,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t tcount = 0;
     bool ok = true;
     const uint32_t tempty0 = mapa_shared(smem_u32(&tempty[0]), 0);
-    for (int tile = pair; tile < num_tiles; tile += npairs, ++tcount) {
-      int mb, nb;
-      tile_coords(tile, m2_tiles, p.n_tiles, p.group_m, mb, nb);
-      const int prow = mb * 2 + static_cast<int>(rank);  // this CTA's 128-row block
-      const int m0 = prow * kBM, n0 = nb * BN;
+    for (int u = pair; u < sched.num_units; u += npairs, ++tcount) {
+      const PairUnit w = sched.unit(u, m2_tiles, p.n_tiles, p.group_m);
+      const int prow = w.mb * 2 + static_cast<int>(rank);  // this CTA's 128-row block
+      const int m0 = prow * kBM;
+      const int n0 = w.nb * BN + (w.half < 0 ? 0 : w.half * (BN / 2));
+      const int ncols = w.half < 0 ? BN : BN / 2;
       const uint32_t buf = tcount & 1u;
       const uint32_t tph = (tcount >> 1) & 1u;
       float* bs = bias_s + buf * BN;
       float* cp = colp_s + buf * 4 * BN;
-      epi_stage_bias<BN, EPI, BF16>(p, n0, bs, et);
+      epi_stage_bias<BN, EPI, BF16>(p, n0, bs, et, ncols);
       MaskWords<BN> mw{};
       if constexpr (EPI == EPI_DRELU_BGRAD) mw = load_mask_words<BN>(p, m0 + static_cast<int>(ew * 32 + lane), n0);
       named_bar_sync(1, 128);
@@ -207,7 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         epi_rows<BN, EPI, BF16>(p, tmem_base + ((ew * 32u) << 16) + buf * BN, m0 + static_cast<int>(ew * 32 + lane), n0,
                                 bs, cp + ew * BN, &tmY, stg, scount, m0 + static_cast<int>(ew * 32), &tmAux,
-                                auxstg_s + ew * kAuxStageBytesPerWarp, mw);
+                                auxstg_s + ew * kAuxStageBytesPerWarp, mw, ncols, w.half < 0);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(tempty0 + buf * 8);
@@ -215,8 +254,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       if constexpr (EPI == EPI_DRELU_BGRAD) {
         named_bar_sync(1, 128);
         const bool has_row = prow < p.m_tiles;
-        if (ok && has_row) epi_write_partials<BN>(p, prow, n0, cp, et);
-        if (p.col_tickets) epi_finish_dbias<BN>(p, nb, n0, (ok && has_row) ? 1 : 0, et, dflag);
+        if (ok && has_row) epi_write_partials<BN>(p, prow, n0, cp, et, ncols);
+        // tickets count per 128-column half block, so whole tiles and tail halves mix
+        if (p.col_tickets) {
+          const int rows = (ok && has_row) ? 1 : 0;
+          if (w.half < 0) {
+            epi_finish_dbias<BN>(p, 2 * w.nb, n0, rows, et, dflag, BN / 2);
+            epi_finish_dbias<BN>(p, 2 * w.nb + 1, n0 + BN / 2, rows, et, dflag, BN / 2);
+          } else {
+            epi_finish_dbias<BN>(p, 2 * w.nb + w.half, n0, rows, et, dflag, BN / 2);
+          }
+        }
       }
     }
     if (lane == 0) bulk_wait_group_all();  // this warp's output stores are complete

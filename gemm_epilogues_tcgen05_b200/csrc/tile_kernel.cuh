@@ -44,6 +44,7 @@ struct TileParams {
   int32_t aux_tma;          // RELU_AUX_BIAS: mask words go out by TMA store (see AuxByTma)
   int* col_tickets;         // DRELU_BGRAD: per column block, zero between launches; null = no in-kernel finish
   float* dbias;             // DRELU_BGRAD: written by the tile that takes a column block's last ticket
+  int32_t tail_split;       // pair kernel: split the last round's tiles into column halves
 };
 
 constexpr int kBM = 128;
@@ -156,9 +157,9 @@ __device__ __forceinline__ void warp_transpose_reduce32(float (&v)[32]) {
 
 // Stage the tile's bias values (fp32) in shared memory.
 template <int BN, int EPI, bool BF16>
-__device__ __forceinline__ void epi_stage_bias(const TileParams& p, int n0, float* bs, uint32_t et) {
+__device__ __forceinline__ void epi_stage_bias(const TileParams& p, int n0, float* bs, uint32_t et, int ncols = BN) {
   if constexpr (EPI == EPI_BIAS || EPI == EPI_RELU_BIAS || EPI == EPI_RELU_AUX_BIAS) {
-    for (int c = et; c < BN; c += 128) {
+    for (int c = et; c < ncols; c += 128) {
       const int n = n0 + c;
       bs[c] = n < p.N ? load_16<BF16>(p.bias, n) : 0.f;
     }
@@ -201,10 +202,11 @@ template <int BN, int EPI, bool BF16>
 __device__ __forceinline__ void epi_rows(const TileParams& p, uint32_t tbase, int row, int n0, const float* bs,
                                          float* cpw, const CUtensorMap* tmY, uint8_t* stg, uint32_t& scount,
                                          int wrow0, const CUtensorMap* tmAux, uint8_t* auxstg,
-                                         const MaskWords<BN>& mw) {
+                                         const MaskWords<BN>& mw, int ncols = BN, bool aux_block = true) {
   const uint32_t lane = lane_id();
   const bool row_ok = row < p.T;
   constexpr bool kAuxTma = EPI == EPI_RELU_AUX_BIAS && AuxByTma<BN>::value;
+  const bool aux_by_tma = kAuxTma && p.aux_tma && aux_block;  // a tile narrower than BN stores its words directly
   uint32_t auxw[kAuxTma ? BN / 32 : 1];
   if constexpr (kAuxTma) {
 #pragma unroll
@@ -213,7 +215,7 @@ __device__ __forceinline__ void epi_rows(const TileParams& p, uint32_t tbase, in
 #pragma unroll
   for (int c = 0; c < BN / 32; ++c) {
     const int nc0 = n0 + c * 32;
-    if (nc0 >= p.N) break;  // warp-uniform
+    if (nc0 >= p.N || c * 32 >= ncols) break;  // warp-uniform
     uint32_t r[32];
     tmem_ld_32x32b_x32(tbase + c * 32, r);
     tmem_wait_ld();
@@ -238,7 +240,7 @@ __device__ __forceinline__ void epi_rows(const TileParams& p, uint32_t tbase, in
         if constexpr (EPI == EPI_RELU_AUX_BIAS) {
           const int valid = p.N - nc0;
           if (valid < 32) m &= (1u << valid) - 1u;
-          if (kAuxTma && p.aux_tma)
+          if (aux_by_tma)
             auxw[kAuxTma ? c : 0] = m;
           else if (row_ok)
             p.aux_out[static_cast<int64_t>(row) * p.aux_words + (nc0 >> 5)] = m;
@@ -278,7 +280,7 @@ __device__ __forceinline__ void epi_rows(const TileParams& p, uint32_t tbase, in
       cpw[c * 32 + lane] = v[0];
     }
   }
-  if (kAuxTma && p.aux_tma) {
+  if (aux_by_tma) {
     // row `lane` of the warp's [32][BN/32] word block; the previous tile's
     // block was read by its store before any later chunk's wait returned
     constexpr int WB = BN / 32 * 4;  // bytes per row
@@ -297,8 +299,9 @@ __device__ __forceinline__ void epi_rows(const TileParams& p, uint32_t tbase, in
 // DRELU_BGRAD: combine the four warps' column sums (rows in lane-quarter
 // order) into the partial row `prow` of the workspace.
 template <int BN>
-__device__ __forceinline__ void epi_write_partials(const TileParams& p, int prow, int n0, const float* cp, uint32_t et) {
-  for (int c = et; c < BN; c += 128) {
+__device__ __forceinline__ void epi_write_partials(const TileParams& p, int prow, int n0, const float* cp, uint32_t et,
+                                                   int ncols = BN) {
+  for (int c = et; c < ncols; c += 128) {
     const int n = n0 + c;
     if (n < p.N)
       p.partials[static_cast<int64_t>(prow) * p.N + n] = ((cp[0 * BN + c] + cp[1 * BN + c]) + cp[2 * BN + c]) + cp[3 * BN + c];
@@ -313,7 +316,7 @@ __device__ __forceinline__ void epi_write_partials(const TileParams& p, int prow
 // epilogue threads; `flag` is a shared-memory word.
 template <int BN>
 __device__ __forceinline__ void epi_finish_dbias(const TileParams& p, int nb, int n0, int rows, uint32_t et,
-                                                 volatile int* flag) {
+                                                 volatile int* flag, int ncols = BN) {
   __threadfence();
   named_bar_sync(1, 128);
   if (et == 0) {
@@ -325,7 +328,7 @@ __device__ __forceinline__ void epi_finish_dbias(const TileParams& p, int nb, in
   named_bar_sync(1, 128);
   if (*flag) {
     __threadfence();
-    for (int c = et; c < BN; c += 128) {
+    for (int c = et; c < ncols; c += 128) {
       const int n = n0 + c;
       if (n < p.N) {
         float s = 0.f;

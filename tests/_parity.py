@@ -123,7 +123,10 @@ def assert_within(got: np.ndarray, ref: np.ndarray, scale: np.ndarray, rel: floa
                              f"first at {idx}")
 
 
-def check_forward(inp_cpu, epilog, dtype, gpu, rows=None, cols=None, exact=False):
+def check_forward(inp_cpu, epilog, dtype, gpu, rows=None, cols=None, exact=False, stored_xw=False):
+    """Y (and the mask) against the oracle.  ``stored_xw``: the path under test stored X·W in the
+    16-bit output type before adding the bias (the unfused ablation), a second rounding that may
+    add up to u·|X·W|, so the bound gains that term."""
     bits = synth.bits_u16
     ref = oracle.linear_fwd(bits(inp_cpu["X"]), bits(inp_cpu["W"]), bits(inp_cpu["bias"]), odt(dtype), epilog,
                             rows=rows, cols=cols)
@@ -135,7 +138,12 @@ def check_forward(inp_cpu, epilog, dtype, gpu, rows=None, cols=None, exact=False
         expect = torch.from_numpy(ref["Y"]).to(dtype).double().numpy()  # exact Z rounded once
         assert np.array_equal(Ys, expect), f"{epilog}: Y not bit-exact on integer inputs"
     else:
-        assert_within(Ys, ref["Y"], ref["S"], Y_REL, f"{epilog} Y", unit_roundoff(dtype))
+        scale = ref["S"]
+        if stored_xw:
+            b = inp_cpu["bias"].double().numpy()
+            b = b if cols is None else b[cols]
+            scale = scale + (unit_roundoff(dtype) / Y_REL) * np.abs(ref["Z"] - b[None, :])
+        assert_within(Ys, ref["Y"], scale, Y_REL, f"{epilog} Y", unit_roundoff(dtype))
     if epilog != "BIAS":
         assert np.all(Ys >= 0), "ReLU output negative"
     if epilog == "RELU_AUX_BIAS":

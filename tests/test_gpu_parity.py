@@ -21,7 +21,10 @@ SKINNY_SHAPES = [(16, 1032, 2048), (100, 264, 1000), (256, 4104, 520), (40, 2056
 FWD_EPILOGS = ["BIAS", "RELU_BIAS", "RELU_AUX_BIAS"]
 # CTA-pair shapes: T not a multiple of 256 (the peer CTA's rows partly or
 # wholly past T), N not a multiple of 256 (the peer's columns past N)
-PAIR_SHAPES = [(300, 264, 136), (600, 520, 328), (1000, 1032, 264), (257, 8, 64), (600, 1024, 328)]
+PAIR_SHAPES = [(300, 264, 136), (600, 520, 328), (1000, 1032, 264), (257, 8, 64), (600, 1024, 328),
+               # more than one wave of pair tiles (74 pairs): the last round's tiles are split
+               # into column halves; ragged T and N, one with mask words by TMA store
+               (1000, 5000, 72), (1024, 5120, 64)]
 # kernel variants: the tile kernel at each width, the few-row kernel and the
 # CTA-pair tile kernel
 VARIANTS = ["tile64", "tile128", "tile256", "skinny", "pair"]
@@ -96,7 +99,7 @@ def test_pair_kernel_ragged(monkeypatch, T, N, K, dtype):
         check_backward(inp, fwd["aux"], DT[dtype], gpu)
     assert torch.equal(outs[0]["dbias"], outs[1]["dbias"])
     for ep in FWD_EPILOGS:
-        check_forward(inp, ep, DT[dtype], run_forward(inp, ep, DT[dtype], unfused=True))
+        check_forward(inp, ep, DT[dtype], run_forward(inp, ep, DT[dtype], unfused=True), stored_xw=True)
 
 
 @pytest.mark.parametrize("dtype", ["fp16", "bf16"])
@@ -153,7 +156,7 @@ def test_unfused_path_matches_oracle(dtype):
     inp = synth.make_shape_inputs(T, N, K, dtype, seed=31, D2=D2)
     for ep in FWD_EPILOGS:
         gpu = run_forward(inp, ep, DT[dtype], unfused=True)
-        check_forward(inp, ep, DT[dtype], gpu)
+        check_forward(inp, ep, DT[dtype], gpu, stored_xw=True)
     fwd = run_forward(inp, "RELU_AUX_BIAS", DT[dtype])
     gpu = run_backward(inp, fwd["aux"], DT[dtype], unfused=True)
     check_backward(inp, fwd["aux"], DT[dtype], gpu)
