@@ -175,39 +175,59 @@ int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
 
 using SkinnyKernelFn = void (*)(CUtensorMap, CUtensorMap, ge::SkinnyParams);
 
-template <int TP, bool BF>
+template <int TP, int KPS, bool BF>
 SkinnyKernelFn pick_skinny_epi(int epi) {
   switch (epi) {
-    case ge::EPI_BIAS: return ge::skinny_kernel<TP, ge::EPI_BIAS, BF>;
-    case ge::EPI_RELU_BIAS: return ge::skinny_kernel<TP, ge::EPI_RELU_BIAS, BF>;
-    case ge::EPI_RELU_AUX_BIAS: return ge::skinny_kernel<TP, ge::EPI_RELU_AUX_BIAS, BF>;
-    default: return ge::skinny_kernel<TP, ge::EPI_DRELU_BGRAD, BF>;
+    case ge::EPI_BIAS: return ge::skinny_kernel<TP, KPS, ge::EPI_BIAS, BF>;
+    case ge::EPI_RELU_BIAS: return ge::skinny_kernel<TP, KPS, ge::EPI_RELU_BIAS, BF>;
+    case ge::EPI_RELU_AUX_BIAS: return ge::skinny_kernel<TP, KPS, ge::EPI_RELU_AUX_BIAS, BF>;
+    default: return ge::skinny_kernel<TP, KPS, ge::EPI_DRELU_BGRAD, BF>;
   }
 }
 
 struct SkinnyCfg {
   int TP = 16;
+  int KPS = 1;  // 64-deep k-blocks per pipeline stage
   SkinnyKernelFn fn = nullptr;
   uint32_t smem = 0;
   int stages = 0;
 };
 
-template <int TP>
-SkinnyCfg skinny_cfg_tp(int epi, bool bf16) {
+template <int TP, int KPS>
+SkinnyCfg skinny_cfg_kps(int epi, bool bf16) {
   SkinnyCfg c;
   c.TP = TP;
-  c.fn = bf16 ? pick_skinny_epi<TP, true>(epi) : pick_skinny_epi<TP, false>(epi);
-  c.smem = ge::SkinnySmem<TP>::BYTES;
-  c.stages = ge::SkinnySmem<TP>::STAGES;
+  c.KPS = KPS;
+  c.fn = bf16 ? pick_skinny_epi<TP, KPS, true>(epi) : pick_skinny_epi<TP, KPS, false>(epi);
+  c.smem = ge::SkinnySmem<TP, KPS>::BYTES;
+  c.stages = ge::SkinnySmem<TP, KPS>::STAGES;
   return c;
 }
 
+template <int TP>
+SkinnyCfg skinny_cfg_tp(int epi, bool bf16, int kps) {
+  if (kps >= 2) return skinny_cfg_kps<TP, 2>(epi, bf16);
+  return skinny_cfg_kps<TP, 1>(epi, bf16);
+}
+
+// Two k-blocks per stage (W stages of 32 KB) while X's share of a stage is
+// small: at T = 1 and 8 (N = 11008, K = 4096) 26.7 us against 28.7 us with
+// one; at T = 33..64 the two tie and at T = 128 one k-block per stage (7
+// stages against 3) is faster (35.7 against 38.8 us). Four per stage never
+// beat two.
+int default_kps(int64_t T) { return T <= 32 ? 2 : 1; }
+
 SkinnyCfg skinny_cfg(int64_t T, int epi, bool bf16) {
-  if (T <= 16) return skinny_cfg_tp<16>(epi, bf16);
-  if (T <= 32) return skinny_cfg_tp<32>(epi, bf16);
-  if (T <= 64) return skinny_cfg_tp<64>(epi, bf16);
-  if (T <= 128) return skinny_cfg_tp<128>(epi, bf16);
-  return skinny_cfg_tp<256>(epi, bf16);
+  int kps = default_kps(T);
+  if (const char* f = getenv("GEMM_EPI_SKINNY_KPS")) {  // tuning override: 1 or 2
+    const int v = atoi(f);
+    if (v == 1 || v == 2) kps = v;
+  }
+  if (T <= 16) return skinny_cfg_tp<16>(epi, bf16, kps);
+  if (T <= 32) return skinny_cfg_tp<32>(epi, bf16, kps);
+  if (T <= 64) return skinny_cfg_tp<64>(epi, bf16, kps);
+  if (T <= 128) return skinny_cfg_tp<128>(epi, bf16, kps);
+  return skinny_cfg_tp<256>(epi, bf16, kps);
 }
 
 // Few-row problems (T <= 256) use the swap-AB stream-K kernel unless
@@ -277,6 +297,8 @@ struct gemm_epi_plan_s {
   size_t sk_bytes = 0;
   const void* xs_ptr = nullptr;
   CUtensorMap tmXs;  // the row operand with a TP-row box
+  const void* ws_ptr = nullptr;
+  CUtensorMap tmWs;  // the weight operand with a 64·KPS-row box
 };
 
 namespace {
@@ -402,10 +424,11 @@ int prepare_skinny_maps(gemm_epi_plan_s* p, const void* A, const void* B) {
     if (rc) return rc;
     p->xs_ptr = A;
   }
-  if (B != p->b_ptr) {
-    int rc = encode_2d(&p->tmB, B, (uint64_t)p->N, (uint64_t)p->K, 64, ge::kBK, "the weight operand");
+  if (B != p->ws_ptr) {  // W in boxes of 64 features x 64·KPS k-rows (the tile kernels' map is tmB)
+    int rc = encode_2d(&p->tmWs, B, (uint64_t)p->N, (uint64_t)p->K, 64, (uint32_t)(ge::kBK * p->sk.KPS),
+                       "the weight operand");
     if (rc) return rc;
-    p->b_ptr = B;
+    p->ws_ptr = B;
   }
   return GEMM_EPI_OK;
 }
@@ -429,7 +452,7 @@ ge::SkinnyParams skinny_params(const gemm_epi_plan_s* p) {
 }
 
 int launch_skinny(const gemm_epi_plan_s* p, const ge::SkinnyParams& k, cudaStream_t s) {
-  p->sk.fn<<<p->sk_grid, ge::kThreads, p->sk.smem, s>>>(p->tmB, p->tmXs, k);
+  p->sk.fn<<<p->sk_grid, ge::kThreads, p->sk.smem, s>>>(p->tmWs, p->tmXs, k);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "few-row kernel launch");
   return GEMM_EPI_OK;
@@ -543,8 +566,9 @@ gemm_epi_plan_t gemm_epi_plan(int64_t T, int64_t N, int64_t K, gemm_epi_dtype dt
     p->kernel = 1;
     p->sk = skinny_cfg(T, (int)epilog, bf16);
     const int n_tiles = ceil_div(N, 128);
-    p->sk_kbt = ceil_div(K, ge::kBK);
+    p->sk_kbt = ceil_div(K, (int64_t)ge::kBK * p->sk.KPS);
     p->sk_total = n_tiles * p->sk_kbt;
+    const int min_stages = 8 / p->sk.KPS;  // at least 512 k per CTA under stream-K
     // every CTA gets at least 8 k-blocks, so a tile is shared by few CTAs
     // With at least half as many feature tiles as SMs (and no more than
     // SMs), every CTA takes whole tiles: no split-tile partials or fixups,
@@ -553,7 +577,7 @@ gemm_epi_plan_t gemm_epi_plan(int64_t T, int64_t N, int64_t K, gemm_epi_dtype dt
     if (n_tiles * 2 >= sms && n_tiles <= sms) {
       p->sk_grid = n_tiles;
     } else {
-      int g = p->sk_total / 8;
+      int g = p->sk_total / min_stages;
       g = g < 1 ? 1 : g;
       p->sk_grid = g < sms ? g : sms;
     }
@@ -642,7 +666,7 @@ int gemm_epi_query(gemm_epi_plan_t plan, gemm_epi_info* info) {
   if (p->kernel == 1) {
     info->tile_m = 128;  // features per tile (the MMA's M)
     info->tile_n = p->sk.TP;  // padded rows (the MMA's N)
-    info->tile_k = ge::kBK;
+    info->tile_k = ge::kBK * p->sk.KPS;  // k per pipeline stage
     info->stages = p->sk.stages;
     info->split_k = p->sk_max_segs;
     info->grid = p->sk_grid;

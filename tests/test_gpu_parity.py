@@ -121,6 +121,32 @@ def test_skinny_split_tiles(monkeypatch, T, N, K, dtype):
     assert torch.equal(outs[0]["dbias"], outs[1]["dbias"])
 
 
+# k per pipeline stage (64·KPS): K ragged against 128, K below one k-block
+# (a stage's second 64-k box wholly past K), stream-K segments
+KPS_SHAPES = [(1, 1032, 200), (16, 1032, 72), (40, 264, 40), (64, 2056, 1000), (128, 1032, 520), (33, 11008, 1096)]
+
+
+@pytest.mark.parametrize("kps", [1, 2])
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+@pytest.mark.parametrize("T,N,K", KPS_SHAPES)
+def test_skinny_stage_depth(monkeypatch, T, N, K, dtype, kps):
+    """Few-row kernel with 1 or 2 k-blocks per stage, every epilog."""
+    monkeypatch.setenv("GEMM_EPI_FORCE_KERNEL", "skinny")
+    monkeypatch.setenv("GEMM_EPI_SKINNY_KPS", str(kps))
+    D2 = max(8, K // 8 * 8 + 8)
+    inp = synth.make_shape_inputs(T, N, K, dtype, seed=11 * T + N + K + kps, D2=D2)
+    for ep in FWD_EPILOGS:
+        gpu = run_forward(inp, ep, DT[dtype])
+        assert gpu["info"]["kernel"] == 1
+        assert gpu["info"]["tile_k"] == 64 * kps
+        check_forward(inp, ep, DT[dtype], gpu)
+    fwd = run_forward(inp, "RELU_AUX_BIAS", DT[dtype])
+    outs = run_backward(inp, fwd["aux"], DT[dtype], repeats=2)
+    for gpu in outs:
+        check_backward(inp, fwd["aux"], DT[dtype], gpu)
+    assert torch.equal(outs[0]["dbias"], outs[1]["dbias"])
+
+
 @pytest.mark.parametrize("dtype", ["fp16", "bf16"])
 @pytest.mark.parametrize("T,N,K,D2", [(130, 72, 64, 40), (257, 520, 128, 96), (64, 8, 8, 8), (16, 1032, 1024, 512),
                                       (300, 1024, 64, 40)])
