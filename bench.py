@@ -65,8 +65,11 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def step_spec(w: synth.Workload):
-    """Which epilogs a step of this workload runs."""
+def step_spec(w: synth.Workload, args=None):
+    """Which epilogs a step of this workload runs. --fwd-epilog GELU_BIAS
+    times that forward alone (the library has no GELU backward)."""
+    if args is not None and getattr(args, "fwd_epilog", None):
+        return args.fwd_epilog, False
     if w.name in ("ffn", "pr1"):
         return "RELU_AUX_BIAS", True
     if w.name == "square":
@@ -163,7 +166,7 @@ class ClockSampler:
 def run_ours(args, w: synth.Workload, rank: int, world: int, dev: torch.device):
     from gemm_epilogues_tcgen05_b200 import Plan, binding
 
-    fwd_epi, has_bwd = step_spec(w)
+    fwd_epi, has_bwd = step_spec(w, args)
     dt = w.torch_dtype
     inp = synth.make_inputs(w, device=dev)
     X, W, b = inp["X"], inp["W"], inp["bias"]
@@ -375,7 +378,7 @@ def run_reference(args, w: synth.Workload):
     """--impl reference: the oracle as it stands, on a bounded row sample per step."""
     import oracle
 
-    fwd_epi, has_bwd = step_spec(w)
+    fwd_epi, has_bwd = step_spec(w, args)
     oracle.build()
     threads = oracle.default_threads()
     inp = synth.make_inputs(w, device="cpu")
@@ -427,11 +430,13 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ablation", action="store_true", help="time the unfused path instead")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fwd-epilog", choices=["BIAS", "RELU_BIAS", "RELU_AUX_BIAS", "GELU_BIAS"], default=None,
+                    help="time this forward epilog alone on the workload's shape instead of its own step")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     w = synth.WORKLOADS[args.workload]
-    fwd_epi, has_bwd = step_spec(w)
+    fwd_epi, has_bwd = step_spec(w, args)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -13,8 +13,9 @@ import os
 import torch
 
 F16, BF16 = 0, 1
-BIAS, RELU_BIAS, RELU_AUX_BIAS, DRELU_BGRAD = 0, 1, 2, 3
-EPILOGS = {"BIAS": BIAS, "RELU_BIAS": RELU_BIAS, "RELU_AUX_BIAS": RELU_AUX_BIAS, "DRELU_BGRAD": DRELU_BGRAD}
+BIAS, RELU_BIAS, RELU_AUX_BIAS, DRELU_BGRAD, GELU_BIAS = 0, 1, 2, 3, 4
+EPILOGS = {"BIAS": BIAS, "RELU_BIAS": RELU_BIAS, "RELU_AUX_BIAS": RELU_AUX_BIAS, "DRELU_BGRAD": DRELU_BGRAD,
+           "GELU_BIAS": GELU_BIAS}
 DTYPES = {torch.float16: F16, torch.bfloat16: BF16}
 
 OK = 0

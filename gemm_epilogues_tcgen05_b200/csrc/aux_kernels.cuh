@@ -51,6 +51,19 @@ __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
   return w;
 }
 
+// Unfused GELU: out = gelu(in), 8 elements per thread (n_vec = T * N / 8).
+template <bool BF16>
+__global__ void gelu_kernel(const uint4* __restrict__ in, uint4* __restrict__ out, int64_t n_vec) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n_vec;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float f[8];
+    unpack8<BF16>(in[i], f);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) f[j] = 0.5f * f[j] * (1.0f + erff(f[j] * 0.70710678118654752f));
+    out[i] = pack8<BF16>(f);
+  }
+}
+
 // Unfused BiasAdd: out[t][n] = in[t][n] + bias[n] (8 elements per thread).
 template <bool BF16>
 __global__ void bias_add_kernel(const uint4* __restrict__ in, const void* __restrict__ bias, uint4* __restrict__ out,

@@ -112,6 +112,12 @@ int encode_aux(CUtensorMap* map, const void* aux, int64_t T, int64_t N, int bn) 
   return GEMM_EPI_OK;
 }
 
+static_assert(static_cast<int>(GEMM_EPI_BIAS) == ge::EPI_BIAS && static_cast<int>(GEMM_EPI_RELU_BIAS) == ge::EPI_RELU_BIAS &&
+                  static_cast<int>(GEMM_EPI_RELU_AUX_BIAS) == ge::EPI_RELU_AUX_BIAS &&
+                  static_cast<int>(GEMM_EPI_DRELU_BGRAD) == ge::EPI_DRELU_BGRAD &&
+                  static_cast<int>(GEMM_EPI_GELU_BIAS) == ge::EPI_GELU_BIAS,
+              "the public epilog values are the kernels' epilog kinds");
+
 template <int BN, int ST, bool BF>
 TileKernelFn pick_epi(int epi) {
   switch (epi) {
@@ -119,6 +125,7 @@ TileKernelFn pick_epi(int epi) {
     case ge::EPI_RELU_BIAS: return ge::tile_kernel<BN, ST, ge::EPI_RELU_BIAS, BF>;
     case ge::EPI_RELU_AUX_BIAS: return ge::tile_kernel<BN, ST, ge::EPI_RELU_AUX_BIAS, BF>;
     case ge::EPI_DRELU_BGRAD: return ge::tile_kernel<BN, ST, ge::EPI_DRELU_BGRAD, BF>;
+    case ge::EPI_GELU_BIAS: return ge::tile_kernel<BN, ST, ge::EPI_GELU_BIAS, BF>;
     default: return ge::tile_kernel<BN, ST, ge::EPI_STORE, BF>;
   }
 }
@@ -137,6 +144,7 @@ TileKernelFn pick_pair_epi(int epi) {
     case ge::EPI_RELU_BIAS: return ge::tile2_kernel<256, 6, ge::EPI_RELU_BIAS, BF>;
     case ge::EPI_RELU_AUX_BIAS: return ge::tile2_kernel<256, 6, ge::EPI_RELU_AUX_BIAS, BF>;
     case ge::EPI_DRELU_BGRAD: return ge::tile2_kernel<256, 6, ge::EPI_DRELU_BGRAD, BF>;
+    case ge::EPI_GELU_BIAS: return ge::tile2_kernel<256, 6, ge::EPI_GELU_BIAS, BF>;
     default: return ge::tile2_kernel<256, 6, ge::EPI_STORE, BF>;
   }
 }
@@ -181,6 +189,7 @@ SkinnyKernelFn pick_skinny_epi(int epi) {
     case ge::EPI_BIAS: return ge::skinny_kernel<TP, KPS, ge::EPI_BIAS, BF>;
     case ge::EPI_RELU_BIAS: return ge::skinny_kernel<TP, KPS, ge::EPI_RELU_BIAS, BF>;
     case ge::EPI_RELU_AUX_BIAS: return ge::skinny_kernel<TP, KPS, ge::EPI_RELU_AUX_BIAS, BF>;
+    case ge::EPI_GELU_BIAS: return ge::skinny_kernel<TP, KPS, ge::EPI_GELU_BIAS, BF>;
     default: return ge::skinny_kernel<TP, KPS, ge::EPI_DRELU_BGRAD, BF>;
   }
 }
@@ -490,7 +499,7 @@ gemm_epi_plan_t gemm_epi_plan(int64_t T, int64_t N, int64_t K, gemm_epi_dtype dt
     fail(GEMM_EPI_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
     return nullptr;
   }
-  if (epilog < GEMM_EPI_BIAS || epilog > GEMM_EPI_DRELU_BGRAD) {
+  if (epilog < GEMM_EPI_BIAS || epilog > GEMM_EPI_GELU_BIAS) {
     fail(GEMM_EPI_ERR_INVALID_ARG, "unknown epilog %d", (int)epilog);
     return nullptr;
   }
@@ -782,7 +791,13 @@ int gemm_epi_unfused_execute(gemm_epi_plan_t plan, const void* X, const void* W,
     ge::bias_add_kernel<true><<<blocks, 256, 0, stream>>>((const uint4*)T1, bias, (uint4*)T2, p->T, (int)p->N);
   else
     ge::bias_add_kernel<false><<<blocks, 256, 0, stream>>>((const uint4*)T1, bias, (uint4*)T2, p->T, (int)p->N);
-  if (p->epilog != GEMM_EPI_BIAS) {
+  if (p->epilog == GEMM_EPI_GELU_BIAS) {
+    const int64_t n_vec = p->T * p->N / 8;
+    if (bf16)
+      ge::gelu_kernel<true><<<blocks, 256, 0, stream>>>((const uint4*)T2, (uint4*)Y, n_vec);
+    else
+      ge::gelu_kernel<false><<<blocks, 256, 0, stream>>>((const uint4*)T2, (uint4*)Y, n_vec);
+  } else if (p->epilog != GEMM_EPI_BIAS) {
     const bool want_aux = p->epilog == GEMM_EPI_RELU_AUX_BIAS;
     auto* in = (const uint16_t*)T2;
     auto* out = (uint16_t*)Y;

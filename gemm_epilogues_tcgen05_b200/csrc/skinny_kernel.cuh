@@ -152,6 +152,7 @@ __device__ __forceinline__ void skinny_finish16(const SkinnyParams& p, float (&v
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       float z = v[j] + bias_n;
+      if constexpr (EPI == EPI_GELU_BIAS) z = gelu_erf(z);
       if constexpr (EPI == EPI_RELU_BIAS || EPI == EPI_RELU_AUX_BIAS) {
         const bool pos = z > 0.f;
         if constexpr (EPI == EPI_RELU_AUX_BIAS) {
@@ -382,7 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool n_ok = n < p.N;
       const int word = (s.tile * 128 + static_cast<int>(ew) * 32) >> 5;
       float bias_n = 0.f;
-      if constexpr (EPI == EPI_BIAS || EPI == EPI_RELU_BIAS || EPI == EPI_RELU_AUX_BIAS)
+      if constexpr (AddsBias<EPI>::value)
         bias_n = n_ok ? load_16<BF16>(p.bias, n) : 0.f;
       float dbias_acc = 0.f;
       const bool whole = s.kb0 == 0 && s.kb1 == p.kbt;

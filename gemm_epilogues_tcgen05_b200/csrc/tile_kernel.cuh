@@ -26,7 +26,26 @@
 
 namespace ge {
 
-enum EpiKind : int { EPI_BIAS = 0, EPI_RELU_BIAS = 1, EPI_RELU_AUX_BIAS = 2, EPI_DRELU_BGRAD = 3, EPI_STORE = 4 };
+// The first five match gemm_epi_epilog; EPI_STORE (plain store of X.W) is the
+// unfused ablation's GEMM.
+enum EpiKind : int {
+  EPI_BIAS = 0,
+  EPI_RELU_BIAS = 1,
+  EPI_RELU_AUX_BIAS = 2,
+  EPI_DRELU_BGRAD = 3,
+  EPI_GELU_BIAS = 4,
+  EPI_STORE = 5
+};
+
+// Epilogs that add the bias.
+template <int EPI>
+struct AddsBias {
+  static constexpr bool value =
+      EPI == EPI_BIAS || EPI == EPI_RELU_BIAS || EPI == EPI_RELU_AUX_BIAS || EPI == EPI_GELU_BIAS;
+};
+
+// GELU(z) = z * Phi(z), Phi the standard normal CDF, through CUDA's erff.
+__device__ __forceinline__ float gelu_erf(float z) { return 0.5f * z * (1.0f + erff(z * 0.70710678118654752f)); }
 
 struct TileParams {
   int32_t T, N, K;
@@ -158,7 +177,7 @@ __device__ __forceinline__ void warp_transpose_reduce32(float (&v)[32]) {
 // Stage the tile's bias values (fp32) in shared memory.
 template <int BN, int EPI, bool BF16>
 __device__ __forceinline__ void epi_stage_bias(const TileParams& p, int n0, float* bs, uint32_t et, int ncols = BN) {
-  if constexpr (EPI == EPI_BIAS || EPI == EPI_RELU_BIAS || EPI == EPI_RELU_AUX_BIAS) {
+  if constexpr (AddsBias<EPI>::value) {
     for (int c = et; c < ncols; c += 128) {
       const int n = n0 + c;
       bs[c] = n < p.N ? load_16<BF16>(p.bias, n) : 0.f;
@@ -229,6 +248,10 @@ __device__ __forceinline__ void epi_rows(const TileParams& p, uint32_t tbase, in
     } else if constexpr (EPI != EPI_STORE) {
 #pragma unroll
       for (int j = 0; j < 32; ++j) v[j] += bs[c * 32 + j];
+      if constexpr (EPI == EPI_GELU_BIAS) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = gelu_erf(v[j]);
+      }
       if constexpr (EPI == EPI_RELU_BIAS || EPI == EPI_RELU_AUX_BIAS) {
         uint32_t m = 0;
 #pragma unroll

@@ -60,12 +60,17 @@ typedef enum { GEMM_EPI_F16 = 0, GEMM_EPI_BF16 = 1 } gemm_epi_dtype;
 
 /* The pages' epilog names ("Fusing bias addition into matrix multiplication
  * with nvmath-python": BIAS, RELU_BIAS, RELU_AUX_BIAS; "nvmath-python fused
- * epilogs for linear layers": DRELU_BGRAD). */
+ * epilogs for linear layers": DRELU_BGRAD; "nvmath-python cuBLASLt bindings
+ * for PyTorch fusion", its list of predefined epilogs: GELU_BIAS, bias then
+ * GELU). The pages do not say which GELU; this library computes the
+ * definition GELU(z) = z * Phi(z) = 0.5 * z * (1 + erf(z / sqrt(2))) in fp32
+ * with CUDA's erff, not the tanh approximation. */
 typedef enum {
   GEMM_EPI_BIAS = 0,          /* Y = X.W + bias                              */
   GEMM_EPI_RELU_BIAS = 1,     /* Y = relu(X.W + bias)                        */
   GEMM_EPI_RELU_AUX_BIAS = 2, /* Y = relu(X.W + bias), aux = mask (Z > 0)    */
-  GEMM_EPI_DRELU_BGRAD = 3    /* dZ = (dY2.W2) masked by aux, dbias = sum_t dZ */
+  GEMM_EPI_DRELU_BGRAD = 3,   /* dZ = (dY2.W2) masked by aux, dbias = sum_t dZ */
+  GEMM_EPI_GELU_BIAS = 4      /* Y = gelu(X.W + bias); aux is ignored         */
 } gemm_epi_epilog;
 
 enum {

@@ -16,6 +16,12 @@ their order and notation:
   RELU_AUX_BIAS also returns the bit-encoded ReLU mask ``relu_aux``.
   "AI inference compiler optimisation: operator fusion", section 3.1: the
   fused kernel sums over K, adds ``bias[col]`` and takes ``max(sum, 0)``.
+* ``gelu`` -- epilog GELU_BIAS, which "nvmath-python cuBLASLt bindings for
+  PyTorch fusion" lists among the predefined epilogs as bias followed by
+  GELU. The page does not say which GELU; the oracle takes the definition
+  GELU(z) = z * Phi(z), Phi the standard normal CDF, i.e.
+  z/2 * (1 + erf(z / sqrt 2)), with scipy's double-precision erf as the
+  library primitive.
 * ``relu_aux_words`` -- the mask's bit layout. The pages call it opaque and
   meant only for the dedicated backward epilog ("nvmath-python fused epilogs
   for linear layers", forward section), so its layout is this library's own
@@ -35,6 +41,7 @@ import os
 import subprocess
 
 import numpy as np
+import scipy.special
 
 F16 = 0
 BF16 = 1
@@ -42,6 +49,7 @@ BF16 = 1
 EPILOG_BIAS = "BIAS"
 EPILOG_RELU_BIAS = "RELU_BIAS"
 EPILOG_RELU_AUX_BIAS = "RELU_AUX_BIAS"
+EPILOG_GELU_BIAS = "GELU_BIAS"
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "oracle.c")
@@ -153,22 +161,30 @@ def relu_aux_bits(words: np.ndarray, N: int) -> np.ndarray:
     return bits.reshape(words.shape[0], -1)[:, :N]
 
 
+def gelu(Z):
+    """GELU(z) = z * Phi(z) = z / 2 * (1 + erf(z / sqrt 2)) in binary64."""
+    Z = np.asarray(Z, dtype=np.float64)
+    return 0.5 * Z * (1.0 + scipy.special.erf(Z / np.sqrt(2.0)))
+
+
 def linear_fwd(X, W, bias, dtype: int, epilog: str, rows=None, cols=None, threads=None):
     """Forward epilogs on X (T x K) and W (K x N) with bias (N).
 
     Returns a dict with
       Z     the pre-activation X.W + bias (fp64, exact up to binary64 rounding)
       S     the error scale sum_k |x w| + |b|
-      Y     Z for BIAS; max(Z, 0) for RELU_BIAS / RELU_AUX_BIAS
+      Y     Z for BIAS; max(Z, 0) for RELU_BIAS / RELU_AUX_BIAS; gelu(Z) for GELU_BIAS
       bits  Z > 0 (strict: a zero pre-activation gives bit 0), for RELU_AUX_BIAS
       aux   the packed words (only when every column was computed)
     """
-    if epilog not in (EPILOG_BIAS, EPILOG_RELU_BIAS, EPILOG_RELU_AUX_BIAS):
+    if epilog not in (EPILOG_BIAS, EPILOG_RELU_BIAS, EPILOG_RELU_AUX_BIAS, EPILOG_GELU_BIAS):
         raise ValueError(f"unknown forward epilog {epilog}")
     Z, S = matmul_bias(X, W, bias, dtype, rows=rows, cols=cols, threads=threads)
     out = {"Z": Z, "S": S}
     if epilog == EPILOG_BIAS:
         out["Y"] = Z.copy()
+    elif epilog == EPILOG_GELU_BIAS:
+        out["Y"] = gelu(Z)
     else:
         out["Y"] = np.maximum(Z, 0.0)
     if epilog == EPILOG_RELU_AUX_BIAS:

@@ -18,7 +18,7 @@ SHAPES = [(1, 8, 8), (5, 40, 24), (130, 72, 136), (200, 264, 200), (257, 520, 32
 # few-row shapes whose feature tiles are split over several CTAs (stream-K
 # segments), with ragged K and N, and one where every CTA owns whole tiles
 SKINNY_SHAPES = [(16, 1032, 2048), (100, 264, 1000), (256, 4104, 520), (40, 2056, 64), (1, 11008, 4096)]
-FWD_EPILOGS = ["BIAS", "RELU_BIAS", "RELU_AUX_BIAS"]
+FWD_EPILOGS = ["BIAS", "RELU_BIAS", "RELU_AUX_BIAS", "GELU_BIAS"]
 # CTA-pair shapes: T not a multiple of 256 (the peer CTA's rows partly or
 # wholly past T), N not a multiple of 256 (the peer's columns past N)
 PAIR_SHAPES = [(300, 264, 136), (600, 520, 328), (1000, 1032, 264), (257, 8, 64), (600, 1024, 328),
@@ -250,6 +250,12 @@ def test_error_paths_on_device():
         assert rc == binding.ERR_EPILOG_MISMATCH
     finally:
         binding.gemm_epi_free(hb)
+
+
+def test_unknown_epilog_values_rejected():
+    for bad in (-1, 5, 99):
+        with pytest.raises(binding.GemmEpiError):
+            binding.gemm_epi_plan(64, 64, 64, binding.F16, bad)
 
 
 def test_injected_workspace_allocation_failure(monkeypatch):

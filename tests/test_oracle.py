@@ -440,3 +440,64 @@ def test_mask_pack_roundtrip(oracle_mod):
         tail = N % 32
         if tail:
             assert np.all(words[:, -1] >> np.uint32(tail) == 0)
+
+
+# ---------------------------------------------------------------- GELU_BIAS
+# Standard normal CDF values from a printed normal table (closed-form
+# constants, not computed by the oracle's own erf); GELU(x) = x * Phi(x).
+PHI_TABLE = {0.5: 0.6914624612740131, 1.0: 0.8413447460685429, 1.5: 0.9331927987311419,
+             2.0: 0.9772498680518208, 3.0: 0.9986501019683699, -1.0: 0.15865525393145707}
+
+
+def pin_gelu(gelu, fwd):
+    fails = []
+    for x, phi in PHI_TABLE.items():
+        if abs(gelu(np.array([x]))[0] - x * phi) > 1e-13 * abs(x):
+            fails.append(f"table {x}")
+    xs = np.array([0.25, 0.7, 1.3, 2.6, 4.0])
+    if np.max(np.abs(gelu(xs) - gelu(-xs) - xs)) > 1e-14:  # z*Phi(z) - (-z)*Phi(-z) = z
+        fails.append("odd part")
+    if gelu(np.array([0.0]))[0] != 0.0 or abs(gelu(np.array([12.0]))[0] - 12.0) > 1e-12 \
+            or not (-1e-20 <= gelu(np.array([-12.0]))[0] <= 0.0):
+        fails.append("limits")
+    # through the forward epilog: X a column of exact fp16 values, W = [[1]], bias 0; then bias 1 on x = 1
+    col = [0.5, 1.0, 2.0, -1.0, 3.0]
+    r = fwd(_bits([[v] for v in col], "fp16"), _bits([[1.0]], "fp16"), _bits([0.0], "fp16"), 0, "GELU_BIAS")
+    want = np.array([[v * PHI_TABLE[v]] for v in col])
+    if np.max(np.abs(r["Y"] - want)) > 1e-13:
+        fails.append("epilog")
+    r = fwd(_bits([[1.0]], "bf16"), _bits([[1.0]], "bf16"), _bits([1.0], "bf16"), 1, "GELU_BIAS")
+    if abs(r["Y"][0, 0] - 2.0 * PHI_TABLE[2.0]) > 1e-13 or r["Z"][0, 0] != 2.0:
+        fails.append("epilog with bias")
+    return fails
+
+
+def test_gelu_pins(oracle_mod):
+    fails = pin_gelu(oracle_mod.gelu, oracle_mod.linear_fwd)
+    assert not fails, fails
+
+
+def test_gelu_planted_mistakes_are_caught(oracle_mod):
+    o = oracle_mod
+    mutants = {
+        "tanh approximation": lambda z: 0.5 * z * (1 + np.tanh(math.sqrt(2 / math.pi) * (z + 0.044715 * z ** 3))),
+        "erf without 1/sqrt2": lambda z: 0.5 * z * (1 + np.vectorize(math.erf)(z)),
+        "no one half": lambda z: z * (1 + np.vectorize(math.erf)(z / math.sqrt(2))),
+        "sign of erf": lambda z: 0.5 * z * (1 - np.vectorize(math.erf)(z / math.sqrt(2))),
+    }
+    for name, g in mutants.items():
+        def fwd(X, W, b, dt, ep, g=g, **kw):
+            r = o.linear_fwd(X, W, b, dt, "BIAS", **kw)
+            r["Y"] = g(r["Z"])
+            return r
+        assert pin_gelu(g, fwd), f"pins did not catch: {name}"
+
+
+def test_gelu_epilog_is_bias_then_gelu(oracle_mod):
+    inp = synth.make_shape_inputs(9, 24, 40, "bf16", seed=41)
+    X, W, b = (synth.bits_u16(inp[k]) for k in ("X", "W", "bias"))
+    rb = oracle_mod.linear_fwd(X, W, b, 1, "BIAS")
+    rg = oracle_mod.linear_fwd(X, W, b, 1, "GELU_BIAS")
+    assert np.array_equal(rg["Z"], rb["Z"]) and np.array_equal(rg["S"], rb["S"])
+    z = rb["Z"]
+    assert np.max(np.abs(rg["Y"] - z * 0.5 * (1 + np.vectorize(math.erf)(z / math.sqrt(2))))) < 1e-15
