@@ -68,6 +68,8 @@ def kernel_source_hash() -> str:
 def step_spec(w: synth.Workload, args=None):
     """Which epilogs a step of this workload runs. --fwd-epilog GELU_BIAS
     times that forward alone (the library has no GELU backward)."""
+    if args is not None and getattr(args, "wgrad", False):
+        return "WGRAD", False
     if args is not None and getattr(args, "fwd_epilog", None):
         return args.fwd_epilog, False
     if w.name in ("ffn", "pr1"):
@@ -87,6 +89,8 @@ def algorithmic(w: synth.Workload, fwd_epi: str, bwd: bool):
     aux_bytes = w.T * math.ceil(w.N / 32) * 4
     f_fwd = 2.0 * w.T * w.N * w.K
     b_fwd = e * (w.T * w.K + w.K * w.N + w.N + w.T * w.N) + (aux_bytes if fwd_epi == "RELU_AUX_BIAS" else 0)
+    if fwd_epi == "WGRAD":  # dW = X^T dZ: reads X and dZ, writes dW
+        b_fwd = e * (w.T * w.K + w.T * w.N + w.K * w.N)
     out = {"fwd": {"flops": f_fwd, "bytes": float(b_fwd)}}
     if bwd:
         f_bwd = 2.0 * w.T * w.N * w.D2
@@ -192,7 +196,14 @@ def run_ours(args, w: synth.Workload, rank: int, world: int, dev: torch.device):
     fwd_aux = aux if fwd_epi == "RELU_AUX_BIAS" else None
 
     # prebuilt C calls: the timed loop does no per-call argument checking
-    if args.ablation:
+    if args.wgrad:  # the weight gradient alone: dW (K x N) = X^T dZ, dZ a stand-in for the backward's
+        fplan.free()
+        dZw = synth.masked_grad(w.T, w.N, w.D2 or w.K, dt, seed=w.seed + 21, device=dev)
+        fplan = Plan(w.T, w.N, w.K, dt, "WGRAD")
+        dW = torch.empty((w.K, w.N), dtype=dt, device=dev)
+        fcall = fplan.wgrad_call(X, dZw, dW, stream)
+        bcall = None
+    elif args.ablation:
         fcall = fplan.unfused_call(X, W, b, T1, T2 if fwd_epi != "BIAS" else Y, Y, fwd_aux, stream)
         bcall = bplan.drelu_bgrad_unfused_call(dY2, W2, aux, G, dZ, dbias, stream) if bplan is not None else None
     else:
@@ -272,7 +283,7 @@ def run_ours(args, w: synth.Workload, rank: int, world: int, dev: torch.device):
         launches_per_step = (2 if fwd_epi == "BIAS" else 3) + (4 if bplan is not None else 0)
 
     # e2e: host buffers (pinned), H2D of the step's inputs, both calls, D2H of every output
-    e2e = run_e2e(args, w, fwd_epi, fplan, bplan, inp, dev, stream) if not args.ablation else None
+    e2e = run_e2e(args, w, fwd_epi, fplan, bplan, inp, dev, stream) if not (args.ablation or args.wgrad) else None
 
     kernel = fplan.info()["kernel"]
     fplan.free()
@@ -410,6 +421,9 @@ def metric_name(w: synth.Workload) -> str:
 
 def config_of(w, fwd_epi, has_bwd, args):
     desc = f"{w.name}: fwd {fwd_epi} T={w.T} K={w.K} N={w.N}"
+    if fwd_epi == "WGRAD":
+        desc = (f"{w.name}: WGRAD dW (K x N) = X^T dZ over T={w.T}, K={w.K} N={w.N}; dZ a seeded stand-in "
+                f"(N(0, D2/N), half zeros)")
     if has_bwd:
         desc += f" + bwd DRELU_BGRAD D2={w.D2}"
     desc += f", {w.dtype}"
@@ -430,6 +444,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ablation", action="store_true", help="time the unfused path instead")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--wgrad", action="store_true",
+                    help="time the weight gradient dW = X^T dZ alone on the workload's shape")
     ap.add_argument("--fwd-epilog", choices=["BIAS", "RELU_BIAS", "RELU_AUX_BIAS", "GELU_BIAS"], default=None,
                     help="time this forward epilog alone on the workload's shape instead of its own step")
     args = ap.parse_args()

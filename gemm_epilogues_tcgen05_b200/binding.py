@@ -13,9 +13,9 @@ import os
 import torch
 
 F16, BF16 = 0, 1
-BIAS, RELU_BIAS, RELU_AUX_BIAS, DRELU_BGRAD, GELU_BIAS = 0, 1, 2, 3, 4
+BIAS, RELU_BIAS, RELU_AUX_BIAS, DRELU_BGRAD, GELU_BIAS, WGRAD = 0, 1, 2, 3, 4, 5
 EPILOGS = {"BIAS": BIAS, "RELU_BIAS": RELU_BIAS, "RELU_AUX_BIAS": RELU_AUX_BIAS, "DRELU_BGRAD": DRELU_BGRAD,
-           "GELU_BIAS": GELU_BIAS}
+           "GELU_BIAS": GELU_BIAS, "WGRAD": WGRAD}
 DTYPES = {torch.float16: F16, torch.bfloat16: BF16}
 
 OK = 0
@@ -30,7 +30,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgemm_epi
 
 EXPORTED = ["gemm_epi_plan", "gemm_epi_execute", "drelu_bgrad_execute", "gemm_epi_free", "gemm_epi_last_error",
             "gemm_epi_query", "gemm_epi_status", "gemm_epi_unfused_execute", "drelu_bgrad_unfused_execute",
-            "drelu_bgrad_execute_noalloc"]
+            "drelu_bgrad_execute_noalloc", "gemm_epi_wgrad_execute"]
 
 NOALLOC_SCRATCH_BYTES = 4 << 20  # GEMM_EPI_NOALLOC_SCRATCH_BYTES
 
@@ -83,6 +83,8 @@ def lib() -> ctypes.CDLL:
         L.drelu_bgrad_unfused_execute.argtypes = [vp] * 8
         L.drelu_bgrad_execute_noalloc.restype = ci
         L.drelu_bgrad_execute_noalloc.argtypes = [i64, i64, i64, ci] + [vp] * 6
+        L.gemm_epi_wgrad_execute.restype = ci
+        L.gemm_epi_wgrad_execute.argtypes = [vp] * 5
         _lib = L
     return _lib
 
@@ -205,6 +207,12 @@ class Plan:
                 _ptr(dbias, (N,), torch.float32, "dbias"))
         _check(lib().drelu_bgrad_execute(self.handle, *args, _stream_ptr(stream)))
 
+    def gemm_epi_wgrad_execute(self, X, dZ, dW, stream=None):
+        """WGRAD plan: dW (K x N) = X^T (T x K)^T . dZ (T x N)."""
+        T, N, K, dt = self.T, self.N, self.K, self.dtype
+        args = (_ptr(X, (T, K), dt, "X"), _ptr(dZ, (T, N), dt, "dZ"), _ptr(dW, (K, N), dt, "dW"))
+        _check(lib().gemm_epi_wgrad_execute(self.handle, *args, _stream_ptr(stream)))
+
     def gemm_epi_unfused_execute(self, X, W, bias, T1, T2, Y, aux=None, stream=None):
         T, N, K, dt = self.T, self.N, self.K, self.dtype
         args = (_ptr(X, (T, K), dt, "X"), _ptr(W, (K, N), dt, "W"), _ptr(bias, (N,), dt, "bias"),
@@ -234,6 +242,12 @@ class Plan:
                 _ptr(dbias, (N,), torch.float32, "dbias"), _stream_ptr(stream))
         return lib().drelu_bgrad_execute, args
 
+    def wgrad_call(self, X, dZ, dW, stream=None):
+        T, N, K, dt = self.T, self.N, self.K, self.dtype
+        args = (self.handle, _ptr(X, (T, K), dt, "X"), _ptr(dZ, (T, N), dt, "dZ"), _ptr(dW, (K, N), dt, "dW"),
+                _stream_ptr(stream))
+        return lib().gemm_epi_wgrad_execute, args
+
     def unfused_call(self, X, W, bias, T1, T2, Y, aux=None, stream=None):
         T, N, K, dt = self.T, self.N, self.K, self.dtype
         args = (self.handle, _ptr(X, (T, K), dt, "X"), _ptr(W, (K, N), dt, "W"), _ptr(bias, (N,), dt, "bias"),
@@ -262,3 +276,8 @@ class Plan:
         dbias = torch.empty((self.N,), dtype=torch.float32, device=dY2.device)
         self.drelu_bgrad_execute(dY2, W2, aux, dZ, dbias, stream)
         return dZ, dbias
+
+    def wgrad(self, X, dZ, stream=None):
+        dW = torch.empty((self.K, self.N), dtype=self.dtype, device=X.device)
+        self.gemm_epi_wgrad_execute(X, dZ, dW, stream)
+        return dW

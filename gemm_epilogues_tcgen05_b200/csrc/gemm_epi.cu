@@ -115,7 +115,8 @@ int encode_aux(CUtensorMap* map, const void* aux, int64_t T, int64_t N, int bn) 
 static_assert(static_cast<int>(GEMM_EPI_BIAS) == ge::EPI_BIAS && static_cast<int>(GEMM_EPI_RELU_BIAS) == ge::EPI_RELU_BIAS &&
                   static_cast<int>(GEMM_EPI_RELU_AUX_BIAS) == ge::EPI_RELU_AUX_BIAS &&
                   static_cast<int>(GEMM_EPI_DRELU_BGRAD) == ge::EPI_DRELU_BGRAD &&
-                  static_cast<int>(GEMM_EPI_GELU_BIAS) == ge::EPI_GELU_BIAS,
+                  static_cast<int>(GEMM_EPI_GELU_BIAS) == ge::EPI_GELU_BIAS &&
+                  static_cast<int>(GEMM_EPI_WGRAD) == ge::EPI_WGRAD,
               "the public epilog values are the kernels' epilog kinds");
 
 template <int BN, int ST, bool BF>
@@ -126,6 +127,7 @@ TileKernelFn pick_epi(int epi) {
     case ge::EPI_RELU_AUX_BIAS: return ge::tile_kernel<BN, ST, ge::EPI_RELU_AUX_BIAS, BF>;
     case ge::EPI_DRELU_BGRAD: return ge::tile_kernel<BN, ST, ge::EPI_DRELU_BGRAD, BF>;
     case ge::EPI_GELU_BIAS: return ge::tile_kernel<BN, ST, ge::EPI_GELU_BIAS, BF>;
+    case ge::EPI_WGRAD: return ge::tile_kernel<BN, ST, ge::EPI_WGRAD, BF>;
     default: return ge::tile_kernel<BN, ST, ge::EPI_STORE, BF>;
   }
 }
@@ -145,6 +147,7 @@ TileKernelFn pick_pair_epi(int epi) {
     case ge::EPI_RELU_AUX_BIAS: return ge::tile2_kernel<256, 6, ge::EPI_RELU_AUX_BIAS, BF>;
     case ge::EPI_DRELU_BGRAD: return ge::tile2_kernel<256, 6, ge::EPI_DRELU_BGRAD, BF>;
     case ge::EPI_GELU_BIAS: return ge::tile2_kernel<256, 6, ge::EPI_GELU_BIAS, BF>;
+    case ge::EPI_WGRAD: return ge::tile2_kernel<256, 6, ge::EPI_WGRAD, BF>;
     default: return ge::tile2_kernel<256, 6, ge::EPI_STORE, BF>;
   }
 }
@@ -276,7 +279,8 @@ bool use_skinny(int64_t T) {
 }  // namespace
 
 struct gemm_epi_plan_s {
-  int64_t T, N, K;
+  int64_t T, N, K;   // the kernels' rows, columns and contraction length
+  int64_t uT, uK;    // the caller's T and K (WGRAD: rows = uK, contraction = uT)
   int dtype, epilog;
   int device, num_sms;
   int m_tiles, n_tiles, k_blocks, num_tiles, aux_words, grid, group_m;
@@ -333,7 +337,12 @@ int take_status(gemm_epi_plan_s* p) {
 }
 
 int prepare_maps(gemm_epi_plan_s* p, const void* A, const void* B) {
-  if (A != p->a_ptr) {
+  if (A != p->a_ptr && p->epilog == GEMM_EPI_WGRAD) {
+    // X (uT x uK) read as the MN-major A = X^T: boxes of 64 features x 64 rows
+    int rc = encode_2d(&p->tmA, A, (uint64_t)p->T, (uint64_t)p->K, 64, ge::kBK, "X");
+    if (rc) return rc;
+    p->a_ptr = A;
+  } else if (A != p->a_ptr) {
     int rc = encode_2d(&p->tmA, A, (uint64_t)p->K, (uint64_t)p->T, ge::kBK, ge::kBM, "the row operand");
     if (rc) return rc;
     p->a_ptr = A;
@@ -499,7 +508,7 @@ gemm_epi_plan_t gemm_epi_plan(int64_t T, int64_t N, int64_t K, gemm_epi_dtype dt
     fail(GEMM_EPI_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
     return nullptr;
   }
-  if (epilog < GEMM_EPI_BIAS || epilog > GEMM_EPI_GELU_BIAS) {
+  if (epilog < GEMM_EPI_BIAS || epilog > GEMM_EPI_WGRAD) {
     fail(GEMM_EPI_ERR_INVALID_ARG, "unknown epilog %d", (int)epilog);
     return nullptr;
   }
@@ -519,7 +528,18 @@ gemm_epi_plan_t gemm_epi_plan(int64_t T, int64_t N, int64_t K, gemm_epi_dtype dt
     return nullptr;
   }
 
+  if (epilog == GEMM_EPI_WGRAD && K * N > ((int64_t)1 << 40)) {
+    fail(GEMM_EPI_ERR_INVALID_ARG, "shape too large for 32-bit tile coordinates");
+    return nullptr;
+  }
   auto* p = new gemm_epi_plan_s();
+  p->uT = T;
+  p->uK = K;
+  if (epilog == GEMM_EPI_WGRAD) {  // dW (K x N) = X^T dZ: K output rows, contraction over the T rows
+    const int64_t rows = K;
+    K = T;
+    T = rows;
+  }
   p->T = T;
   p->N = N;
   p->K = K;
@@ -571,7 +591,7 @@ gemm_epi_plan_t gemm_epi_plan(int64_t T, int64_t N, int64_t K, gemm_epi_dtype dt
     e = cudaFuncSetAttribute(c->fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)c->smem);
     if (e != cudaSuccess) return cleanup(cuda_fail(e, "cudaFuncSetAttribute(max dynamic shared memory)"));
   }
-  if (!pair && use_skinny(T)) {
+  if (!pair && epilog != GEMM_EPI_WGRAD && use_skinny(T)) {
     p->kernel = 1;
     p->sk = skinny_cfg(T, (int)epilog, bf16);
     const int n_tiles = ceil_div(N, 128);
@@ -665,9 +685,9 @@ int gemm_epi_query(gemm_epi_plan_t plan, gemm_epi_info* info) {
   gemm_epi_plan_s* p = lookup(plan);
   if (!p || !info) return fail(GEMM_EPI_ERR_INVALID_ARG, "gemm_epi_query: unknown plan or NULL info");
   memset(info, 0, sizeof(*info));
-  info->T = p->T;
+  info->T = p->uT;
   info->N = p->N;
-  info->K = p->K;
+  info->K = p->uK;
   info->dtype = p->dtype;
   info->epilog = p->epilog;
   info->kernel = p->kernel;
@@ -704,8 +724,9 @@ int gemm_epi_execute(gemm_epi_plan_t plan, const void* X, const void* W, const v
                      cudaStream_t stream) {
   gemm_epi_plan_s* p = lookup(plan);
   if (!p) return fail(GEMM_EPI_ERR_INVALID_ARG, "gemm_epi_execute: unknown plan");
-  if (p->epilog == GEMM_EPI_DRELU_BGRAD)
-    return fail(GEMM_EPI_ERR_EPILOG_MISMATCH, "gemm_epi_execute called on a DRELU_BGRAD plan");
+  if (p->epilog == GEMM_EPI_DRELU_BGRAD || p->epilog == GEMM_EPI_WGRAD)
+    return fail(GEMM_EPI_ERR_EPILOG_MISMATCH, "gemm_epi_execute called on a %s plan",
+                p->epilog == GEMM_EPI_WGRAD ? "WGRAD" : "DRELU_BGRAD");
   if (!X || !W || !bias || !Y) return fail(GEMM_EPI_ERR_INVALID_ARG, "gemm_epi_execute: NULL X, W, bias or Y");
   if (p->epilog == GEMM_EPI_RELU_AUX_BIAS && !aux)
     return fail(GEMM_EPI_ERR_EPILOG_MISMATCH, "RELU_AUX_BIAS needs an aux buffer");
@@ -769,8 +790,8 @@ int gemm_epi_unfused_execute(gemm_epi_plan_t plan, const void* X, const void* W,
                              void* Y, uint32_t* aux, cudaStream_t stream) {
   gemm_epi_plan_s* p = lookup(plan);
   if (!p) return fail(GEMM_EPI_ERR_INVALID_ARG, "gemm_epi_unfused_execute: unknown plan");
-  if (p->epilog == GEMM_EPI_DRELU_BGRAD)
-    return fail(GEMM_EPI_ERR_EPILOG_MISMATCH, "gemm_epi_unfused_execute called on a DRELU_BGRAD plan");
+  if (p->epilog == GEMM_EPI_DRELU_BGRAD || p->epilog == GEMM_EPI_WGRAD)
+    return fail(GEMM_EPI_ERR_EPILOG_MISMATCH, "gemm_epi_unfused_execute called on a backward plan");
   if (!X || !W || !bias || !T1 || !T2 || !Y) return fail(GEMM_EPI_ERR_INVALID_ARG, "unfused: NULL pointer");
   if (p->epilog == GEMM_EPI_RELU_AUX_BIAS && !aux)
     return fail(GEMM_EPI_ERR_EPILOG_MISMATCH, "RELU_AUX_BIAS needs an aux buffer");
@@ -816,6 +837,23 @@ int gemm_epi_unfused_execute(gemm_epi_plan_t plan, const void* X, const void* W,
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "unfused elementwise launch");
   return GEMM_EPI_OK;
+}
+
+int gemm_epi_wgrad_execute(gemm_epi_plan_t plan, const void* X, const void* dZ, void* dW, cudaStream_t stream) {
+  gemm_epi_plan_s* p = lookup(plan);
+  if (!p) return fail(GEMM_EPI_ERR_INVALID_ARG, "gemm_epi_wgrad_execute: unknown plan");
+  if (p->epilog != GEMM_EPI_WGRAD)
+    return fail(GEMM_EPI_ERR_EPILOG_MISMATCH, "gemm_epi_wgrad_execute called on a plan whose epilog is not WGRAD");
+  if (!X || !dZ || !dW) return fail(GEMM_EPI_ERR_INVALID_ARG, "gemm_epi_wgrad_execute: NULL X, dZ or dW");
+  if (!aligned(X, 16) || !aligned(dZ, 16) || !aligned(dW, 16))
+    return fail(GEMM_EPI_ERR_MISALIGNED, "gemm_epi_wgrad_execute: X, dZ, dW need 16-byte alignment");
+  int rc = take_status(p);
+  if (rc) return rc;
+  rc = prepare_maps(p, X, dZ);
+  if (rc) return rc;
+  ge::TileParams k = base_params(p);
+  k.out = dW;
+  return launch_tile(p, p->cfg, k, stream);
 }
 
 int drelu_bgrad_unfused_execute(gemm_epi_plan_t plan, const void* dY2, const void* W2, const uint32_t* aux, void* G,

@@ -86,8 +86,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   static_assert(BN == 128 || BN == 256, "the pair kernel splits BN in 64-column chunks per CTA");
   constexpr uint32_t TMEM_COLS = 2 * BN;
   static_assert(BN == 256, "the tail split halves 256-column tiles");
-  constexpr uint32_t IDESC = idesc_f16(BF16, /*A MN-major*/ false, /*B MN-major*/ true, 2 * kBM, BN);
-  constexpr uint32_t IDESC_HALF = idesc_f16(BF16, false, true, 2 * kBM, BN / 2);
+  constexpr bool A_MN = AOperandMN<EPI>::value;
+  constexpr uint32_t IDESC = idesc_f16(BF16, /*A MN-major*/ A_MN, /*B MN-major*/ true, 2 * kBM, BN);
+  constexpr uint32_t IDESC_HALF = idesc_f16(BF16, A_MN, true, 2 * kBM, BN / 2);
   constexpr uint32_t PAIR_TX = 2 * (L::A_BYTES + L::B_BYTES);
   constexpr uint32_t PAIR_TX_HALF = 2 * (L::A_BYTES + L::B_CHUNK);
   constexpr uint16_t BOTH = 0x3;
@@ -165,7 +166,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (rank == 0) mbar_arrive_expect_tx(&full[s], w.half < 0 ? PAIR_TX : PAIR_TX_HALF);
           const uint32_t fbar = full0 + s * 8;  // the leader's full[s]
-          tma_load_2d_pair(sA + s * L::A_BYTES, &tmA, fbar, kb * kBK, m0);
+          if constexpr (A_MN) {
+            tma_load_2d_pair(sA + s * L::A_BYTES, &tmA, fbar, m0, kb * kBK);
+            tma_load_2d_pair(sA + s * L::A_BYTES + kAChunkMN, &tmA, fbar, m0 + 64, kb * kBK);
+          } else {
+            tma_load_2d_pair(sA + s * L::A_BYTES, &tmA, fbar, kb * kBK, m0);
+          }
           for (int j = 0; j < nchunks; ++j)
             tma_load_2d_pair(sB + s * L::B_BYTES + j * L::B_CHUNK, &tmB, fbar, nh0 + j * 64, kb * kBK);
         }
@@ -202,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t b0 = smem_u32(sB + s * L::B_BYTES);
 #pragma unroll
             for (int kk = 0; kk < kBK / 16; ++kk) {
-              const uint64_t adesc = smem_desc_sw128(a0 + kk * 32, 16, 1024);
+              const uint64_t adesc = a_desc<A_MN>(a0, kk);
               const uint64_t bdesc = smem_desc_sw128(b0 + kk * 2048, L::B_CHUNK, 1024);
               umma_f16_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
             }

@@ -26,7 +26,7 @@
 
 namespace ge {
 
-// The first five match gemm_epi_epilog; EPI_STORE (plain store of X.W) is the
+// The first six match gemm_epi_epilog; EPI_STORE (plain store of X.W) is the
 // unfused ablation's GEMM.
 enum EpiKind : int {
   EPI_BIAS = 0,
@@ -34,8 +34,36 @@ enum EpiKind : int {
   EPI_RELU_AUX_BIAS = 2,
   EPI_DRELU_BGRAD = 3,
   EPI_GELU_BIAS = 4,
-  EPI_STORE = 5
+  EPI_WGRAD = 5,
+  EPI_STORE = 6
 };
+
+// The weight gradient dW = X^T dZ reads its A operand (X^T, M = the features
+// of X) straight from row-major X: M is the contiguous index, so A is
+// MN-major and staged like W, as two 64-wide chunks per 128-row tile.
+template <int EPI>
+struct AOperandMN {
+  static constexpr bool value = EPI == EPI_WGRAD;
+};
+constexpr uint32_t kAChunkMN = 64 * 64 * 2;  // one 64-wide M chunk x 64 k (8 KB)
+
+// Epilogs whose output is the plain rounded accumulator.
+template <int EPI>
+struct PlainStore {
+  static constexpr bool value = EPI == EPI_STORE || EPI == EPI_WGRAD;
+};
+
+// A operand descriptor for K step kk (16 elements) of a stage at a0:
+// K-major: 128-byte rows, 8-row groups 1024 B apart, a K step is 32 bytes
+// inside the swizzle atom; MN-major: 64-wide M chunks 8 KB apart (LBO), 8
+// K-rows 1024 B apart (SBO), a K step is 16 rows = 2048 bytes.
+template <bool A_MN>
+__device__ __forceinline__ uint64_t a_desc(uint32_t a0, int kk) {
+  if constexpr (A_MN)
+    return smem_desc_sw128(a0 + kk * 2048, kAChunkMN, 1024);
+  else
+    return smem_desc_sw128(a0 + kk * 32, 16, 1024);
+}
 
 // Epilogs that add the bias.
 template <int EPI>
@@ -245,7 +273,7 @@ __device__ __forceinline__ void epi_rows(const TileParams& p, uint32_t tbase, in
       const uint32_t m = mw.w[c];
 #pragma unroll
       for (int j = 0; j < 32; ++j) v[j] = ((m >> j) & 1u) ? v[j] : 0.f;
-    } else if constexpr (EPI != EPI_STORE) {
+    } else if constexpr (!PlainStore<EPI>::value) {
 #pragma unroll
       for (int j = 0; j < 32; ++j) v[j] += bs[c * 32 + j];
       if constexpr (EPI == EPI_GELU_BIAS) {
@@ -372,7 +400,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN must be 64, 128, 192 or 256");
   constexpr uint32_t TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
                                  : (2 * BN <= 256) ? 256 : 512;
-  constexpr uint32_t IDESC = idesc_f16(BF16, /*A MN-major*/ false, /*B MN-major*/ true, kBM, BN);
+  constexpr bool A_MN = AOperandMN<EPI>::value;
+  constexpr uint32_t IDESC = idesc_f16(BF16, /*A MN-major*/ A_MN, /*B MN-major*/ true, kBM, BN);
   constexpr uint32_t STAGE_TX = L::A_BYTES + L::B_BYTES;
 
   extern __shared__ uint8_t smem_raw[];
@@ -439,7 +468,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           mbar_arrive_expect_tx(&full[s], STAGE_TX);
-          tma_load_2d(sA + s * L::A_BYTES, &tmA, &full[s], kb * kBK, m0);
+          if constexpr (A_MN) {
+            tma_load_2d(sA + s * L::A_BYTES, &tmA, &full[s], m0, kb * kBK);
+            tma_load_2d(sA + s * L::A_BYTES + kAChunkMN, &tmA, &full[s], m0 + 64, kb * kBK);
+          } else {
+            tma_load_2d(sA + s * L::A_BYTES, &tmA, &full[s], kb * kBK, m0);
+          }
 #pragma unroll
           for (int j = 0; j < BN / 64; ++j)
             tma_load_2d(sB + s * L::B_BYTES + j * L::B_CHUNK, &tmB, &full[s], n0 + j * 64, kb * kBK);
@@ -474,9 +508,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t b0 = smem_u32(sB + s * L::B_BYTES);
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
-            // A: K-major, 128-byte rows, 8-row groups 1024 B apart; a K step of
-            // 16 elements is 32 bytes inside the swizzle atom.
-            const uint64_t adesc = smem_desc_sw128(a0 + kk * 32, 16, 1024);
+            const uint64_t adesc = a_desc<A_MN>(a0, kk);
             // B: N-major, 64-wide N chunks 8 KB apart (LBO), 8 K-rows 1024 B
             // apart (SBO); a K step of 16 rows is 2048 bytes.
             const uint64_t bdesc = smem_desc_sw128(b0 + kk * 2048, L::B_CHUNK, 1024);

@@ -90,6 +90,16 @@ def integers(shape, lo: int, hi: int, dtype, seed: int, device="cpu") -> torch.T
     return x.to(dtype)
 
 
+def masked_grad(T: int, N: int, D2: int, dtype, seed: int, device="cpu") -> torch.Tensor:
+    """A stand-in for the backward's dZ (T x N) with its value distribution:
+    N(0, D2/N) draws (dY2 ~ N(0, 1) against W2 ~ N(0, 1/N), summed over D2),
+    set to zero where a fair coin marks the unit inactive (the ReLU mask of a
+    symmetric pre-activation)."""
+    g = normal((T, N), (D2 / N) ** 0.5, torch.float32, seed, device)
+    keep = torch.rand((T, N), generator=_gen(seed + 1, device), device=device) < 0.5
+    return torch.where(keep, g, torch.zeros_like(g)).to(dtype)
+
+
 def make_inputs(w: Workload, device="cpu", parts=("fwd", "bwd"), T: int | None = None) -> dict:
     """Inputs of one workload: X, W, bias (fwd) and dY2, W2 (bwd).
 

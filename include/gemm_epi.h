@@ -70,7 +70,8 @@ typedef enum {
   GEMM_EPI_RELU_BIAS = 1,     /* Y = relu(X.W + bias)                        */
   GEMM_EPI_RELU_AUX_BIAS = 2, /* Y = relu(X.W + bias), aux = mask (Z > 0)    */
   GEMM_EPI_DRELU_BGRAD = 3,   /* dZ = (dY2.W2) masked by aux, dbias = sum_t dZ */
-  GEMM_EPI_GELU_BIAS = 4      /* Y = gelu(X.W + bias); aux is ignored         */
+  GEMM_EPI_GELU_BIAS = 4,     /* Y = gelu(X.W + bias); aux is ignored         */
+  GEMM_EPI_WGRAD = 5          /* dW = X^T . dZ, see gemm_epi_wgrad_execute    */
 } gemm_epi_epilog;
 
 enum {
@@ -104,7 +105,8 @@ typedef struct {
  *   T >= 1 rows; N >= 8 and K >= 8, both multiples of 8 (16-byte row
  *   strides); dtype and epilog from the enums above. For DRELU_BGRAD, K is
  *   the contraction length D2 of G = dY2 . W2 (a backward plan is separate
- *   from the forward plan, as the pages build a separate matmul for it).
+ *   from the forward plan, as the pages build a separate matmul for it). For
+ *   WGRAD, (T, N, K) are the forward's: dW is K x N, summed over T (any T).
  *   Uses the current CUDA device; allocates the plan's workspace there.
  * Returns a plan, or NULL with gemm_epi_last_error() set.
  */
@@ -136,6 +138,22 @@ GEMM_EPI_API int gemm_epi_execute(gemm_epi_plan_t plan, const void* X, const voi
  */
 GEMM_EPI_API int drelu_bgrad_execute(gemm_epi_plan_t plan, const void* dY2, const void* W2, const uint32_t* aux,
                         void* dZ, float* dbias, cudaStream_t stream);
+
+/*
+ * gemm_epi_wgrad_execute: the weight gradient of the linear layer,
+ * dW[k][n] = sum over t of X[t][k] * dZ[t][n], rounded to dtype. The pages
+ * name no epilog for it: "nvmath-python fused epilogs for linear layers"
+ * (FAQ) says DRELU_BGRAD covers the mask and the bias gradient but not the
+ * whole backward pass; this is the remaining product of that pass, with the
+ * dZ that drelu_bgrad_execute returns. Plan it with epilog GEMM_EPI_WGRAD and
+ * the forward's (T, N, K): the contraction runs over the T rows.
+ *   X (T x K), dZ (T x N), dW (K x N): device, 16-byte aligned, row-major.
+ * Returns as gemm_epi_execute; GEMM_EPI_ERR_EPILOG_MISMATCH on a plan whose
+ * epilog is not WGRAD (and gemm_epi_execute / drelu_bgrad_execute return it
+ * on a WGRAD plan).
+ */
+GEMM_EPI_API int gemm_epi_wgrad_execute(gemm_epi_plan_t plan, const void* X, const void* dZ, void* dW,
+                                        cudaStream_t stream);
 
 /* Release a plan and its workspace. NULL and already-freed plans are
  * ignored. The caller must make sure no work of the plan is still running

@@ -22,6 +22,11 @@ their order and notation:
   GELU(z) = z * Phi(z), Phi the standard normal CDF, i.e.
   z/2 * (1 + erf(z / sqrt 2)), with scipy's double-precision erf as the
   library primitive.
+* ``wgrad`` -- the weight gradient dW = X^T . dZ of the linear layer, the
+  part of the backward pass that "nvmath-python fused epilogs for linear
+  layers" (FAQ) says DRELU_BGRAD does not cover. The plain definition:
+  dW[k, n] = sum_t X[t, k] * dZ[t, n], i.e. the contraction above applied to
+  the transposed X.
 * ``relu_aux_words`` -- the mask's bit layout. The pages call it opaque and
   meant only for the dedicated backward epilog ("nvmath-python fused epilogs
   for linear layers", forward section), so its layout is this library's own
@@ -192,6 +197,22 @@ def linear_fwd(X, W, bias, dtype: int, epilog: str, rows=None, cols=None, thread
         if cols is None:
             out["aux"] = relu_aux_words(out["bits"])
     return out
+
+
+def wgrad(X, dZ, dtype: int, rows=None, cols=None, threads=None):
+    """dW = X^T . dZ for X (T x K) and dZ (T x N): K x N, summed over t.
+
+    Returns a dict with
+      dW    the product (fp64)
+      S     sum_t |x dz|, its error scale
+    ``rows`` / ``cols`` select rows k / columns n of dW.
+    """
+    X = np.asarray(X, dtype=np.uint16)
+    dZ = np.asarray(dZ, dtype=np.uint16)
+    if X.shape[0] != dZ.shape[0]:
+        raise ValueError(f"X and dZ need the same row count: {X.shape[0]} vs {dZ.shape[0]}")
+    dW, S = matmul_bias(np.ascontiguousarray(X.T), dZ, None, dtype, rows=rows, cols=cols, threads=threads)
+    return {"dW": dW, "S": S}
 
 
 def drelu_bgrad(dY2, W2, aux, dtype: int, N: int, rows=None, cols=None, threads=None):

@@ -214,3 +214,32 @@ def assert_dbias_is_column_sum(dbias, dZ, dtype):
     err = np.abs(dbias.double().numpy() - col)
     bound = (DBIAS_REL + unit_roundoff(dtype)) * mag
     assert np.all(err <= bound), f"dbias is not the column sum of dZ: worst {np.max(err / np.maximum(bound, 1e-300)):.3g}"
+
+
+def run_wgrad(inp_cpu: dict, dtype, device="cuda", dz_key="dY2"):
+    """dW = X^T dZ through the WGRAD plan; dZ is the T x N tensor under ``dz_key``."""
+    X, dZ = inp_cpu["X"].to(device), inp_cpu[dz_key].to(device)
+    T, K = X.shape
+    N = dZ.shape[1]
+    with Plan(T, N, K, dtype, "WGRAD") as plan:
+        info = plan.info()
+        wbuf, dW = guarded((K, N), dtype, device)
+        plan.gemm_epi_wgrad_execute(X, dZ, dW)
+        torch.cuda.synchronize()
+        assert plan.status() == 0, "watchdog fired"
+    assert guards_intact(wbuf), "dW guard region overwritten"
+    return {"dW": dW.cpu(), "info": info}
+
+
+def check_wgrad(inp_cpu, dtype, gpu, rows=None, cols=None, exact=False, dz_key="dY2"):
+    bits = synth.bits_u16
+    ref = oracle.wgrad(bits(inp_cpu["X"]), bits(inp_cpu[dz_key]), odt(dtype), rows=rows, cols=cols)
+    r_idx = slice(None) if rows is None else torch.tensor(rows)
+    c_idx = slice(None) if cols is None else torch.tensor(cols)
+    got = gpu["dW"][r_idx][:, c_idx].double().numpy()
+    if exact:
+        expect = torch.from_numpy(ref["dW"]).to(dtype).double().numpy()
+        assert np.array_equal(got, expect), "dW not bit-exact on integer inputs"
+    else:
+        assert_within(got, ref["dW"], ref["S"], Y_REL, "dW", unit_roundoff(dtype))
+    return ref

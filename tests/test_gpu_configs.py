@@ -13,7 +13,8 @@ import torch
 import oracle
 from gemm_epilogues_tcgen05_b200 import Plan, synth
 
-from _parity import Y_REL, assert_dbias_is_column_sum, assert_within, dbias_scale, odt, unit_roundoff
+from _parity import (Y_REL, assert_dbias_is_column_sum, assert_within, check_wgrad, dbias_scale, odt, run_wgrad,
+                     unit_roundoff)
 
 pytestmark = pytest.mark.gpu
 
@@ -128,6 +129,20 @@ def test_square_sampled():
 
 def test_ffn_sampled():
     _run(synth.WORKLOADS["ffn"], full=False)
+
+
+def test_ffn_wgrad_sampled():
+    """Weight gradient on the FFN shape: dW (4096 x 11008) = X^T dZ over T = 4096,
+    checked on 256 sampled rows and 256 sampled columns."""
+    w = synth.WORKLOADS["ffn"]
+    inp = {"X": synth.make_inputs(w, parts=("fwd",))["X"],
+           "dZ": synth.masked_grad(w.T, w.N, w.D2, w.torch_dtype, seed=w.seed + 21)}
+    gpu = run_wgrad(inp, w.torch_dtype, dz_key="dZ")
+    assert gpu["info"]["kernel"] == 2
+    rows = synth.sample_indices(w.K, SAMPLE, seed=w.seed + 13)
+    cols = synth.sample_indices(w.N, SAMPLE, seed=w.seed + 14)
+    check_wgrad(inp, w.torch_dtype, gpu, rows=rows, dz_key="dZ")
+    check_wgrad(inp, w.torch_dtype, gpu, cols=cols, dz_key="dZ")
 
 
 @pytest.mark.slow

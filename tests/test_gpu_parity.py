@@ -8,7 +8,7 @@ import torch
 import oracle
 from gemm_epilogues_tcgen05_b200 import binding, synth
 
-from _parity import check_backward, check_forward, run_backward, run_forward
+from _parity import check_backward, check_forward, check_wgrad, run_backward, run_forward, run_wgrad
 
 pytestmark = pytest.mark.gpu
 
@@ -252,8 +252,58 @@ def test_error_paths_on_device():
         binding.gemm_epi_free(hb)
 
 
+# weight gradient dW = X^T dZ: ragged K (dW rows), N and T (the contraction),
+# T = 1, and enough tiles for more than one wave of CTA pairs
+WGRAD_SHAPES = [(200, 264, 136), (1, 72, 64), (130, 520, 328), (1000, 1032, 264), (257, 8, 8), (64, 640, 192),
+                (777, 2056, 1104)]
+
+
+@pytest.mark.parametrize("variant", ["tile64", "tile128", "tile256", "pair"])
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+@pytest.mark.parametrize("T,N,K", WGRAD_SHAPES)
+def test_wgrad_matches_oracle(monkeypatch, T, N, K, dtype, variant):
+    _force(monkeypatch, variant)
+    inp = synth.make_shape_inputs(T, N, K, dtype, seed=3 * T + N + 5 * K, D2=N)
+    gpu = run_wgrad(inp, DT[dtype])
+    # dW has K rows: the CTA-pair kernel when forced and K > 128, else one CTA per tile (never the few-row kernel)
+    assert gpu["info"]["kernel"] == (2 if variant == "pair" and K > 128 else 0)
+    assert (gpu["info"]["T"], gpu["info"]["N"], gpu["info"]["K"]) == (T, N, K)
+    check_wgrad(inp, DT[dtype], gpu)
+
+
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+@pytest.mark.parametrize("variant", ["auto", "pair"])
+def test_wgrad_integer_inputs_bit_exact(monkeypatch, dtype, variant):
+    if variant == "pair":
+        _force(monkeypatch, "pair")
+    T, N, K = 300, 520, 264
+    inp = synth.make_shape_inputs(T, N, K, dtype, seed=41, D2=N, kind="int")
+    check_wgrad(inp, DT[dtype], run_wgrad(inp, DT[dtype]), exact=True)
+
+
+def test_wgrad_plan_rejects_other_calls():
+    T, N, K = 64, 64, 64
+    X = torch.zeros(T, K, dtype=torch.float16, device="cuda")
+    L = binding.lib()
+    h = binding.gemm_epi_plan(T, N, K, binding.F16, binding.WGRAD)
+    try:
+        s = torch.cuda.current_stream().cuda_stream
+        p = X.data_ptr()
+        assert L.gemm_epi_execute(h, p, p, p, p, p, s) == binding.ERR_EPILOG_MISMATCH
+        assert L.drelu_bgrad_execute(h, p, p, p, p, p, s) == binding.ERR_EPILOG_MISMATCH
+        assert L.gemm_epi_wgrad_execute(h, p + 2, p, p, s) == binding.ERR_MISALIGNED
+        assert L.gemm_epi_wgrad_execute(h, p, None, p, s) == binding.ERR_INVALID_ARG
+    finally:
+        binding.gemm_epi_free(h)
+    hf = binding.gemm_epi_plan(T, N, K, binding.F16, binding.RELU_BIAS)
+    try:
+        assert L.gemm_epi_wgrad_execute(hf, p, p, p, None) == binding.ERR_EPILOG_MISMATCH
+    finally:
+        binding.gemm_epi_free(hf)
+
+
 def test_unknown_epilog_values_rejected():
-    for bad in (-1, 5, 99):
+    for bad in (-1, 6, 99):
         with pytest.raises(binding.GemmEpiError):
             binding.gemm_epi_plan(64, 64, 64, binding.F16, bad)
 

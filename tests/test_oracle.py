@@ -501,3 +501,71 @@ def test_gelu_epilog_is_bias_then_gelu(oracle_mod):
     assert np.array_equal(rg["Z"], rb["Z"]) and np.array_equal(rg["S"], rb["S"])
     z = rb["Z"]
     assert np.max(np.abs(rg["Y"] - z * 0.5 * (1 + np.vectorize(math.erf)(z / math.sqrt(2))))) < 1e-15
+
+
+# ------------------------------------------------------------------ WGRAD
+def pin_wgrad(wg):
+    fails = []
+    # worked by hand: X (T=3 x K=2), dZ (T=3 x N=3)
+    #   dW[0] = 1*[1,0,2] + 3*[0,1,0] + 5*[1,1,1] = [6, 8, 7]
+    #   dW[1] = 2*[1,0,2] + 4*[0,1,0] + 6*[1,1,1] = [8, 10, 10]
+    X = _bits([[1, 2], [3, 4], [5, 6]], "fp16")
+    dZ = _bits([[1, 0, 2], [0, 1, 0], [1, 1, 1]], "fp16")
+    r = wg(X, dZ, 0)
+    if not np.array_equal(r["dW"], np.array([[6.0, 8.0, 7.0], [8.0, 10.0, 10.0]])):
+        fails.append("hand-worked")
+    # closed form: X = 1, dZ = 2 -> dW = 2T everywhere; S = 2T
+    T = 37
+    r = wg(_bits(np.ones((T, 5)).tolist(), "bf16"), _bits((2 * np.ones((T, 9))).tolist(), "bf16"), 1)
+    if not (np.all(r["dW"] == 2.0 * T) and np.all(r["S"] == 2.0 * T) and r["dW"].shape == (5, 9)):
+        fails.append("closed form")
+    # brute force in exact rationals on a random tiny case
+    rng = np.random.default_rng(5)
+    Xv = (rng.integers(-40, 40, size=(6, 3)) / 8.0).tolist()
+    Dv = (rng.integers(-40, 40, size=(6, 4)) / 16.0).tolist()
+    r = wg(_bits(Xv, "fp16"), _bits(Dv, "fp16"), 0)
+    for k in range(3):
+        for n in range(4):
+            exact = sum(Fraction(Xv[t][k]) * Fraction(Dv[t][n]) for t in range(6))
+            if Fraction(r["dW"][k, n]) != exact:
+                fails.append(f"rational {k},{n}")
+    return fails
+
+
+def test_wgrad_pins(oracle_mod):
+    fails = pin_wgrad(oracle_mod.wgrad)
+    assert not fails, fails
+
+
+def test_wgrad_planted_mistakes_are_caught(oracle_mod):
+    o = oracle_mod
+
+    def no_transpose_rows_flipped(X, dZ, dt, **kw):  # pairs X row t with dZ row T-1-t
+        return o.wgrad(np.ascontiguousarray(np.asarray(X)[::-1]), dZ, dt, **kw)
+
+    def last_row_dropped(X, dZ, dt, **kw):
+        return o.wgrad(np.asarray(X)[:-1], np.asarray(dZ)[:-1], dt, **kw)
+
+    def sign(X, dZ, dt, **kw):
+        r = o.wgrad(X, dZ, dt, **kw)
+        return {"dW": -r["dW"], "S": r["S"]}
+
+    def dz_transposed_product(X, dZ, dt, **kw):  # (dZ^T X)^T computed with X and dZ swapped roles
+        r = o.wgrad(dZ, X, dt, **kw)
+        return {"dW": r["dW"].T.copy(), "S": r["S"].T.copy()}
+
+    for name, m in {"rows flipped": no_transpose_rows_flipped, "last row dropped": last_row_dropped,
+                    "sign": sign}.items():
+        assert pin_wgrad(m), f"pins did not catch: {name}"
+    # the swapped-role product is the same matrix (a correct identity), so the pins must pass it
+    assert not pin_wgrad(dz_transposed_product)
+
+
+def test_wgrad_subsets_match_full(oracle_mod):
+    inp = synth.make_shape_inputs(33, 40, 24, "bf16", seed=8, D2=40)
+    X, dZ = synth.bits_u16(inp["X"]), synth.bits_u16(inp["dY2"])
+    full = oracle_mod.wgrad(X, dZ, 1)
+    part = oracle_mod.wgrad(X, dZ, 1, rows=[0, 5, 23], cols=[1, 39])
+    assert np.array_equal(part["dW"], full["dW"][np.ix_([0, 5, 23], [1, 39])])
+    with pytest.raises(ValueError):
+        oracle_mod.wgrad(X, dZ[:-1], 1)
