@@ -30,7 +30,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgemm_epi
 
 EXPORTED = ["gemm_epi_plan", "gemm_epi_execute", "drelu_bgrad_execute", "gemm_epi_free", "gemm_epi_last_error",
             "gemm_epi_query", "gemm_epi_status", "gemm_epi_unfused_execute", "drelu_bgrad_unfused_execute",
-            "drelu_bgrad_execute_noalloc", "gemm_epi_wgrad_execute"]
+            "drelu_bgrad_execute_noalloc", "gemm_epi_wgrad_execute", "gemm_epi_set_bias_f32"]
 
 NOALLOC_SCRATCH_BYTES = 4 << 20  # GEMM_EPI_NOALLOC_SCRATCH_BYTES
 
@@ -83,6 +83,8 @@ def lib() -> ctypes.CDLL:
         L.drelu_bgrad_unfused_execute.argtypes = [vp] * 8
         L.drelu_bgrad_execute_noalloc.restype = ci
         L.drelu_bgrad_execute_noalloc.argtypes = [i64, i64, i64, ci] + [vp] * 6
+        L.gemm_epi_set_bias_f32.restype = ci
+        L.gemm_epi_set_bias_f32.argtypes = [vp, ci]
         L.gemm_epi_wgrad_execute.restype = ci
         L.gemm_epi_wgrad_execute.argtypes = [vp] * 5
         _lib = L
@@ -164,7 +166,13 @@ class Plan:
         self.dtype = dtype
         self.epilog = EPILOGS[epilog] if isinstance(epilog, str) else epilog
         self.aux_words = (N + 31) // 32
+        self.bias_dtype = dtype
         self.handle = gemm_epi_plan(T, N, K, dtype, self.epilog)
+
+    def set_bias_f32(self, on: bool = True):
+        """Read the forward bias as fp32 (True) or in the plan's 16-bit type (False)."""
+        _check(lib().gemm_epi_set_bias_f32(self.handle, 1 if on else 0))
+        self.bias_dtype = torch.float32 if on else self.dtype
 
     # life cycle ----------------------------------------------------------
     def free(self):
@@ -196,7 +204,7 @@ class Plan:
     # calls -------------------------------------------------------------
     def gemm_epi_execute(self, X, W, bias, Y, aux=None, stream=None):
         T, N, K, dt = self.T, self.N, self.K, self.dtype
-        args = (_ptr(X, (T, K), dt, "X"), _ptr(W, (K, N), dt, "W"), _ptr(bias, (N,), dt, "bias"),
+        args = (_ptr(X, (T, K), dt, "X"), _ptr(W, (K, N), dt, "W"), _ptr(bias, (N,), self.bias_dtype, "bias"),
                 _ptr(Y, (T, N), dt, "Y"), _ptr(aux, (T, self.aux_words), torch.int32, "aux"))
         _check(lib().gemm_epi_execute(self.handle, *args, _stream_ptr(stream)))
 
@@ -215,7 +223,7 @@ class Plan:
 
     def gemm_epi_unfused_execute(self, X, W, bias, T1, T2, Y, aux=None, stream=None):
         T, N, K, dt = self.T, self.N, self.K, self.dtype
-        args = (_ptr(X, (T, K), dt, "X"), _ptr(W, (K, N), dt, "W"), _ptr(bias, (N,), dt, "bias"),
+        args = (_ptr(X, (T, K), dt, "X"), _ptr(W, (K, N), dt, "W"), _ptr(bias, (N,), self.bias_dtype, "bias"),
                 _ptr(T1, (T, N), dt, "T1"), _ptr(T2, (T, N), dt, "T2"), _ptr(Y, (T, N), dt, "Y"),
                 _ptr(aux, (T, self.aux_words), torch.int32, "aux"))
         _check(lib().gemm_epi_unfused_execute(self.handle, *args, _stream_ptr(stream)))
@@ -231,7 +239,7 @@ class Plan:
     # per-call argument checking (for tight launch loops; check rc yourself)
     def execute_call(self, X, W, bias, Y, aux=None, stream=None):
         T, N, K, dt = self.T, self.N, self.K, self.dtype
-        args = (self.handle, _ptr(X, (T, K), dt, "X"), _ptr(W, (K, N), dt, "W"), _ptr(bias, (N,), dt, "bias"),
+        args = (self.handle, _ptr(X, (T, K), dt, "X"), _ptr(W, (K, N), dt, "W"), _ptr(bias, (N,), self.bias_dtype, "bias"),
                 _ptr(Y, (T, N), dt, "Y"), _ptr(aux, (T, self.aux_words), torch.int32, "aux"), _stream_ptr(stream))
         return lib().gemm_epi_execute, args
 
@@ -250,7 +258,7 @@ class Plan:
 
     def unfused_call(self, X, W, bias, T1, T2, Y, aux=None, stream=None):
         T, N, K, dt = self.T, self.N, self.K, self.dtype
-        args = (self.handle, _ptr(X, (T, K), dt, "X"), _ptr(W, (K, N), dt, "W"), _ptr(bias, (N,), dt, "bias"),
+        args = (self.handle, _ptr(X, (T, K), dt, "X"), _ptr(W, (K, N), dt, "W"), _ptr(bias, (N,), self.bias_dtype, "bias"),
                 _ptr(T1, (T, N), dt, "T1"), _ptr(T2, (T, N), dt, "T2"), _ptr(Y, (T, N), dt, "Y"),
                 _ptr(aux, (T, self.aux_words), torch.int32, "aux"), _stream_ptr(stream))
         return lib().gemm_epi_unfused_execute, args

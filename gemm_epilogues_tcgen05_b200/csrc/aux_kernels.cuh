@@ -67,7 +67,7 @@ __global__ void gelu_kernel(const uint4* __restrict__ in, uint4* __restrict__ ou
 // Unfused BiasAdd: out[t][n] = in[t][n] + bias[n] (8 elements per thread).
 template <bool BF16>
 __global__ void bias_add_kernel(const uint4* __restrict__ in, const void* __restrict__ bias, uint4* __restrict__ out,
-                                int64_t T, int N) {
+                                int64_t T, int N, int bias_f32) {
   const int vec_per_row = N / 8;
   const int64_t total = T * vec_per_row;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
@@ -77,7 +77,9 @@ __global__ void bias_add_kernel(const uint4* __restrict__ in, const void* __rest
     unpack8<BF16>(in[i], f);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      if constexpr (BF16)
+      if (bias_f32)
+        f[j] += reinterpret_cast<const float*>(bias)[n0 + j];
+      else if constexpr (BF16)
         f[j] += __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(bias)[n0 + j]);
       else
         f[j] += __half2float(reinterpret_cast<const __half*>(bias)[n0 + j]);

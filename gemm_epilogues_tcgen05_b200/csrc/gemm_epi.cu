@@ -295,6 +295,7 @@ struct gemm_epi_plan_s {
   uint64_t timeout_ns = 0;
   int inject_stall = 0;  // GEMM_EPI_INJECT_STALL at plan time (watchdog tests)
   int tail_split = 1;    // GEMM_EPI_TAIL_SPLIT=0 keeps whole tiles in the pair kernel's last round
+  int bias_f32 = 0;      // gemm_epi_set_bias_f32: the forward bias is fp32
   // tensor-map cache
   const void* a_ptr = nullptr;
   const void* b_ptr = nullptr;
@@ -370,6 +371,7 @@ ge::TileParams base_params(const gemm_epi_plan_s* p) {
   k.timeout_ns = p->timeout_ns;
   k.inject_stall = p->inject_stall;
   k.tail_split = p->tail_split;
+  k.bias_f32 = p->bias_f32;
   return k;
 }
 
@@ -466,6 +468,7 @@ ge::SkinnyParams skinny_params(const gemm_epi_plan_s* p) {
   k.tickets = p->sk_tickets;
   k.status = p->status_dev;
   k.timeout_ns = p->timeout_ns;
+  k.bias_f32 = p->bias_f32;
   return k;
 }
 
@@ -730,7 +733,7 @@ int gemm_epi_execute(gemm_epi_plan_t plan, const void* X, const void* W, const v
   if (!X || !W || !bias || !Y) return fail(GEMM_EPI_ERR_INVALID_ARG, "gemm_epi_execute: NULL X, W, bias or Y");
   if (p->epilog == GEMM_EPI_RELU_AUX_BIAS && !aux)
     return fail(GEMM_EPI_ERR_EPILOG_MISMATCH, "RELU_AUX_BIAS needs an aux buffer");
-  if (!aligned(X, 16) || !aligned(W, 16) || !aligned(Y, 16) || !aligned(bias, 2) ||
+  if (!aligned(X, 16) || !aligned(W, 16) || !aligned(Y, 16) || !aligned(bias, p->bias_f32 ? 4 : 2) ||
       (p->epilog == GEMM_EPI_RELU_AUX_BIAS && !aligned(aux, 4)))
     return fail(GEMM_EPI_ERR_MISALIGNED, "gemm_epi_execute: X, W, Y need 16-byte, bias 2-byte, aux 4-byte alignment");
   int rc = take_status(p);
@@ -796,7 +799,7 @@ int gemm_epi_unfused_execute(gemm_epi_plan_t plan, const void* X, const void* W,
   if (p->epilog == GEMM_EPI_RELU_AUX_BIAS && !aux)
     return fail(GEMM_EPI_ERR_EPILOG_MISMATCH, "RELU_AUX_BIAS needs an aux buffer");
   if (!aligned(X, 16) || !aligned(W, 16) || !aligned(T1, 16) || !aligned(T2, 16) || !aligned(Y, 16) ||
-      !aligned(bias, 2) || (aux && !aligned(aux, 4)))
+      !aligned(bias, p->bias_f32 ? 4 : 2) || (aux && !aligned(aux, 4)))
     return fail(GEMM_EPI_ERR_MISALIGNED, "unfused: misaligned pointer");
   int rc = take_status(p);
   if (rc) return rc;
@@ -809,9 +812,11 @@ int gemm_epi_unfused_execute(gemm_epi_plan_t plan, const void* X, const void* W,
   const bool bf16 = p->dtype == GEMM_EPI_BF16;
   const int blocks = p->num_sms * 8;
   if (bf16)
-    ge::bias_add_kernel<true><<<blocks, 256, 0, stream>>>((const uint4*)T1, bias, (uint4*)T2, p->T, (int)p->N);
+    ge::bias_add_kernel<true><<<blocks, 256, 0, stream>>>((const uint4*)T1, bias, (uint4*)T2, p->T, (int)p->N,
+                                                          p->bias_f32);
   else
-    ge::bias_add_kernel<false><<<blocks, 256, 0, stream>>>((const uint4*)T1, bias, (uint4*)T2, p->T, (int)p->N);
+    ge::bias_add_kernel<false><<<blocks, 256, 0, stream>>>((const uint4*)T1, bias, (uint4*)T2, p->T, (int)p->N,
+                                                           p->bias_f32);
   if (p->epilog == GEMM_EPI_GELU_BIAS) {
     const int64_t n_vec = p->T * p->N / 8;
     if (bf16)
@@ -836,6 +841,15 @@ int gemm_epi_unfused_execute(gemm_epi_plan_t plan, const void* X, const void* W,
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "unfused elementwise launch");
+  return GEMM_EPI_OK;
+}
+
+int gemm_epi_set_bias_f32(gemm_epi_plan_t plan, int bias_f32) {
+  gemm_epi_plan_s* p = lookup(plan);
+  if (!p) return fail(GEMM_EPI_ERR_INVALID_ARG, "gemm_epi_set_bias_f32: unknown plan");
+  if (p->epilog == GEMM_EPI_DRELU_BGRAD || p->epilog == GEMM_EPI_WGRAD)
+    return fail(GEMM_EPI_ERR_EPILOG_MISMATCH, "gemm_epi_set_bias_f32: only forward plans take a bias");
+  p->bias_f32 = bias_f32 ? 1 : 0;
   return GEMM_EPI_OK;
 }
 

@@ -39,6 +39,7 @@ struct SkinnyParams {
   int* tickets;                    // [n_tiles], zero between launches
   int* status;
   uint64_t timeout_ns;
+  int32_t bias_f32;                // the bias is N fp32 values (else the 16-bit type)
 };
 
 // A stage holds KPS consecutive 64-deep k-blocks: W as one box of 64 features
@@ -384,7 +385,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int word = (s.tile * 128 + static_cast<int>(ew) * 32) >> 5;
       float bias_n = 0.f;
       if constexpr (AddsBias<EPI>::value)
-        bias_n = n_ok ? load_16<BF16>(p.bias, n) : 0.f;
+        bias_n = n_ok ? load_bias<BF16>(p.bias, p.bias_f32, n) : 0.f;
       float dbias_acc = 0.f;
       const bool whole = s.kb0 == 0 && s.kb1 == p.kbt;
       Mask16 mk{};

@@ -92,6 +92,7 @@ struct TileParams {
   int* col_tickets;         // DRELU_BGRAD: per column block, zero between launches; null = no in-kernel finish
   float* dbias;             // DRELU_BGRAD: written by the tile that takes a column block's last ticket
   int32_t tail_split;       // pair kernel: split the last round's tiles into column halves
+  int32_t bias_f32;         // the bias is N fp32 values (else the 16-bit type)
 };
 
 constexpr int kBM = 128;
@@ -169,6 +170,12 @@ __device__ __forceinline__ float load_16(const void* base, int64_t i) {
     return __half2float(reinterpret_cast<const __half*>(base)[i]);
 }
 
+// bias[n] as fp32, stored either as fp32 or in the 16-bit type
+template <bool BF16>
+__device__ __forceinline__ float load_bias(const void* bias, int bias_f32, int64_t n) {
+  return bias_f32 ? reinterpret_cast<const float*>(bias)[n] : load_16<BF16>(bias, n);
+}
+
 template <bool BF16>
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   if constexpr (BF16) {
@@ -208,7 +215,7 @@ __device__ __forceinline__ void epi_stage_bias(const TileParams& p, int n0, floa
   if constexpr (AddsBias<EPI>::value) {
     for (int c = et; c < ncols; c += 128) {
       const int n = n0 + c;
-      bs[c] = n < p.N ? load_16<BF16>(p.bias, n) : 0.f;
+      bs[c] = n < p.N ? load_bias<BF16>(p.bias, p.bias_f32, n) : 0.f;
     }
   }
 }

@@ -140,6 +140,19 @@ GEMM_EPI_API int drelu_bgrad_execute(gemm_epi_plan_t plan, const void* dY2, cons
                         void* dZ, float* dbias, cudaStream_t stream);
 
 /*
+ * gemm_epi_set_bias_f32: forward plans only. With bias_f32 != 0, later
+ * execute calls of this plan read the bias as N fp32 values (4-byte aligned)
+ * instead of the plan's 16-bit type; 0 restores the default. "Fusing bias
+ * addition into matrix multiplication with nvmath-python" (engineering
+ * checklist, types and device) allows a float32 bias with float16 operands
+ * and has the library convert it. The bias is added in fp32 either way.
+ * Takes effect for calls enqueued after it returns (host-side state).
+ * Returns GEMM_EPI_OK; GEMM_EPI_ERR_INVALID_ARG for an unknown plan;
+ * GEMM_EPI_ERR_EPILOG_MISMATCH on a DRELU_BGRAD or WGRAD plan.
+ */
+GEMM_EPI_API int gemm_epi_set_bias_f32(gemm_epi_plan_t plan, int bias_f32);
+
+/*
  * gemm_epi_wgrad_execute: the weight gradient of the linear layer,
  * dW[k][n] = sum over t of X[t][k] * dZ[t][n], rounded to dtype. The pages
  * name no epilog for it: "nvmath-python fused epilogs for linear layers"

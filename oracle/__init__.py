@@ -173,7 +173,8 @@ def gelu(Z):
 
 
 def linear_fwd(X, W, bias, dtype: int, epilog: str, rows=None, cols=None, threads=None):
-    """Forward epilogs on X (T x K) and W (K x N) with bias (N).
+    """Forward epilogs on X (T x K) and W (K x N) with bias (N): 16-bit
+    patterns (uint16), or float32 values for an fp32 bias.
 
     Returns a dict with
       Z     the pre-activation X.W + bias (fp64, exact up to binary64 rounding)
@@ -184,7 +185,19 @@ def linear_fwd(X, W, bias, dtype: int, epilog: str, rows=None, cols=None, thread
     """
     if epilog not in (EPILOG_BIAS, EPILOG_RELU_BIAS, EPILOG_RELU_AUX_BIAS, EPILOG_GELU_BIAS):
         raise ValueError(f"unknown forward epilog {epilog}")
-    Z, S = matmul_bias(X, W, bias, dtype, rows=rows, cols=cols, threads=threads)
+    if bias is not None and np.asarray(bias).dtype == np.float32:
+        # an fp32 bias ("Fusing bias addition ...", engineering checklist: a
+        # float32 bias with 16-bit operands): the product, then the bias added
+        # in binary64 -- the same last step the C routine takes for a 16-bit bias
+        Z, S = matmul_bias(X, W, None, dtype, rows=rows, cols=cols, threads=threads)
+        b = np.asarray(bias, dtype=np.float64).ravel()
+        if b.shape[0] != np.asarray(W).shape[1]:
+            raise ValueError("bias length must equal the column count")
+        b = b if cols is None else b[np.asarray(cols, dtype=np.int64)]
+        Z = Z + b[None, :]
+        S = S + np.abs(b)[None, :]
+    else:
+        Z, S = matmul_bias(X, W, bias, dtype, rows=rows, cols=cols, threads=threads)
     out = {"Z": Z, "S": S}
     if epilog == EPILOG_BIAS:
         out["Y"] = Z.copy()

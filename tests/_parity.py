@@ -56,11 +56,14 @@ def guards_intact(buf) -> bool:
     return bool(torch.all(torch.isnan(head))) and bool(torch.all(torch.isnan(tail)))
 
 
-def run_forward(inp_cpu: dict, epilog: str, dtype, device="cuda", unfused=False):
-    X, W, b = (inp_cpu[k].to(device) for k in ("X", "W", "bias"))
+def run_forward(inp_cpu: dict, epilog: str, dtype, device="cuda", unfused=False, bias_f32=False):
+    """One forward call; with bias_f32 the plan reads the fp32 bias under "bias32"."""
+    X, W, b = (inp_cpu[k].to(device) for k in ("X", "W", "bias32" if bias_f32 else "bias"))
     T, K = X.shape
     N = W.shape[1]
     with Plan(T, N, K, dtype, epilog) as plan:
+        if bias_f32:
+            plan.set_bias_f32(True)
         info = plan.info()
         ybuf, Y = guarded((T, N), dtype, device)
         abuf, aux = guarded((T, (N + 31) // 32), torch.int32, device)
@@ -128,13 +131,13 @@ def assert_within(got: np.ndarray, ref: np.ndarray, scale: np.ndarray, rel: floa
 GELU_SLOPE = 1.13
 
 
-def check_forward(inp_cpu, epilog, dtype, gpu, rows=None, cols=None, exact=False, stored_xw=False):
+def check_forward(inp_cpu, epilog, dtype, gpu, rows=None, cols=None, exact=False, stored_xw=False, bias_f32=False):
     """Y (and the mask) against the oracle.  ``stored_xw``: the path under test stored X·W in the
     16-bit output type before adding the bias (the unfused ablation), a second rounding that may
     add up to u·|X·W|, so the bound gains that term."""
     bits = synth.bits_u16
-    ref = oracle.linear_fwd(bits(inp_cpu["X"]), bits(inp_cpu["W"]), bits(inp_cpu["bias"]), odt(dtype), epilog,
-                            rows=rows, cols=cols)
+    bias = inp_cpu["bias32"].numpy() if bias_f32 else bits(inp_cpu["bias"])
+    ref = oracle.linear_fwd(bits(inp_cpu["X"]), bits(inp_cpu["W"]), bias, odt(dtype), epilog, rows=rows, cols=cols)
     Y = gpu["Y"]
     r_idx = slice(None) if rows is None else torch.tensor(rows)
     c_idx = slice(None) if cols is None else torch.tensor(cols)
@@ -150,7 +153,7 @@ def check_forward(inp_cpu, epilog, dtype, gpu, rows=None, cols=None, exact=False
     else:
         scale = ref["S"]
         if stored_xw:
-            b = inp_cpu["bias"].double().numpy()
+            b = inp_cpu["bias32" if bias_f32 else "bias"].double().numpy()
             b = b if cols is None else b[cols]
             scale = scale + (unit_roundoff(dtype) / Y_REL) * np.abs(ref["Z"] - b[None, :])
             if epilog == "GELU_BIAS":  # the unfused path also stores X.W + b before the GELU kernel

@@ -252,6 +252,21 @@ def test_error_paths_on_device():
         binding.gemm_epi_free(hb)
 
 
+@pytest.mark.parametrize("variant", ["tile128", "tile256", "skinny", "pair"])
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+@pytest.mark.parametrize("T,N,K", [(200, 264, 136), (16, 1032, 520), (600, 1024, 328)])
+def test_fp32_bias(monkeypatch, T, N, K, dtype, variant):
+    """Forward epilogs with an fp32 bias (values no 16-bit type holds), fused and unfused."""
+    _force(monkeypatch, variant)
+    inp = synth.make_shape_inputs(T, N, K, dtype, seed=17 * T + N + K)
+    inp["bias32"] = synth.normal((N,), synth.BIAS_STD, torch.float32, seed=T + 2 * N)
+    for ep in FWD_EPILOGS:
+        gpu = run_forward(inp, ep, DT[dtype], bias_f32=True)
+        check_forward(inp, ep, DT[dtype], gpu, bias_f32=True)
+        gpu = run_forward(inp, ep, DT[dtype], bias_f32=True, unfused=True)
+        check_forward(inp, ep, DT[dtype], gpu, bias_f32=True, stored_xw=True)
+
+
 # weight gradient dW = X^T dZ: ragged K (dW rows), N and T (the contraction),
 # T = 1, and enough tiles for more than one wave of CTA pairs
 WGRAD_SHAPES = [(200, 264, 136), (1, 72, 64), (130, 520, 328), (1000, 1032, 264), (257, 8, 8), (64, 640, 192),
@@ -293,6 +308,7 @@ def test_wgrad_plan_rejects_other_calls():
         assert L.drelu_bgrad_execute(h, p, p, p, p, p, s) == binding.ERR_EPILOG_MISMATCH
         assert L.gemm_epi_wgrad_execute(h, p + 2, p, p, s) == binding.ERR_MISALIGNED
         assert L.gemm_epi_wgrad_execute(h, p, None, p, s) == binding.ERR_INVALID_ARG
+        assert L.gemm_epi_set_bias_f32(h, 1) == binding.ERR_EPILOG_MISMATCH
     finally:
         binding.gemm_epi_free(h)
     hf = binding.gemm_epi_plan(T, N, K, binding.F16, binding.RELU_BIAS)

@@ -569,3 +569,30 @@ def test_wgrad_subsets_match_full(oracle_mod):
     assert np.array_equal(part["dW"], full["dW"][np.ix_([0, 5, 23], [1, 39])])
     with pytest.raises(ValueError):
         oracle_mod.wgrad(X, dZ[:-1], 1)
+
+
+# ------------------------------------------------------------- fp32 bias
+def test_fp32_bias_equal_to_16bit_bias_gives_the_same_result(oracle_mod):
+    inp = synth.make_shape_inputs(7, 40, 24, "fp16", seed=12)
+    X, W, b16 = (synth.bits_u16(inp[k]) for k in ("X", "W", "bias"))
+    b32 = inp["bias"].float().numpy()  # the same values, held as fp32
+    for ep in ("BIAS", "RELU_AUX_BIAS", "GELU_BIAS"):
+        r16 = oracle_mod.linear_fwd(X, W, b16, 0, ep)
+        r32 = oracle_mod.linear_fwd(X, W, b32, 0, ep)
+        for key in ("Z", "S", "Y"):
+            assert np.array_equal(r16[key], r32[key]), (ep, key)
+    part = oracle_mod.linear_fwd(X, W, b32, 0, "BIAS", cols=[3, 39])
+    assert np.array_equal(part["Z"], oracle_mod.linear_fwd(X, W, b32, 0, "BIAS")["Z"][:, [3, 39]])
+
+
+def test_fp32_bias_values_are_taken_exactly(oracle_mod):
+    # X = 0: Z is the fp32 bias itself (values no 16-bit type holds), S = |bias|
+    b32 = np.array([0.1, -1e-3, 3.14159274, 65519.0, -7.0e-8, 0.0, 1.0, 2.5], dtype=np.float32)
+    X = _bits(np.zeros((3, 16)).tolist(), "bf16")
+    W = _bits(np.ones((16, 8)).tolist(), "bf16")
+    r = oracle_mod.linear_fwd(X, W, b32, 1, "RELU_BIAS")
+    assert np.array_equal(r["Z"], np.tile(b32.astype(np.float64), (3, 1)))
+    assert np.array_equal(r["S"], np.tile(np.abs(b32.astype(np.float64)), (3, 1)))
+    assert np.array_equal(r["Y"], np.maximum(r["Z"], 0.0))
+    with pytest.raises(ValueError):
+        oracle_mod.linear_fwd(X, W, b32[:5], 1, "BIAS")
