@@ -493,21 +493,25 @@ def main():
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak}
     else:
         achieved = alg[part]["flops"] / (part_ms / 1e3) / 1e12
-        # fp16 dense peak = bf16 dense peak. A launch shorter than a
-        # millisecond runs before the 1 kW power cap settles the clocks, so
-        # the burst figure applies; a longer launch is a sustained load.
+        # fp16 dense peak = bf16 dense peak. The burst figure is for a kernel
+        # that runs before the 1 kW power cap settles the clocks; a launch of
+        # a millisecond or more, or a timed region during which the sampled
+        # clocks report the power cap active (back-to-back steps), is a
+        # sustained load and is measured against the sustained figure.
         burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
         sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
         long_launch = part_ms >= 1.0
-        peak = sustained if long_launch else burst
+        capped = "sw_power_cap" in ((res.get("clocks") or {}).get("reasons") or [])
+        peak = sustained if (long_launch or capped) else burst
+        kind = ("sustained (launch >= 1 ms)" if long_launch else
+                "sustained (power cap active in the timed region)" if capped else "burst (launch < 1 ms)")
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                "frac_of_burst": achieved / burst,
-                "peak_kind": "sustained (launch >= 1 ms)" if long_launch else "burst (launch < 1 ms)"}
+                "frac_of_burst": achieved / burst, "peak_kind": kind}
     kname = {0: "tile_kernel", 1: "skinny_kernel", 2: "tile2_kernel (CTA pair)"}[res["kernel"]]
     roof["kernel"] = f"{part}: {kname} " + (fwd_epi if part == "fwd" else "DRELU_BGRAD" +
                                               (" + dbias finish" if res["kernel"] != 1 else ""))
     roof["peak_source"] = "measured (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
-    roof["traffic"] = measured_traffic(w, part)
+    roof["traffic"] = measured_traffic(w, part, fwd_epi)
     # roofline time of the whole step: slower of FLOPs at the tensor peak and bytes at HBM
     t_roof = sum(max(v["flops"] / (float(peaks.get("bf16_tflops", 1590.0)) * 1e12),
                      v["bytes"] / (float(peaks.get("hbm_gbs", 6650.0)) * 1e9)) for v in alg.values())
@@ -530,9 +534,10 @@ def main():
     print(json.dumps(line), flush=True)
 
 
-def measured_traffic(w, part):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel sources; else None."""
+def measured_traffic(w, part, fwd_epi):
+    """DRAM bytes per launch of the timed call (keys "<workload>:fwd:<epilog>",
+    "<workload>:bwd", "<workload>:wgrad") from the committed ncu summaries, if
+    they were taken on the current kernel sources; else None."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
@@ -540,10 +545,11 @@ def measured_traffic(w, part):
     except Exception:
         return None
     current = kernel_source_hash()
-    for key, entry in d.items():
-        if key.split("#")[0] == f"{w.name}:{part}" and isinstance(entry, dict) \
-                and entry.get("source_hash") == current:
-            return entry.get("dram_bytes_per_launch")
+    want = (f"{w.name}:wgrad" if fwd_epi == "WGRAD" else f"{w.name}:bwd" if part == "bwd"
+            else f"{w.name}:fwd:{fwd_epi}")
+    entry = d.get(want)
+    if isinstance(entry, dict) and entry.get("source_hash") == current:
+        return entry.get("dram_bytes_per_launch")
     return None
 
 
