@@ -166,6 +166,22 @@ class ClockSampler:
                 "power_w_max": max((num(p[4]) or 0.0) for p in inside)}
 
 
+# ------------------------------------------------------- across the ranks
+def max_over_ranks(values, device, world: int) -> list[float]:
+    """Each entry's maximum over all ranks (the slowest rank's time): an
+    all-reduce with MAX on the default process group when world > 1."""
+    t = torch.tensor([float(v) for v in values], device=device, dtype=torch.float64)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def whole_job_tflops(flops_per_rank_step: float, world: int, slowest_step_ms: float) -> float:
+    """Every rank runs its own replica of the step (weak scaling): the units of
+    all ranks divided by the slowest rank's step time."""
+    return flops_per_rank_step * world / (slowest_step_ms / 1e3) / 1e12
+
+
 # ----------------------------------------------------------------- our arm
 def run_ours(args, w: synth.Workload, rank: int, world: int, dev: torch.device):
     from gemm_epilogues_tcgen05_b200 import Plan, binding
@@ -269,10 +285,8 @@ def run_ours(args, w: synth.Workload, rank: int, world: int, dev: torch.device):
     fwd_ms = [e[0].elapsed_time(e[1]) for e in evs]
     bwd_ms = [e[1].elapsed_time(e[2]) for e in evs] if bplan is not None else [0.0] * args.steps
     step_ms = sum(fwd_ms) / args.steps + sum(bwd_ms) / args.steps
-    t = torch.tensor([step_ms, sum(fwd_ms) / args.steps, sum(bwd_ms) / args.steps], device=dev, dtype=torch.float64)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    step_ms, fwd_avg, bwd_avg = (float(x) for x in t.tolist())
+    step_ms, fwd_avg, bwd_avg = max_over_ranks([step_ms, sum(fwd_ms) / args.steps, sum(bwd_ms) / args.steps], dev,
+                                               world)
 
     alg = algorithmic(w, fwd_epi, bplan is not None)
     flops_step = sum(v["flops"] for v in alg.values())
@@ -482,7 +496,7 @@ def main():
         return
 
     alg = res["alg"]
-    value = res["flops_step"] * world / (res["step_ms"] / 1e3) / 1e12
+    value = whole_job_tflops(res["flops_step"], world, res["step_ms"])
     # dominant kernel: the one of the two calls that takes longer
     part = "fwd" if res["fwd_ms"] >= res["bwd_ms"] else "bwd"
     part_ms = res[f"{part}_ms"]
