@@ -30,7 +30,8 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgemm_epi
 
 EXPORTED = ["gemm_epi_plan", "gemm_epi_execute", "drelu_bgrad_execute", "gemm_epi_free", "gemm_epi_last_error",
             "gemm_epi_query", "gemm_epi_status", "gemm_epi_unfused_execute", "drelu_bgrad_unfused_execute",
-            "drelu_bgrad_execute_noalloc", "gemm_epi_wgrad_execute", "gemm_epi_set_bias_f32"]
+            "drelu_bgrad_execute_noalloc", "gemm_epi_wgrad_execute", "gemm_epi_set_bias_f32", "gemm_epi_plan_ex"]
+FLAG_W_NK = 1  # GEMM_EPI_FLAG_W_NK
 
 NOALLOC_SCRATCH_BYTES = 4 << 20  # GEMM_EPI_NOALLOC_SCRATCH_BYTES
 
@@ -65,6 +66,8 @@ def lib() -> ctypes.CDLL:
         vp, i64, ci = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
         L.gemm_epi_plan.restype = vp
         L.gemm_epi_plan.argtypes = [i64, i64, i64, ci, ci]
+        L.gemm_epi_plan_ex.restype = vp
+        L.gemm_epi_plan_ex.argtypes = [i64, i64, i64, ci, ci, ctypes.c_uint32]
         L.gemm_epi_execute.restype = ci
         L.gemm_epi_execute.argtypes = [vp] * 7
         L.drelu_bgrad_execute.restype = ci
@@ -122,13 +125,13 @@ def _ptr(t, shape, dtype, name) -> int | None:
     return t.data_ptr()
 
 
-def gemm_epi_plan(T: int, N: int, K: int, dtype, epilog) -> int:
-    """Raw handle (int) from the C gemm_epi_plan; raises on error."""
+def gemm_epi_plan(T: int, N: int, K: int, dtype, epilog, flags: int = 0) -> int:
+    """Raw handle (int) from the C gemm_epi_plan_ex; raises on error."""
     if isinstance(dtype, torch.dtype):
         dtype = DTYPES[dtype]
     if isinstance(epilog, str):
         epilog = EPILOGS[epilog]
-    h = lib().gemm_epi_plan(T, N, K, dtype, epilog)
+    h = lib().gemm_epi_plan_ex(T, N, K, dtype, epilog, flags)
     if not h:
         raise GemmEpiError(ERR_INVALID_ARG, gemm_epi_last_error())
     return h
@@ -161,13 +164,15 @@ def drelu_bgrad_execute_noalloc(dY2, W2, aux, dZ, dbias, stream=None):
 class Plan:
     """A plan for one (T, N, K, dtype, epilog); execute any number of times."""
 
-    def __init__(self, T: int, N: int, K: int, dtype: torch.dtype, epilog: str | int):
+    def __init__(self, T: int, N: int, K: int, dtype: torch.dtype, epilog: str | int, w_nk: bool = False):
+        """w_nk: the weight (W, or W2 of DRELU_BGRAD) is N x K, K contiguous."""
         self.T, self.N, self.K = T, N, K
+        self.w_shape = (N, K) if w_nk else (K, N)
         self.dtype = dtype
         self.epilog = EPILOGS[epilog] if isinstance(epilog, str) else epilog
         self.aux_words = (N + 31) // 32
         self.bias_dtype = dtype
-        self.handle = gemm_epi_plan(T, N, K, dtype, self.epilog)
+        self.handle = gemm_epi_plan(T, N, K, dtype, self.epilog, FLAG_W_NK if w_nk else 0)
 
     def set_bias_f32(self, on: bool = True):
         """Read the forward bias as fp32 (True) or in the plan's 16-bit type (False)."""
@@ -204,13 +209,13 @@ class Plan:
     # calls -------------------------------------------------------------
     def gemm_epi_execute(self, X, W, bias, Y, aux=None, stream=None):
         T, N, K, dt = self.T, self.N, self.K, self.dtype
-        args = (_ptr(X, (T, K), dt, "X"), _ptr(W, (K, N), dt, "W"), _ptr(bias, (N,), self.bias_dtype, "bias"),
+        args = (_ptr(X, (T, K), dt, "X"), _ptr(W, self.w_shape, dt, "W"), _ptr(bias, (N,), self.bias_dtype, "bias"),
                 _ptr(Y, (T, N), dt, "Y"), _ptr(aux, (T, self.aux_words), torch.int32, "aux"))
         _check(lib().gemm_epi_execute(self.handle, *args, _stream_ptr(stream)))
 
     def drelu_bgrad_execute(self, dY2, W2, aux, dZ, dbias, stream=None):
         T, N, K, dt = self.T, self.N, self.K, self.dtype
-        args = (_ptr(dY2, (T, K), dt, "dY2"), _ptr(W2, (K, N), dt, "W2"),
+        args = (_ptr(dY2, (T, K), dt, "dY2"), _ptr(W2, self.w_shape, dt, "W2"),
                 _ptr(aux, (T, self.aux_words), torch.int32, "aux"), _ptr(dZ, (T, N), dt, "dZ"),
                 _ptr(dbias, (N,), torch.float32, "dbias"))
         _check(lib().drelu_bgrad_execute(self.handle, *args, _stream_ptr(stream)))
@@ -223,14 +228,14 @@ class Plan:
 
     def gemm_epi_unfused_execute(self, X, W, bias, T1, T2, Y, aux=None, stream=None):
         T, N, K, dt = self.T, self.N, self.K, self.dtype
-        args = (_ptr(X, (T, K), dt, "X"), _ptr(W, (K, N), dt, "W"), _ptr(bias, (N,), self.bias_dtype, "bias"),
+        args = (_ptr(X, (T, K), dt, "X"), _ptr(W, self.w_shape, dt, "W"), _ptr(bias, (N,), self.bias_dtype, "bias"),
                 _ptr(T1, (T, N), dt, "T1"), _ptr(T2, (T, N), dt, "T2"), _ptr(Y, (T, N), dt, "Y"),
                 _ptr(aux, (T, self.aux_words), torch.int32, "aux"))
         _check(lib().gemm_epi_unfused_execute(self.handle, *args, _stream_ptr(stream)))
 
     def drelu_bgrad_unfused_execute(self, dY2, W2, aux, G, dZ, dbias, stream=None):
         T, N, K, dt = self.T, self.N, self.K, self.dtype
-        args = (_ptr(dY2, (T, K), dt, "dY2"), _ptr(W2, (K, N), dt, "W2"),
+        args = (_ptr(dY2, (T, K), dt, "dY2"), _ptr(W2, self.w_shape, dt, "W2"),
                 _ptr(aux, (T, self.aux_words), torch.int32, "aux"), _ptr(G, (T, N), dt, "G"),
                 _ptr(dZ, (T, N), dt, "dZ"), _ptr(dbias, (N,), torch.float32, "dbias"))
         _check(lib().drelu_bgrad_unfused_execute(self.handle, *args, _stream_ptr(stream)))
@@ -239,13 +244,13 @@ class Plan:
     # per-call argument checking (for tight launch loops; check rc yourself)
     def execute_call(self, X, W, bias, Y, aux=None, stream=None):
         T, N, K, dt = self.T, self.N, self.K, self.dtype
-        args = (self.handle, _ptr(X, (T, K), dt, "X"), _ptr(W, (K, N), dt, "W"), _ptr(bias, (N,), self.bias_dtype, "bias"),
+        args = (self.handle, _ptr(X, (T, K), dt, "X"), _ptr(W, self.w_shape, dt, "W"), _ptr(bias, (N,), self.bias_dtype, "bias"),
                 _ptr(Y, (T, N), dt, "Y"), _ptr(aux, (T, self.aux_words), torch.int32, "aux"), _stream_ptr(stream))
         return lib().gemm_epi_execute, args
 
     def drelu_bgrad_call(self, dY2, W2, aux, dZ, dbias, stream=None):
         T, N, K, dt = self.T, self.N, self.K, self.dtype
-        args = (self.handle, _ptr(dY2, (T, K), dt, "dY2"), _ptr(W2, (K, N), dt, "W2"),
+        args = (self.handle, _ptr(dY2, (T, K), dt, "dY2"), _ptr(W2, self.w_shape, dt, "W2"),
                 _ptr(aux, (T, self.aux_words), torch.int32, "aux"), _ptr(dZ, (T, N), dt, "dZ"),
                 _ptr(dbias, (N,), torch.float32, "dbias"), _stream_ptr(stream))
         return lib().drelu_bgrad_execute, args
@@ -258,14 +263,14 @@ class Plan:
 
     def unfused_call(self, X, W, bias, T1, T2, Y, aux=None, stream=None):
         T, N, K, dt = self.T, self.N, self.K, self.dtype
-        args = (self.handle, _ptr(X, (T, K), dt, "X"), _ptr(W, (K, N), dt, "W"), _ptr(bias, (N,), self.bias_dtype, "bias"),
+        args = (self.handle, _ptr(X, (T, K), dt, "X"), _ptr(W, self.w_shape, dt, "W"), _ptr(bias, (N,), self.bias_dtype, "bias"),
                 _ptr(T1, (T, N), dt, "T1"), _ptr(T2, (T, N), dt, "T2"), _ptr(Y, (T, N), dt, "Y"),
                 _ptr(aux, (T, self.aux_words), torch.int32, "aux"), _stream_ptr(stream))
         return lib().gemm_epi_unfused_execute, args
 
     def drelu_bgrad_unfused_call(self, dY2, W2, aux, G, dZ, dbias, stream=None):
         T, N, K, dt = self.T, self.N, self.K, self.dtype
-        args = (self.handle, _ptr(dY2, (T, K), dt, "dY2"), _ptr(W2, (K, N), dt, "W2"),
+        args = (self.handle, _ptr(dY2, (T, K), dt, "dY2"), _ptr(W2, self.w_shape, dt, "W2"),
                 _ptr(aux, (T, self.aux_words), torch.int32, "aux"), _ptr(G, (T, N), dt, "G"),
                 _ptr(dZ, (T, N), dt, "dZ"), _ptr(dbias, (N,), torch.float32, "dbias"), _stream_ptr(stream))
         return lib().drelu_bgrad_unfused_execute, args

@@ -296,6 +296,7 @@ struct gemm_epi_plan_s {
   int inject_stall = 0;  // GEMM_EPI_INJECT_STALL at plan time (watchdog tests)
   int tail_split = 1;    // GEMM_EPI_TAIL_SPLIT=0 keeps whole tiles in the pair kernel's last round
   int bias_f32 = 0;      // gemm_epi_set_bias_f32: the forward bias is fp32
+  int w_nk = 0;          // GEMM_EPI_FLAG_W_NK: W / W2 given N x K (K contiguous)
   // tensor-map cache
   const void* a_ptr = nullptr;
   const void* b_ptr = nullptr;
@@ -348,7 +349,13 @@ int prepare_maps(gemm_epi_plan_s* p, const void* A, const void* B) {
     if (rc) return rc;
     p->a_ptr = A;
   }
-  if (B != p->b_ptr) {
+  if (B != p->b_ptr && p->w_nk) {
+    // N x K weight, K-major: one box of 64 k x (the CTA's) BN rows per stage
+    const uint32_t rows = p->kernel == 2 ? 128u : (uint32_t)p->cfg.BN;
+    int rc = encode_2d(&p->tmB, B, (uint64_t)p->K, (uint64_t)p->N, ge::kBK, rows, "the N x K weight operand");
+    if (rc) return rc;
+    p->b_ptr = B;
+  } else if (B != p->b_ptr) {
     int rc = encode_2d(&p->tmB, B, (uint64_t)p->N, (uint64_t)p->K, 64, ge::kBK, "the weight operand");
     if (rc) return rc;
     p->b_ptr = B;
@@ -372,6 +379,7 @@ ge::TileParams base_params(const gemm_epi_plan_s* p) {
   k.inject_stall = p->inject_stall;
   k.tail_split = p->tail_split;
   k.bias_f32 = p->bias_f32;
+  k.b_kmajor = p->w_nk;
   return k;
 }
 
@@ -498,6 +506,20 @@ int choose_bn(int64_t T, int64_t N, int num_sms) {
 extern "C" {
 
 gemm_epi_plan_t gemm_epi_plan(int64_t T, int64_t N, int64_t K, gemm_epi_dtype dtype, gemm_epi_epilog epilog) {
+  return gemm_epi_plan_ex(T, N, K, dtype, epilog, 0u);
+}
+
+gemm_epi_plan_t gemm_epi_plan_ex(int64_t T, int64_t N, int64_t K, gemm_epi_dtype dtype, gemm_epi_epilog epilog,
+                                 uint32_t flags) {
+  if ((flags & ~(uint32_t)GEMM_EPI_FLAG_W_NK) != 0) {
+    fail(GEMM_EPI_ERR_INVALID_ARG, "unknown plan flags 0x%x", flags);
+    return nullptr;
+  }
+  const bool w_nk = (flags & GEMM_EPI_FLAG_W_NK) != 0;
+  if (w_nk && epilog == GEMM_EPI_WGRAD) {
+    fail(GEMM_EPI_ERR_INVALID_ARG, "GEMM_EPI_FLAG_W_NK applies to the weight of forward and DRELU_BGRAD plans");
+    return nullptr;
+  }
   if (T < 1 || N < 8 || K < 8 || (N % 8) != 0 || (K % 8) != 0) {
     fail(GEMM_EPI_ERR_INVALID_ARG, "bad shape T=%lld N=%lld K=%lld (need T>=1, N,K>=8 and multiples of 8)",
          (long long)T, (long long)N, (long long)K);
@@ -548,6 +570,7 @@ gemm_epi_plan_t gemm_epi_plan(int64_t T, int64_t N, int64_t K, gemm_epi_dtype dt
   p->K = K;
   p->dtype = dtype;
   p->epilog = epilog;
+  p->w_nk = w_nk ? 1 : 0;
   p->device = dev;
   p->num_sms = sms;
   const bool bf16 = dtype == GEMM_EPI_BF16;
@@ -594,7 +617,7 @@ gemm_epi_plan_t gemm_epi_plan(int64_t T, int64_t N, int64_t K, gemm_epi_dtype dt
     e = cudaFuncSetAttribute(c->fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)c->smem);
     if (e != cudaSuccess) return cleanup(cuda_fail(e, "cudaFuncSetAttribute(max dynamic shared memory)"));
   }
-  if (!pair && epilog != GEMM_EPI_WGRAD && use_skinny(T)) {
+  if (!pair && epilog != GEMM_EPI_WGRAD && !w_nk && use_skinny(T)) {
     p->kernel = 1;
     p->sk = skinny_cfg(T, (int)epilog, bf16);
     const int n_tiles = ceil_div(N, 128);

@@ -89,6 +89,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr bool A_MN = AOperandMN<EPI>::value;
   constexpr uint32_t IDESC = idesc_f16(BF16, /*A MN-major*/ A_MN, /*B MN-major*/ true, 2 * kBM, BN);
   constexpr uint32_t IDESC_HALF = idesc_f16(BF16, A_MN, true, 2 * kBM, BN / 2);
+  constexpr uint32_t IDESC_BK = idesc_f16(BF16, A_MN, /*B MN-major*/ false, 2 * kBM, BN);
   constexpr uint32_t PAIR_TX = 2 * (L::A_BYTES + L::B_BYTES);
   constexpr uint32_t PAIR_TX_HALF = 2 * (L::A_BYTES + L::B_CHUNK);
   constexpr uint16_t BOTH = 0x3;
@@ -143,7 +144,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int m2_tiles = (p.m_tiles + 1) / 2;  // 256-row tiles
-  const PairSchedule sched(m2_tiles * p.n_tiles, npairs, p.tail_split != 0);
+  // half units need a 64-row box of a K-major W: with b_kmajor every unit is a whole tile
+  const PairSchedule sched(m2_tiles * p.n_tiles, npairs, p.tail_split != 0 && p.b_kmajor == 0);
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -172,8 +174,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             tma_load_2d_pair(sA + s * L::A_BYTES, &tmA, fbar, kb * kBK, m0);
           }
-          for (int j = 0; j < nchunks; ++j)
-            tma_load_2d_pair(sB + s * L::B_BYTES + j * L::B_CHUNK, &tmB, fbar, nh0 + j * 64, kb * kBK);
+          if (p.b_kmajor) {  // this CTA's 128 rows of the N x K weight in one box
+            tma_load_2d_pair(sB + s * L::B_BYTES, &tmB, fbar, kb * kBK, nh0);
+          } else {
+            for (int j = 0; j < nchunks; ++j)
+              tma_load_2d_pair(sB + s * L::B_BYTES + j * L::B_CHUNK, &tmB, fbar, nh0 + j * 64, kb * kBK);
+          }
         }
       }
       // the last fills have landed once the MMA has released them
@@ -190,7 +196,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         for (int u = pair; ok && u < sched.num_units; u += npairs, ++tcount) {
           const PairUnit w = sched.unit(u, m2_tiles, p.n_tiles, p.group_m);
-          const uint32_t idesc = w.half < 0 ? IDESC : IDESC_HALF;
+          const uint32_t idesc = p.b_kmajor ? IDESC_BK : w.half < 0 ? IDESC : IDESC_HALF;
           const uint32_t buf = tcount & 1u;
           const uint32_t tph = (tcount >> 1) & 1u;
           if (!wait_bounded(&tempty[buf], tph ^ 1u, p, abort_flag, 3)) break;
@@ -209,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int kk = 0; kk < kBK / 16; ++kk) {
               const uint64_t adesc = a_desc<A_MN>(a0, kk);
-              const uint64_t bdesc = smem_desc_sw128(b0 + kk * 2048, L::B_CHUNK, 1024);
+              const uint64_t bdesc = b_desc(b0, kk, p.b_kmajor != 0, L::B_CHUNK);
               umma_f16_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
             }
             umma_commit_pair(&empty[s], BOTH);

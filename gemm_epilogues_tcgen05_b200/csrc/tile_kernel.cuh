@@ -57,6 +57,14 @@ struct PlainStore {
 // K-major: 128-byte rows, 8-row groups 1024 B apart, a K step is 32 bytes
 // inside the swizzle atom; MN-major: 64-wide M chunks 8 KB apart (LBO), 8
 // K-rows 1024 B apart (SBO), a K step is 16 rows = 2048 bytes.
+// B operand descriptor for K step kk of a stage at b0. MN-major (W is K x N):
+// 64-wide N chunks `chunk` bytes apart (LBO), 8 K-rows 1024 B apart (SBO), a
+// K step of 16 rows is 2048 bytes. K-major (W is N x K): 128-byte rows of 64
+// k, 8-row groups 1024 B apart, a K step is 32 bytes inside the swizzle atom.
+__device__ __forceinline__ uint64_t b_desc(uint32_t b0, int kk, bool k_major, uint32_t chunk) {
+  return k_major ? smem_desc_sw128(b0 + kk * 32, 16, 1024) : smem_desc_sw128(b0 + kk * 2048, chunk, 1024);
+}
+
 template <bool A_MN>
 __device__ __forceinline__ uint64_t a_desc(uint32_t a0, int kk) {
   if constexpr (A_MN)
@@ -93,6 +101,7 @@ struct TileParams {
   float* dbias;             // DRELU_BGRAD: written by the tile that takes a column block's last ticket
   int32_t tail_split;       // pair kernel: split the last round's tiles into column halves
   int32_t bias_f32;         // the bias is N fp32 values (else the 16-bit type)
+  int32_t b_kmajor;         // W is N x K (K contiguous): B is staged K-major, one box of BN rows per stage
 };
 
 constexpr int kBM = 128;
@@ -409,6 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                  : (2 * BN <= 256) ? 256 : 512;
   constexpr bool A_MN = AOperandMN<EPI>::value;
   constexpr uint32_t IDESC = idesc_f16(BF16, /*A MN-major*/ A_MN, /*B MN-major*/ true, kBM, BN);
+  constexpr uint32_t IDESC_BK = idesc_f16(BF16, A_MN, /*B MN-major*/ false, kBM, BN);
   constexpr uint32_t STAGE_TX = L::A_BYTES + L::B_BYTES;
 
   extern __shared__ uint8_t smem_raw[];
@@ -481,9 +491,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             tma_load_2d(sA + s * L::A_BYTES, &tmA, &full[s], kb * kBK, m0);
           }
+          if (p.b_kmajor) {
+            tma_load_2d(sB + s * L::B_BYTES, &tmB, &full[s], kb * kBK, n0);
+          } else {
 #pragma unroll
-          for (int j = 0; j < BN / 64; ++j)
-            tma_load_2d(sB + s * L::B_BYTES + j * L::B_CHUNK, &tmB, &full[s], n0 + j * 64, kb * kBK);
+            for (int j = 0; j < BN / 64; ++j)
+              tma_load_2d(sB + s * L::B_BYTES + j * L::B_CHUNK, &tmB, &full[s], n0 + j * 64, kb * kBK);
+          }
         }
       }
       // let every issued copy land before the CTA can exit
@@ -497,6 +511,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t it = 0, tcount = 0;
       bool ok = true;
+      const bool bk = p.b_kmajor != 0;
+      const uint32_t idesc = bk ? IDESC_BK : IDESC;
       for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++tcount) {
         const uint32_t buf = tcount & 1u;
         const uint32_t tph = (tcount >> 1) & 1u;
@@ -516,10 +532,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
             const uint64_t adesc = a_desc<A_MN>(a0, kk);
-            // B: N-major, 64-wide N chunks 8 KB apart (LBO), 8 K-rows 1024 B
-            // apart (SBO); a K step of 16 rows is 2048 bytes.
-            const uint64_t bdesc = smem_desc_sw128(b0 + kk * 2048, L::B_CHUNK, 1024);
-            umma_f16(d_tmem, adesc, bdesc, IDESC, (kb | kk) != 0 ? 1u : 0u);
+            const uint64_t bdesc = b_desc(b0, kk, bk, L::B_CHUNK);
+            umma_f16(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
           umma_commit(&empty[s]);
         }

@@ -113,6 +113,25 @@ typedef struct {
 GEMM_EPI_API gemm_epi_plan_t gemm_epi_plan(int64_t T, int64_t N, int64_t K, gemm_epi_dtype dtype,
                               gemm_epi_epilog epilog);
 
+/* Flags of gemm_epi_plan_ex. */
+enum { GEMM_EPI_FLAG_W_NK = 1u };
+
+/*
+ * gemm_epi_plan_ex: gemm_epi_plan with flags (gemm_epi_plan passes 0).
+ *   GEMM_EPI_FLAG_W_NK: the weight operand -- W of a forward plan, W2 of a
+ *   DRELU_BGRAD plan -- is given N x K row-major (K contiguous: the
+ *   [out_features, in_features] layout of a framework's linear layer)
+ *   instead of K x N. Chaining two layers needs both orientations of one
+ *   weight (the forward reads it as N x K, the backward through it as
+ *   K x N); with this flag neither has to be transposed in memory. Such plans
+ *   run on the one-CTA or CTA-pair kernels, never the few-row kernel. Not
+ *   valid for WGRAD plans.
+ * Returns a plan, or NULL with gemm_epi_last_error() set (unknown flags:
+ * GEMM_EPI_ERR_INVALID_ARG).
+ */
+GEMM_EPI_API gemm_epi_plan_t gemm_epi_plan_ex(int64_t T, int64_t N, int64_t K, gemm_epi_dtype dtype,
+                                              gemm_epi_epilog epilog, uint32_t flags);
+
 /*
  * gemm_epi_execute: the forward epilogs (BIAS, RELU_BIAS, RELU_AUX_BIAS).
  *   X, W, Y: device pointers, 16-byte aligned. bias: device pointer, 2-byte

@@ -56,12 +56,15 @@ def guards_intact(buf) -> bool:
     return bool(torch.all(torch.isnan(head))) and bool(torch.all(torch.isnan(tail)))
 
 
-def run_forward(inp_cpu: dict, epilog: str, dtype, device="cuda", unfused=False, bias_f32=False):
-    """One forward call; with bias_f32 the plan reads the fp32 bias under "bias32"."""
+def run_forward(inp_cpu: dict, epilog: str, dtype, device="cuda", unfused=False, bias_f32=False, w_nk=False):
+    """One forward call; with bias_f32 the plan reads the fp32 bias under "bias32"; with
+    w_nk the library gets W transposed to N x K (the oracle keeps the K x N original)."""
     X, W, b = (inp_cpu[k].to(device) for k in ("X", "W", "bias32" if bias_f32 else "bias"))
     T, K = X.shape
     N = W.shape[1]
-    with Plan(T, N, K, dtype, epilog) as plan:
+    if w_nk:
+        W = W.t().contiguous()
+    with Plan(T, N, K, dtype, epilog, w_nk=w_nk) as plan:
         if bias_f32:
             plan.set_bias_f32(True)
         info = plan.info()
@@ -85,13 +88,15 @@ def run_forward(inp_cpu: dict, epilog: str, dtype, device="cuda", unfused=False,
     return out
 
 
-def run_backward(inp_cpu: dict, aux_words: np.ndarray, dtype, device="cuda", unfused=False, repeats=1):
+def run_backward(inp_cpu: dict, aux_words: np.ndarray, dtype, device="cuda", unfused=False, repeats=1, w_nk=False):
     dY2, W2 = inp_cpu["dY2"].to(device), inp_cpu["W2"].to(device)
     T, D2 = dY2.shape
     N = W2.shape[1]
+    if w_nk:
+        W2 = W2.t().contiguous()
     aux = torch.from_numpy(np.ascontiguousarray(aux_words).view(np.int32)).to(device)
     outs = []
-    with Plan(T, N, D2, dtype, "DRELU_BGRAD") as plan:
+    with Plan(T, N, D2, dtype, "DRELU_BGRAD", w_nk=w_nk) as plan:
         info = plan.info()
         for _ in range(repeats):
             zbuf, dZ = guarded((T, N), dtype, device)

@@ -267,6 +267,52 @@ def test_fp32_bias(monkeypatch, T, N, K, dtype, variant):
         check_forward(inp, ep, DT[dtype], gpu, bias_f32=True, stored_xw=True)
 
 
+# weight given N x K (a framework linear layer's [out, in] layout): ragged
+# shapes, one with more than a wave of CTA pairs (no half tiles then)
+NK_SHAPES = [(200, 264, 136), (16, 1032, 520), (600, 1024, 328), (1000, 5000, 72)]
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+@pytest.mark.parametrize("T,N,K", NK_SHAPES)
+def test_weight_nk_layout(monkeypatch, T, N, K, dtype, variant):
+    _force(monkeypatch, variant)
+    D2 = max(8, (K // 2) // 8 * 8)
+    inp = synth.make_shape_inputs(T, N, K, dtype, seed=13 * T + N + 3 * K, D2=D2)
+    for ep in FWD_EPILOGS:
+        gpu = run_forward(inp, ep, DT[dtype], w_nk=True)
+        assert gpu["info"]["kernel"] != 1  # an N x K weight never runs on the few-row kernel
+        check_forward(inp, ep, DT[dtype], gpu)
+    check_forward(inp, "RELU_BIAS", DT[dtype], run_forward(inp, "RELU_BIAS", DT[dtype], w_nk=True, unfused=True),
+                  stored_xw=True)
+    fwd = run_forward(inp, "RELU_AUX_BIAS", DT[dtype])
+    outs = run_backward(inp, fwd["aux"], DT[dtype], w_nk=True, repeats=2)
+    for gpu in outs:
+        assert gpu["info"]["kernel"] != 1
+        check_backward(inp, fwd["aux"], DT[dtype], gpu)
+    assert torch.equal(outs[0]["dbias"], outs[1]["dbias"])
+
+
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+@pytest.mark.parametrize("variant", ["auto", "pair"])
+def test_weight_nk_integer_inputs_bit_exact(monkeypatch, dtype, variant):
+    if variant == "pair":
+        _force(monkeypatch, "pair")
+    T, N, K, D2 = 300, 1024, 64, 40
+    inp = synth.make_shape_inputs(T, N, K, dtype, seed=77, D2=D2, kind="int")
+    for ep in ("BIAS", "RELU_AUX_BIAS"):
+        check_forward(inp, ep, DT[dtype], run_forward(inp, ep, DT[dtype], w_nk=True), exact=True)
+    fwd = run_forward(inp, "RELU_AUX_BIAS", DT[dtype])
+    check_backward(inp, fwd["aux"], DT[dtype], run_backward(inp, fwd["aux"], DT[dtype], w_nk=True), exact=True)
+
+
+def test_plan_flags_are_checked():
+    with pytest.raises(binding.GemmEpiError):
+        binding.gemm_epi_plan(64, 64, 64, binding.F16, binding.RELU_BIAS, flags=2)
+    with pytest.raises(binding.GemmEpiError):
+        binding.gemm_epi_plan(64, 64, 64, binding.F16, binding.WGRAD, flags=binding.FLAG_W_NK)
+
+
 # weight gradient dW = X^T dZ: ragged K (dW rows), N and T (the contraction),
 # T = 1, and enough tiles for more than one wave of CTA pairs
 WGRAD_SHAPES = [(200, 264, 136), (1, 72, 64), (130, 520, 328), (1000, 1032, 264), (257, 8, 8), (64, 640, 192),
