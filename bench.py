@@ -68,6 +68,8 @@ def kernel_source_hash() -> str:
 def step_spec(w: synth.Workload, args=None):
     """Which epilogs a step of this workload runs. --fwd-epilog GELU_BIAS
     times that forward alone (the library has no GELU backward)."""
+    if args is not None and getattr(args, "ffn_step", False):
+        return "FFN_STEP", True
     if args is not None and getattr(args, "wgrad", False):
         return "WGRAD", False
     if args is not None and getattr(args, "fwd_epilog", None):
@@ -91,6 +93,14 @@ def algorithmic(w: synth.Workload, fwd_epi: str, bwd: bool):
     b_fwd = e * (w.T * w.K + w.K * w.N + w.N + w.T * w.N) + (aux_bytes if fwd_epi == "RELU_AUX_BIAS" else 0)
     if fwd_epi == "WGRAD":  # dW = X^T dZ: reads X and dZ, writes dW
         b_fwd = e * (w.T * w.K + w.T * w.N + w.K * w.N)
+    if fwd_epi == "FFN_STEP":  # two-layer block, D = K, F = N: 2 forward and 4 backward products
+        T, D, F = w.T, w.K, w.N
+        g = 2.0 * T * D * F
+        fwd_b = e * (T * D + F * D + F + T * F) + aux_bytes + e * (T * F + D * F + D + T * D)
+        bwd_b = (e * (T * D + D * F + T * F) + aux_bytes + 4 * F +        # dZ1, db1
+                 e * (T * D + T * F + D * F) + e * T * D + 4 * D +       # dW2, db2 (second read of dY)
+                 e * (T * F + T * D + F * D) + e * (T * F + F * D + T * D))  # dW1, dX
+        return {"fwd": {"flops": 2 * g, "bytes": float(fwd_b)}, "bwd": {"flops": 4 * g, "bytes": float(bwd_b)}}
     out = {"fwd": {"flops": f_fwd, "bytes": float(b_fwd)}}
     if bwd:
         f_bwd = 2.0 * w.T * w.N * w.D2
@@ -193,9 +203,9 @@ def run_ours(args, w: synth.Workload, rank: int, world: int, dev: torch.device):
     Y = torch.empty((w.T, w.N), dtype=dt, device=dev)
     aux_words = math.ceil(w.N / 32)
     aux = torch.zeros((w.T, aux_words), dtype=torch.int32, device=dev)
-    fplan = Plan(w.T, w.N, w.K, dt, fwd_epi)
+    fplan = Plan(w.T, w.N, w.K, dt, "RELU_AUX_BIAS" if args.ffn_step else fwd_epi)
     bplan = None
-    if has_bwd:
+    if has_bwd and not args.ffn_step:
         dY2, W2 = inp["dY2"], inp["W2"]
         dZ = torch.empty((w.T, w.N), dtype=dt, device=dev)
         dbias = torch.empty((w.N,), dtype=torch.float32, device=dev)
@@ -212,12 +222,40 @@ def run_ours(args, w: synth.Workload, rank: int, world: int, dev: torch.device):
     fwd_aux = aux if fwd_epi == "RELU_AUX_BIAS" else None
 
     # prebuilt C calls: the timed loop does no per-call argument checking
-    if args.wgrad:  # the weight gradient alone: dW (K x N) = X^T dZ, dZ a stand-in for the backward's
+    plan_ms = None
+    step_plans = None
+    if args.ffn_step:  # a whole two-layer block step, weights in the [out, in] layout; D = K, F = N
+        fplan.free()
+        T, D, F = w.T, w.K, w.N
+        si = synth.ffn_step_inputs(T, D, F, w.dtype, seed=w.seed, device=dev)
+        t0 = time.perf_counter()
+        sp = [Plan(T, F, D, dt, "RELU_AUX_BIAS", w_nk=True), Plan(T, D, F, dt, "BIAS", w_nk=True),
+              Plan(T, F, D, dt, "DRELU_BGRAD"), Plan(T, F, D, dt, "WGRAD"), Plan(T, D, F, dt, "WGRAD"),
+              Plan(T, D, F, dt, "NONE")]
+        plan_ms = (time.perf_counter() - t0) * 1e3 / len(sp)
+        H = torch.empty((T, F), dtype=dt, device=dev)
+        aux1 = torch.empty((T, math.ceil(F / 32)), dtype=torch.int32, device=dev)
+        Ys = torch.empty((T, D), dtype=dt, device=dev)
+        dZ1 = torch.empty((T, F), dtype=dt, device=dev)
+        db1 = torch.empty((F,), dtype=torch.float32, device=dev)
+        dW2 = torch.empty((D, F), dtype=dt, device=dev)
+        db2 = torch.empty((D,), dtype=torch.float32, device=dev)
+        dW1 = torch.empty((F, D), dtype=dt, device=dev)
+        dX = torch.empty((T, D), dtype=dt, device=dev)
+        fcall = [sp[0].execute_call(si["X"], si["W1"], si["b1"], H, aux1, stream),
+                 sp[1].execute_call(H, si["W2"], si["b2"], Ys, None, stream)]
+        bcall = [sp[2].drelu_bgrad_call(si["dY"], si["W2"], aux1, dZ1, db1, stream),
+                 sp[3].wgrad_call(si["dY"], H, dW2, db2, stream),
+                 sp[4].wgrad_call(dZ1, si["X"], dW1, None, stream),
+                 sp[5].execute_call(dZ1, si["W1"], None, dX, None, stream)]
+        fplan, bplan = sp[0], sp[2]
+        step_plans = sp
+    elif args.wgrad:  # the weight gradient alone: dW (K x N) = X^T dZ, dZ a stand-in for the backward's
         fplan.free()
         dZw = synth.masked_grad(w.T, w.N, w.D2 or w.K, dt, seed=w.seed + 21, device=dev)
         fplan = Plan(w.T, w.N, w.K, dt, "WGRAD")
         dW = torch.empty((w.K, w.N), dtype=dt, device=dev)
-        fcall = fplan.wgrad_call(X, dZw, dW, stream)
+        fcall = fplan.wgrad_call(X, dZw, dW, None, stream)
         bcall = None
     elif args.ablation:
         fcall = fplan.unfused_call(X, W, b, T1, T2 if fwd_epi != "BIAS" else Y, Y, fwd_aux, stream)
@@ -227,9 +265,10 @@ def run_ours(args, w: synth.Workload, rank: int, world: int, dev: torch.device):
         bcall = bplan.drelu_bgrad_call(dY2, W2, aux, dZ, dbias, stream) if bplan is not None else None
 
     def call(c):
-        rc = c[0](*c[1])
-        if rc != 0:
-            raise RuntimeError(f"library call failed ({rc}): {binding.gemm_epi_last_error()}")
+        for fn, a in (c if isinstance(c, list) else [c]):
+            rc = fn(*a)
+            if rc != 0:
+                raise RuntimeError(f"library call failed ({rc}): {binding.gemm_epi_last_error()}")
 
     def step(ev):
         ev[0].record(stream)
@@ -254,7 +293,7 @@ def run_ours(args, w: synth.Workload, rank: int, world: int, dev: torch.device):
 
     run_steps([new_events() for _ in range(args.warmup)])
     torch.cuda.synchronize(dev)
-    for p in (fplan, bplan):
+    for p in (step_plans if args.ffn_step else (fplan, bplan)):
         if p is not None and p.status() != 0:
             raise RuntimeError("watchdog fired during warm-up")
 
@@ -278,7 +317,7 @@ def run_ours(args, w: synth.Workload, rank: int, world: int, dev: torch.device):
     if world > 1:
         torch.distributed.barrier()
     clocks = sampler.stop(wall0, wall1) if sampler else None
-    for p in (fplan, bplan):
+    for p in (step_plans if args.ffn_step else (fplan, bplan)):
         if p is not None and p.status() != 0:
             raise RuntimeError("watchdog fired during the timed region")
 
@@ -293,19 +332,26 @@ def run_ours(args, w: synth.Workload, rank: int, world: int, dev: torch.device):
     # our kernels per step, as the plans report them (the L2 flush between
     # steps is torch's and sits outside the timed events)
     launches_per_step = fplan.info()["launches"] + (bplan.info()["launches"] if bplan is not None else 0)
+    if args.ffn_step:  # 2 forward GEMMs; DRELU_BGRAD, 2 WGRAD (+2 reduction launches for db2), NONE
+        launches_per_step = 8
     if args.ablation:  # GEMM + bias + ReLU kernels; GEMM + mask + two column-sum kernels
         launches_per_step = (2 if fwd_epi == "BIAS" else 3) + (4 if bplan is not None else 0)
 
     # e2e: host buffers (pinned), H2D of the step's inputs, both calls, D2H of every output
-    e2e = run_e2e(args, w, fwd_epi, fplan, bplan, inp, dev, stream) if not (args.ablation or args.wgrad) else None
+    e2e = (run_e2e(args, w, fwd_epi, fplan, bplan, inp, dev, stream)
+           if not (args.ablation or args.wgrad or args.ffn_step) else None)
 
     kernel = fplan.info()["kernel"]
-    fplan.free()
-    if bplan is not None:
-        bplan.free()
+    if args.ffn_step:
+        for p in step_plans:
+            p.free()
+    else:
+        fplan.free()
+        if bplan is not None:
+            bplan.free()
     return {"step_ms": step_ms, "fwd_ms": fwd_avg, "bwd_ms": bwd_avg, "alg": alg, "flops_step": flops_step,
             "kernel": kernel,
-            "launches": launches_per_step * args.steps, "clocks": clocks, "e2e": e2e,
+            "launches": launches_per_step * args.steps, "clocks": clocks, "e2e": e2e, "plan_ms": plan_ms,
             "wall_s": wall1 - wall0}
 
 
@@ -435,17 +481,22 @@ def metric_name(w: synth.Workload) -> str:
 
 def config_of(w, fwd_epi, has_bwd, args):
     desc = f"{w.name}: fwd {fwd_epi} T={w.T} K={w.K} N={w.N}"
+    if fwd_epi == "FFN_STEP":
+        desc = (f"{w.name}: two-layer block step, T={w.T} D={w.K} F={w.N} {w.dtype}, weights [out, in]: "
+                f"H = relu(X W1^T + b1), Y = H W2^T + b2; dZ1, db1 = DRELU_BGRAD(dY, W2); dW2, db2; dW1; dX")
     if fwd_epi == "WGRAD":
         desc = (f"{w.name}: WGRAD dW (K x N) = X^T dZ over T={w.T}, K={w.K} N={w.N}; dZ a seeded stand-in "
                 f"(N(0, D2/N), half zeros)")
-    if has_bwd:
+    if has_bwd and fwd_epi != "FFN_STEP":
         desc += f" + bwd DRELU_BGRAD D2={w.D2}"
     desc += f", {w.dtype}"
     if args.ablation:
         desc += ", UNFUSED ablation (GEMM, then separate bias / ReLU+mask / mask / column-sum kernels)"
     return {"workload": desc, "T": w.T, "K": w.K, "N": w.N, "D2": w.D2, "dtype": w.dtype,
             "l2": "flushed between steps (256 MiB write outside the timed events)",
-            "inputs": "seeded synthetic: X~N(0,1), W~N(0,1/K), bias~N(0,0.1), dY2~N(0,1), W2~N(0,1/N)"}
+            "inputs": ("seeded synthetic: X~N(0,1), W1~N(0,1/D), W2~N(0,1/F), biases~N(0,0.1), dY~N(0,1)"
+                       if fwd_epi == "FFN_STEP" else
+                       "seeded synthetic: X~N(0,1), W~N(0,1/K), bias~N(0,0.1), dY2~N(0,1), W2~N(0,1/N)")}
 
 
 # -------------------------------------------------------------------- main
@@ -458,6 +509,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ablation", action="store_true", help="time the unfused path instead")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ffn-step", action="store_true",
+                    help="time a whole two-layer block step (2 forward, 4 backward products) on the workload's shape")
     ap.add_argument("--wgrad", action="store_true",
                     help="time the weight gradient dW = X^T dZ alone on the workload's shape")
     ap.add_argument("--fwd-epilog", choices=["BIAS", "RELU_BIAS", "RELU_AUX_BIAS", "GELU_BIAS"], default=None,
@@ -524,6 +577,9 @@ def main():
     kname = {0: "tile_kernel", 1: "skinny_kernel", 2: "tile2_kernel (CTA pair)"}[res["kernel"]]
     roof["kernel"] = f"{part}: {kname} " + (fwd_epi if part == "fwd" else "DRELU_BGRAD" +
                                               (" + dbias finish" if res["kernel"] != 1 else ""))
+    if fwd_epi == "FFN_STEP":
+        roof["kernel"] = (f"{part}: " + ("layer 1 RELU_AUX_BIAS + layer 2 BIAS" if part == "fwd" else
+                                         "DRELU_BGRAD, WGRAD (+db2), WGRAD, NONE") + f" ({kname} kernels)")
     roof["peak_source"] = "measured (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
     roof["traffic"] = measured_traffic(w, part, fwd_epi)
     # roofline time of the whole step: slower of FLOPs at the tensor peak and bytes at HBM
@@ -538,6 +594,8 @@ def main():
             "parallelism": f"replicas x{world} (no exchange step)",
             "fwd_ms": res["fwd_ms"], "bwd_ms": res["bwd_ms"], "roofline": roof,
             "gpu_launches": res["launches"], "clocks": res["clocks"]}
+    if res.get("plan_ms") is not None:
+        line["plan_ms"] = res["plan_ms"]  # host time to create one plan (created once, reused every step)
     if res["e2e"]:
         e = res["e2e"]
         line["e2e"] = {"value": res["flops_step"] / (e["ms_per_step"] / 1e3) / 1e12, "unit": "TFLOP/s",

@@ -13,9 +13,9 @@ import os
 import torch
 
 F16, BF16 = 0, 1
-BIAS, RELU_BIAS, RELU_AUX_BIAS, DRELU_BGRAD, GELU_BIAS, WGRAD = 0, 1, 2, 3, 4, 5
+BIAS, RELU_BIAS, RELU_AUX_BIAS, DRELU_BGRAD, GELU_BIAS, WGRAD, NONE = 0, 1, 2, 3, 4, 5, 6
 EPILOGS = {"BIAS": BIAS, "RELU_BIAS": RELU_BIAS, "RELU_AUX_BIAS": RELU_AUX_BIAS, "DRELU_BGRAD": DRELU_BGRAD,
-           "GELU_BIAS": GELU_BIAS, "WGRAD": WGRAD}
+           "GELU_BIAS": GELU_BIAS, "WGRAD": WGRAD, "NONE": NONE}
 DTYPES = {torch.float16: F16, torch.bfloat16: BF16}
 
 OK = 0
@@ -89,7 +89,7 @@ def lib() -> ctypes.CDLL:
         L.gemm_epi_set_bias_f32.restype = ci
         L.gemm_epi_set_bias_f32.argtypes = [vp, ci]
         L.gemm_epi_wgrad_execute.restype = ci
-        L.gemm_epi_wgrad_execute.argtypes = [vp] * 5
+        L.gemm_epi_wgrad_execute.argtypes = [vp] * 6
         _lib = L
     return _lib
 
@@ -220,10 +220,11 @@ class Plan:
                 _ptr(dbias, (N,), torch.float32, "dbias"))
         _check(lib().drelu_bgrad_execute(self.handle, *args, _stream_ptr(stream)))
 
-    def gemm_epi_wgrad_execute(self, X, dZ, dW, stream=None):
-        """WGRAD plan: dW (K x N) = X^T (T x K)^T . dZ (T x N)."""
+    def gemm_epi_wgrad_execute(self, X, dZ, dW, dbias=None, stream=None):
+        """WGRAD plan: dW (K x N) = X^T . dZ; dbias (K floats, optional) = sum over t of X."""
         T, N, K, dt = self.T, self.N, self.K, self.dtype
-        args = (_ptr(X, (T, K), dt, "X"), _ptr(dZ, (T, N), dt, "dZ"), _ptr(dW, (K, N), dt, "dW"))
+        args = (_ptr(X, (T, K), dt, "X"), _ptr(dZ, (T, N), dt, "dZ"), _ptr(dW, (K, N), dt, "dW"),
+                _ptr(dbias, (K,), torch.float32, "dbias"))
         _check(lib().gemm_epi_wgrad_execute(self.handle, *args, _stream_ptr(stream)))
 
     def gemm_epi_unfused_execute(self, X, W, bias, T1, T2, Y, aux=None, stream=None):
@@ -255,10 +256,10 @@ class Plan:
                 _ptr(dbias, (N,), torch.float32, "dbias"), _stream_ptr(stream))
         return lib().drelu_bgrad_execute, args
 
-    def wgrad_call(self, X, dZ, dW, stream=None):
+    def wgrad_call(self, X, dZ, dW, dbias=None, stream=None):
         T, N, K, dt = self.T, self.N, self.K, self.dtype
         args = (self.handle, _ptr(X, (T, K), dt, "X"), _ptr(dZ, (T, N), dt, "dZ"), _ptr(dW, (K, N), dt, "dW"),
-                _stream_ptr(stream))
+                _ptr(dbias, (K,), torch.float32, "dbias"), _stream_ptr(stream))
         return lib().gemm_epi_wgrad_execute, args
 
     def unfused_call(self, X, W, bias, T1, T2, Y, aux=None, stream=None):
@@ -290,7 +291,8 @@ class Plan:
         self.drelu_bgrad_execute(dY2, W2, aux, dZ, dbias, stream)
         return dZ, dbias
 
-    def wgrad(self, X, dZ, stream=None):
+    def wgrad(self, X, dZ, with_dbias=False, stream=None):
         dW = torch.empty((self.K, self.N), dtype=self.dtype, device=X.device)
-        self.gemm_epi_wgrad_execute(X, dZ, dW, stream)
-        return dW
+        dbias = torch.empty((self.K,), dtype=torch.float32, device=X.device) if with_dbias else None
+        self.gemm_epi_wgrad_execute(X, dZ, dW, dbias, stream)
+        return (dW, dbias) if with_dbias else dW

@@ -116,7 +116,8 @@ static_assert(static_cast<int>(GEMM_EPI_BIAS) == ge::EPI_BIAS && static_cast<int
                   static_cast<int>(GEMM_EPI_RELU_AUX_BIAS) == ge::EPI_RELU_AUX_BIAS &&
                   static_cast<int>(GEMM_EPI_DRELU_BGRAD) == ge::EPI_DRELU_BGRAD &&
                   static_cast<int>(GEMM_EPI_GELU_BIAS) == ge::EPI_GELU_BIAS &&
-                  static_cast<int>(GEMM_EPI_WGRAD) == ge::EPI_WGRAD,
+                  static_cast<int>(GEMM_EPI_WGRAD) == ge::EPI_WGRAD &&
+                  static_cast<int>(GEMM_EPI_NONE) == ge::EPI_STORE,
               "the public epilog values are the kernels' epilog kinds");
 
 template <int BN, int ST, bool BF>
@@ -193,6 +194,7 @@ SkinnyKernelFn pick_skinny_epi(int epi) {
     case ge::EPI_RELU_BIAS: return ge::skinny_kernel<TP, KPS, ge::EPI_RELU_BIAS, BF>;
     case ge::EPI_RELU_AUX_BIAS: return ge::skinny_kernel<TP, KPS, ge::EPI_RELU_AUX_BIAS, BF>;
     case ge::EPI_GELU_BIAS: return ge::skinny_kernel<TP, KPS, ge::EPI_GELU_BIAS, BF>;
+    case ge::EPI_STORE: return ge::skinny_kernel<TP, KPS, ge::EPI_STORE, BF>;
     default: return ge::skinny_kernel<TP, KPS, ge::EPI_DRELU_BGRAD, BF>;
   }
 }
@@ -533,7 +535,7 @@ gemm_epi_plan_t gemm_epi_plan_ex(int64_t T, int64_t N, int64_t K, gemm_epi_dtype
     fail(GEMM_EPI_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
     return nullptr;
   }
-  if (epilog < GEMM_EPI_BIAS || epilog > GEMM_EPI_WGRAD) {
+  if (epilog < GEMM_EPI_BIAS || epilog > GEMM_EPI_NONE) {
     fail(GEMM_EPI_ERR_INVALID_ARG, "unknown epilog %d", (int)epilog);
     return nullptr;
   }
@@ -679,6 +681,10 @@ gemm_epi_plan_t gemm_epi_plan_ex(int64_t T, int64_t N, int64_t K, gemm_epi_dtype
       e = cudaMemset(p->col_tickets, 0, sizeof(int) * (size_t)p->n_tickets);
       if (e != cudaSuccess) return cleanup(cuda_fail(e, "cudaMemset(column tickets)"));
     }
+  } else if (epilog == GEMM_EPI_WGRAD) {  // partials of the optional bias gradient (sum of X over its rows)
+    p->partial_bytes = (size_t)ceil_div(p->uT, 128) * (size_t)p->uK * sizeof(float);
+    e = cudaMalloc((void**)&p->partials, p->partial_bytes);
+    if (e != cudaSuccess) return cleanup(cuda_fail(e, "cudaMalloc(workspace)"));
   }
   {
     std::lock_guard<std::mutex> g(g_mu);
@@ -735,7 +741,9 @@ int gemm_epi_query(gemm_epi_plan_t plan, gemm_epi_info* info) {
     info->split_k = 1;
     info->grid = p->grid;
     info->launches = 1;
-    info->workspace_bytes = p->epilog == GEMM_EPI_DRELU_BGRAD ? p->partial_bytes + sizeof(int) * (size_t)p->n_tickets : 0;
+    info->workspace_bytes = p->epilog == GEMM_EPI_DRELU_BGRAD ? p->partial_bytes + sizeof(int) * (size_t)p->n_tickets
+                            : p->epilog == GEMM_EPI_WGRAD    ? p->partial_bytes
+                                                             : 0;
   }
   return GEMM_EPI_OK;
 }
@@ -753,7 +761,8 @@ int gemm_epi_execute(gemm_epi_plan_t plan, const void* X, const void* W, const v
   if (p->epilog == GEMM_EPI_DRELU_BGRAD || p->epilog == GEMM_EPI_WGRAD)
     return fail(GEMM_EPI_ERR_EPILOG_MISMATCH, "gemm_epi_execute called on a %s plan",
                 p->epilog == GEMM_EPI_WGRAD ? "WGRAD" : "DRELU_BGRAD");
-  if (!X || !W || !bias || !Y) return fail(GEMM_EPI_ERR_INVALID_ARG, "gemm_epi_execute: NULL X, W, bias or Y");
+  if (!X || !W || !Y || (!bias && p->epilog != GEMM_EPI_NONE))
+    return fail(GEMM_EPI_ERR_INVALID_ARG, "gemm_epi_execute: NULL X, W, bias or Y");
   if (p->epilog == GEMM_EPI_RELU_AUX_BIAS && !aux)
     return fail(GEMM_EPI_ERR_EPILOG_MISMATCH, "RELU_AUX_BIAS needs an aux buffer");
   if (!aligned(X, 16) || !aligned(W, 16) || !aligned(Y, 16) || !aligned(bias, p->bias_f32 ? 4 : 2) ||
@@ -816,8 +825,8 @@ int gemm_epi_unfused_execute(gemm_epi_plan_t plan, const void* X, const void* W,
                              void* Y, uint32_t* aux, cudaStream_t stream) {
   gemm_epi_plan_s* p = lookup(plan);
   if (!p) return fail(GEMM_EPI_ERR_INVALID_ARG, "gemm_epi_unfused_execute: unknown plan");
-  if (p->epilog == GEMM_EPI_DRELU_BGRAD || p->epilog == GEMM_EPI_WGRAD)
-    return fail(GEMM_EPI_ERR_EPILOG_MISMATCH, "gemm_epi_unfused_execute called on a backward plan");
+  if (p->epilog == GEMM_EPI_DRELU_BGRAD || p->epilog == GEMM_EPI_WGRAD || p->epilog == GEMM_EPI_NONE)
+    return fail(GEMM_EPI_ERR_EPILOG_MISMATCH, "gemm_epi_unfused_execute: the plan's epilog has nothing to unfuse");
   if (!X || !W || !bias || !T1 || !T2 || !Y) return fail(GEMM_EPI_ERR_INVALID_ARG, "unfused: NULL pointer");
   if (p->epilog == GEMM_EPI_RELU_AUX_BIAS && !aux)
     return fail(GEMM_EPI_ERR_EPILOG_MISMATCH, "RELU_AUX_BIAS needs an aux buffer");
@@ -876,21 +885,34 @@ int gemm_epi_set_bias_f32(gemm_epi_plan_t plan, int bias_f32) {
   return GEMM_EPI_OK;
 }
 
-int gemm_epi_wgrad_execute(gemm_epi_plan_t plan, const void* X, const void* dZ, void* dW, cudaStream_t stream) {
+int gemm_epi_wgrad_execute(gemm_epi_plan_t plan, const void* X, const void* dZ, void* dW, float* dbias,
+                           cudaStream_t stream) {
   gemm_epi_plan_s* p = lookup(plan);
   if (!p) return fail(GEMM_EPI_ERR_INVALID_ARG, "gemm_epi_wgrad_execute: unknown plan");
   if (p->epilog != GEMM_EPI_WGRAD)
     return fail(GEMM_EPI_ERR_EPILOG_MISMATCH, "gemm_epi_wgrad_execute called on a plan whose epilog is not WGRAD");
   if (!X || !dZ || !dW) return fail(GEMM_EPI_ERR_INVALID_ARG, "gemm_epi_wgrad_execute: NULL X, dZ or dW");
-  if (!aligned(X, 16) || !aligned(dZ, 16) || !aligned(dW, 16))
-    return fail(GEMM_EPI_ERR_MISALIGNED, "gemm_epi_wgrad_execute: X, dZ, dW need 16-byte alignment");
+  if (!aligned(X, 16) || !aligned(dZ, 16) || !aligned(dW, 16) || (dbias && !aligned(dbias, 4)))
+    return fail(GEMM_EPI_ERR_MISALIGNED, "gemm_epi_wgrad_execute: X, dZ, dW need 16-byte, dbias 4-byte alignment");
   int rc = take_status(p);
   if (rc) return rc;
   rc = prepare_maps(p, X, dZ);
   if (rc) return rc;
   ge::TileParams k = base_params(p);
   k.out = dW;
-  return launch_tile(p, p->cfg, k, stream);
+  rc = launch_tile(p, p->cfg, k, stream);
+  if (rc || !dbias) return rc;
+  // dbias[k] = sum over the uT rows of X[t][k]: per-128-row partials, then a fixed-order sum
+  const int row_blocks = ceil_div(p->uT, 128);
+  dim3 cgrid(ceil_div(p->uK, 256), row_blocks);
+  if (p->dtype == GEMM_EPI_BF16)
+    ge::colsum_partial_kernel<true><<<cgrid, 256, 0, stream>>>((const uint16_t*)X, p->uT, (int)p->uK, p->partials);
+  else
+    ge::colsum_partial_kernel<false><<<cgrid, 256, 0, stream>>>((const uint16_t*)X, p->uT, (int)p->uK, p->partials);
+  ge::dbias_finish_kernel<<<ceil_div(p->uK, 256), 256, 0, stream>>>(p->partials, row_blocks, (int)p->uK, dbias);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "wgrad bias-gradient launch");
+  return GEMM_EPI_OK;
 }
 
 int drelu_bgrad_unfused_execute(gemm_epi_plan_t plan, const void* dY2, const void* W2, const uint32_t* aux, void* G,

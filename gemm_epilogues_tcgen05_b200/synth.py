@@ -100,6 +100,25 @@ def masked_grad(T: int, N: int, D2: int, dtype, seed: int, device="cpu") -> torc
     return torch.where(keep, g, torch.zeros_like(g)).to(dtype)
 
 
+def ffn_step_inputs(T: int, D: int, F: int, dtype: str, seed: int, kind: str = "normal", device="cpu") -> dict:
+    """Inputs of one two-layer block step, weights in the [out, in] layout:
+    X (T x D), W1 (F x D), b1 (F), W2 (D x F), b2 (D) and the loss gradient
+    dY (T x D). "normal": X, dY ~ N(0, 1), W1 ~ N(0, 1/D), W2 ~ N(0, 1/F),
+    biases ~ N(0, 0.1). "int": integers in [-1, 1] (biases [-2, 2]), so that
+    every sum and product of the step is exact."""
+    dt = DTYPES[dtype]
+    shapes = {"X": (T, D), "W1": (F, D), "b1": (F,), "W2": (D, F), "b2": (D,), "dY": (T, D)}
+    std = {"X": 1.0, "W1": D ** -0.5, "b1": BIAS_STD, "W2": F ** -0.5, "b2": BIAS_STD, "dY": 1.0}
+    out = {}
+    for i, (k, shp) in enumerate(shapes.items()):
+        if kind == "int":
+            r = 2 if k in ("b1", "b2") else 1
+            out[k] = integers(shp, -r, r, dt, seed * 8 + i, device)
+        else:
+            out[k] = normal(shp, std[k], dt, seed * 8 + i, device)
+    return out
+
+
 def make_inputs(w: Workload, device="cpu", parts=("fwd", "bwd"), T: int | None = None) -> dict:
     """Inputs of one workload: X, W, bias (fwd) and dY2, W2 (bwd).
 

@@ -71,7 +71,8 @@ typedef enum {
   GEMM_EPI_RELU_AUX_BIAS = 2, /* Y = relu(X.W + bias), aux = mask (Z > 0)    */
   GEMM_EPI_DRELU_BGRAD = 3,   /* dZ = (dY2.W2) masked by aux, dbias = sum_t dZ */
   GEMM_EPI_GELU_BIAS = 4,     /* Y = gelu(X.W + bias); aux is ignored         */
-  GEMM_EPI_WGRAD = 5          /* dW = X^T . dZ, see gemm_epi_wgrad_execute    */
+  GEMM_EPI_WGRAD = 5,         /* dW = X^T . dZ, see gemm_epi_wgrad_execute    */
+  GEMM_EPI_NONE = 6           /* Y = X.W, no bias (may be NULL) or activation */
 } gemm_epi_epilog;
 
 enum {
@@ -180,12 +181,16 @@ GEMM_EPI_API int gemm_epi_set_bias_f32(gemm_epi_plan_t plan, int bias_f32);
  * dZ that drelu_bgrad_execute returns. Plan it with epilog GEMM_EPI_WGRAD and
  * the forward's (T, N, K): the contraction runs over the T rows.
  *   X (T x K), dZ (T x N), dW (K x N): device, 16-byte aligned, row-major.
+ *   dbias: NULL, or K floats (4-byte aligned) receiving sum over t of
+ *   X[t][k] in fp32, reduced in a fixed order (a second launch in the same
+ *   call). With a layer weight in the [out, in] layout, dW = dY^T . H is
+ *   called with X = dY, and dbias is then that layer's bias gradient.
  * Returns as gemm_epi_execute; GEMM_EPI_ERR_EPILOG_MISMATCH on a plan whose
  * epilog is not WGRAD (and gemm_epi_execute / drelu_bgrad_execute return it
  * on a WGRAD plan).
  */
 GEMM_EPI_API int gemm_epi_wgrad_execute(gemm_epi_plan_t plan, const void* X, const void* dZ, void* dW,
-                                        cudaStream_t stream);
+                                        float* dbias, cudaStream_t stream);
 
 /* Release a plan and its workspace. NULL and already-freed plans are
  * ignored. The caller must make sure no work of the plan is still running

@@ -27,6 +27,13 @@ their order and notation:
   layers" (FAQ) says DRELU_BGRAD does not cover. The plain definition:
   dW[k, n] = sum_t X[t, k] * dZ[t, n], i.e. the contraction above applied to
   the transposed X.
+* ``ffn_step`` -- one training step of a two-layer block (ReLU between
+  the layers, weights in the [out, in] layout) chained from the calls
+  above: forward through both layers, then the backward pass that
+  DRELU_BGRAD plus the weight gradients make up. Intermediates the step
+  stores in the 16-bit type (H, dZ1) are encoded exactly (``encode_exact``
+  refuses values the type cannot hold), so the chain needs no rounding
+  routine; tests feed it integer-valued inputs.
 * ``relu_aux_words`` -- the mask's bit layout. The pages call it opaque and
   meant only for the dedicated backward epilog ("nvmath-python fused epilogs
   for linear layers", forward section), so its layout is this library's own
@@ -55,6 +62,7 @@ EPILOG_BIAS = "BIAS"
 EPILOG_RELU_BIAS = "RELU_BIAS"
 EPILOG_RELU_AUX_BIAS = "RELU_AUX_BIAS"
 EPILOG_GELU_BIAS = "GELU_BIAS"
+EPILOG_NONE = "NONE"
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "oracle.c")
@@ -183,8 +191,10 @@ def linear_fwd(X, W, bias, dtype: int, epilog: str, rows=None, cols=None, thread
       bits  Z > 0 (strict: a zero pre-activation gives bit 0), for RELU_AUX_BIAS
       aux   the packed words (only when every column was computed)
     """
-    if epilog not in (EPILOG_BIAS, EPILOG_RELU_BIAS, EPILOG_RELU_AUX_BIAS, EPILOG_GELU_BIAS):
+    if epilog not in (EPILOG_BIAS, EPILOG_RELU_BIAS, EPILOG_RELU_AUX_BIAS, EPILOG_GELU_BIAS, EPILOG_NONE):
         raise ValueError(f"unknown forward epilog {epilog}")
+    if epilog == EPILOG_NONE:
+        bias = None  # the plain product
     if bias is not None and np.asarray(bias).dtype == np.float32:
         # an fp32 bias ("Fusing bias addition ...", engineering checklist: a
         # float32 bias with 16-bit operands): the product, then the bias added
@@ -199,7 +209,7 @@ def linear_fwd(X, W, bias, dtype: int, epilog: str, rows=None, cols=None, thread
     else:
         Z, S = matmul_bias(X, W, bias, dtype, rows=rows, cols=cols, threads=threads)
     out = {"Z": Z, "S": S}
-    if epilog == EPILOG_BIAS:
+    if epilog in (EPILOG_BIAS, EPILOG_NONE):
         out["Y"] = Z.copy()
     elif epilog == EPILOG_GELU_BIAS:
         out["Y"] = gelu(Z)
@@ -212,12 +222,51 @@ def linear_fwd(X, W, bias, dtype: int, epilog: str, rows=None, cols=None, thread
     return out
 
 
+def encode_exact(values, dtype: int) -> np.ndarray:
+    """fp64 values to 16-bit patterns of ``dtype``; ValueError unless every
+    value is exactly representable (then the encoding needs no rounding)."""
+    v = np.asarray(values, dtype=np.float64)
+    if dtype == F16:
+        bits = v.astype(np.float16).view(np.uint16)
+    elif dtype == BF16:
+        f32 = v.astype(np.float32)
+        bits = (f32.view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+    else:
+        raise ValueError(f"unknown dtype {dtype}")
+    if not np.array_equal(decode(bits, dtype), v):
+        raise ValueError("value not exactly representable in the 16-bit type")
+    return bits
+
+
+def ffn_step(X, W1, b1, W2, b2, dY, dtype: int):
+    """One step of Y = relu(X W1^T + b1) W2^T + b2 and its backward for the
+    loss gradient dY. X: T x D, W1: F x D, b1: F, W2: D x F, b2: D, dY: T x D
+    (16-bit patterns; weights in the [out, in] layout). Returns fp64 H, bits,
+    Y, dZ1, db1, dW2, db2, dW1, dX."""
+    W1 = np.asarray(W1, dtype=np.uint16)
+    W2 = np.asarray(W2, dtype=np.uint16)
+    f1 = linear_fwd(X, np.ascontiguousarray(W1.T), b1, dtype, EPILOG_RELU_AUX_BIAS)
+    H = encode_exact(f1["Y"], dtype)
+    f2 = linear_fwd(H, np.ascontiguousarray(W2.T), b2, dtype, EPILOG_BIAS)
+    F = W1.shape[0]
+    bwd = drelu_bgrad(dY, W2, f1["aux"], dtype, F)     # G = dY . W2 (W2 read as D x F = K x N)
+    dZ1 = encode_exact(bwd["dZ"], dtype)
+    g2 = wgrad(dY, H, dtype)                           # dW2 = dY^T H, db2 = sum_t dY
+    g1 = wgrad(dZ1, X, dtype)                          # dW1 = dZ1^T X
+    dX = linear_fwd(dZ1, W1, None, dtype, EPILOG_NONE)  # dX = dZ1 . W1 (W1 read as F x D = K x N)
+    return {"H": f1["Y"], "bits": f1["bits"], "Y": f2["Y"], "dZ1": bwd["dZ"], "db1": bwd["dbias"],
+            "dW2": g2["dW"], "db2": g2["dbias"], "dW1": g1["dW"], "dX": dX["Y"]}
+
+
 def wgrad(X, dZ, dtype: int, rows=None, cols=None, threads=None):
     """dW = X^T . dZ for X (T x K) and dZ (T x N): K x N, summed over t.
 
     Returns a dict with
       dW    the product (fp64)
       S     sum_t |x dz|, its error scale
+      dbias sum over t of X[t, k] (the bias gradient when X is a layer's
+            output gradient), and Sb = sum_t |X[t, k]|; both for the
+            selected rows k
     ``rows`` / ``cols`` select rows k / columns n of dW.
     """
     X = np.asarray(X, dtype=np.uint16)
@@ -225,7 +274,10 @@ def wgrad(X, dZ, dtype: int, rows=None, cols=None, threads=None):
     if X.shape[0] != dZ.shape[0]:
         raise ValueError(f"X and dZ need the same row count: {X.shape[0]} vs {dZ.shape[0]}")
     dW, S = matmul_bias(np.ascontiguousarray(X.T), dZ, None, dtype, rows=rows, cols=cols, threads=threads)
-    return {"dW": dW, "S": S}
+    xv = decode(X, dtype)
+    if rows is not None:
+        xv = xv[:, np.asarray(rows, dtype=np.int64)]
+    return {"dW": dW, "S": S, "dbias": xv.sum(axis=0), "Sb": np.abs(xv).sum(axis=0)}
 
 
 def drelu_bgrad(dY2, W2, aux, dtype: int, N: int, rows=None, cols=None, threads=None):

@@ -232,11 +232,13 @@ def run_wgrad(inp_cpu: dict, dtype, device="cuda", dz_key="dY2"):
     with Plan(T, N, K, dtype, "WGRAD") as plan:
         info = plan.info()
         wbuf, dW = guarded((K, N), dtype, device)
-        plan.gemm_epi_wgrad_execute(X, dZ, dW)
+        bbuf, dbias = guarded((K,), torch.float32, device)
+        plan.gemm_epi_wgrad_execute(X, dZ, dW, dbias)
         torch.cuda.synchronize()
         assert plan.status() == 0, "watchdog fired"
     assert guards_intact(wbuf), "dW guard region overwritten"
-    return {"dW": dW.cpu(), "info": info}
+    assert guards_intact(bbuf), "dbias guard region overwritten"
+    return {"dW": dW.cpu(), "dbias": dbias.cpu(), "info": info}
 
 
 def check_wgrad(inp_cpu, dtype, gpu, rows=None, cols=None, exact=False, dz_key="dY2"):
@@ -250,4 +252,40 @@ def check_wgrad(inp_cpu, dtype, gpu, rows=None, cols=None, exact=False, dz_key="
         assert np.array_equal(got, expect), "dW not bit-exact on integer inputs"
     else:
         assert_within(got, ref["dW"], ref["S"], Y_REL, "dW", unit_roundoff(dtype))
+    db = gpu["dbias"].double().numpy()
+    db = db if rows is None else db[rows]
+    if exact:
+        assert np.array_equal(db, ref["dbias"]), "wgrad dbias not exact on integer inputs"
+    else:  # fp32 sums of 16-bit values in a fixed order
+        assert_within(db, ref["dbias"], ref["Sb"], 1e-3, "wgrad dbias")
     return ref
+
+
+def run_ffn_step(inp_cpu: dict, dtype, device="cuda"):
+    """One two-layer block step through the public API (six plans, weights in
+    the [out, in] layout): H, aux = layer 1 (RELU_AUX_BIAS); Y = layer 2
+    (BIAS); dZ1, db1 = DRELU_BGRAD(dY, W2, aux); dW2, db2 = WGRAD(dY, H);
+    dW1 = WGRAD(dZ1, X); dX = NONE(dZ1, W1)."""
+    g = {k: v.to(device) for k, v in inp_cpu.items()}
+    T, D = g["X"].shape
+    F = g["W1"].shape[0]
+    plans = [Plan(T, F, D, dtype, "RELU_AUX_BIAS", w_nk=True), Plan(T, D, F, dtype, "BIAS", w_nk=True),
+             Plan(T, F, D, dtype, "DRELU_BGRAD"), Plan(T, F, D, dtype, "WGRAD"), Plan(T, D, F, dtype, "WGRAD"),
+             Plan(T, D, F, dtype, "NONE")]
+    try:
+        H, aux = plans[0].forward(g["X"], g["W1"], g["b1"])
+        Y, _ = plans[1].forward(H, g["W2"], g["b2"])
+        dZ1, db1 = plans[2].backward(g["dY"], g["W2"], aux)
+        dW2, db2 = plans[3].wgrad(g["dY"], H, with_dbias=True)
+        dW1 = plans[4].wgrad(dZ1, g["X"])
+        dX, _ = plans[5].forward(dZ1, g["W1"], None)
+        torch.cuda.synchronize()
+        assert all(p.status() == 0 for p in plans), "watchdog fired"
+        kernels = [p.info()["kernel"] for p in plans]
+    finally:
+        for p in plans:
+            p.free()
+    out = {"H": H, "aux": aux, "Y": Y, "dZ1": dZ1, "db1": db1, "dW2": dW2, "db2": db2, "dW1": dW1, "dX": dX}
+    out = {k: v.cpu() for k, v in out.items()}
+    out["kernels"] = kernels
+    return out

@@ -8,7 +8,8 @@ import torch
 import oracle
 from gemm_epilogues_tcgen05_b200 import binding, synth
 
-from _parity import check_backward, check_forward, check_wgrad, run_backward, run_forward, run_wgrad
+from _parity import (check_backward, check_forward, check_wgrad, odt, run_backward, run_ffn_step, run_forward,
+                     run_wgrad)
 
 pytestmark = pytest.mark.gpu
 
@@ -306,6 +307,25 @@ def test_weight_nk_integer_inputs_bit_exact(monkeypatch, dtype, variant):
     check_backward(inp, fwd["aux"], DT[dtype], run_backward(inp, fwd["aux"], DT[dtype], w_nk=True), exact=True)
 
 
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+@pytest.mark.parametrize("T,D,F", [(256, 136, 264), (300, 512, 1032), (64, 128, 200)])
+def test_ffn_step_chain_bit_exact(T, D, F, dtype):
+    """A whole two-layer block step, six library calls chained on integer
+    inputs: every intermediate and output equals the oracle's exact value
+    (rounded once to the 16-bit type where the step stores it)."""
+    inp = synth.ffn_step_inputs(T, D, F, dtype, seed=T + D + F, kind="int")
+    bits = {k: synth.bits_u16(v) for k, v in inp.items()}
+    dt = DT[dtype]
+    ref = oracle.ffn_step(bits["X"], bits["W1"], bits["b1"], bits["W2"], bits["b2"], bits["dY"], odt(dt))
+    gpu = run_ffn_step(inp, dt)
+    for k in ("H", "Y", "dZ1", "dW2", "dW1", "dX"):
+        expect = torch.from_numpy(ref[k]).to(dt)
+        assert torch.equal(gpu[k].view(torch.int16), expect.view(torch.int16)), f"{k} differs"
+    for k in ("db1", "db2"):
+        assert np.array_equal(gpu[k].double().numpy(), ref[k]), f"{k} differs"
+    assert np.array_equal(oracle.relu_aux_bits(gpu["aux"].numpy().view(np.uint32), F), ref["bits"])
+
+
 def test_plan_flags_are_checked():
     with pytest.raises(binding.GemmEpiError):
         binding.gemm_epi_plan(64, 64, 64, binding.F16, binding.RELU_BIAS, flags=2)
@@ -352,20 +372,21 @@ def test_wgrad_plan_rejects_other_calls():
         p = X.data_ptr()
         assert L.gemm_epi_execute(h, p, p, p, p, p, s) == binding.ERR_EPILOG_MISMATCH
         assert L.drelu_bgrad_execute(h, p, p, p, p, p, s) == binding.ERR_EPILOG_MISMATCH
-        assert L.gemm_epi_wgrad_execute(h, p + 2, p, p, s) == binding.ERR_MISALIGNED
-        assert L.gemm_epi_wgrad_execute(h, p, None, p, s) == binding.ERR_INVALID_ARG
+        assert L.gemm_epi_wgrad_execute(h, p + 2, p, p, None, s) == binding.ERR_MISALIGNED
+        assert L.gemm_epi_wgrad_execute(h, p, None, p, None, s) == binding.ERR_INVALID_ARG
         assert L.gemm_epi_set_bias_f32(h, 1) == binding.ERR_EPILOG_MISMATCH
+        assert L.gemm_epi_wgrad_execute(h, p, p, p, p + 2, s) == binding.ERR_MISALIGNED  # dbias
     finally:
         binding.gemm_epi_free(h)
     hf = binding.gemm_epi_plan(T, N, K, binding.F16, binding.RELU_BIAS)
     try:
-        assert L.gemm_epi_wgrad_execute(hf, p, p, p, None) == binding.ERR_EPILOG_MISMATCH
+        assert L.gemm_epi_wgrad_execute(hf, p, p, p, None, None) == binding.ERR_EPILOG_MISMATCH
     finally:
         binding.gemm_epi_free(hf)
 
 
 def test_unknown_epilog_values_rejected():
-    for bad in (-1, 6, 99):
+    for bad in (-1, 7, 99):
         with pytest.raises(binding.GemmEpiError):
             binding.gemm_epi_plan(64, 64, 64, binding.F16, bad)
 

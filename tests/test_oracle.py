@@ -514,6 +514,8 @@ def pin_wgrad(wg):
     r = wg(X, dZ, 0)
     if not np.array_equal(r["dW"], np.array([[6.0, 8.0, 7.0], [8.0, 10.0, 10.0]])):
         fails.append("hand-worked")
+    if not np.array_equal(r["dbias"], np.array([9.0, 12.0])):  # 1+3+5, 2+4+6
+        fails.append("hand-worked column sums")
     # closed form: X = 1, dZ = 2 -> dW = 2T everywhere; S = 2T
     T = 37
     r = wg(_bits(np.ones((T, 5)).tolist(), "bf16"), _bits((2 * np.ones((T, 9))).tolist(), "bf16"), 1)
@@ -548,11 +550,12 @@ def test_wgrad_planted_mistakes_are_caught(oracle_mod):
 
     def sign(X, dZ, dt, **kw):
         r = o.wgrad(X, dZ, dt, **kw)
-        return {"dW": -r["dW"], "S": r["S"]}
+        return dict(r, dW=-r["dW"])
 
     def dz_transposed_product(X, dZ, dt, **kw):  # (dZ^T X)^T computed with X and dZ swapped roles
         r = o.wgrad(dZ, X, dt, **kw)
-        return {"dW": r["dW"].T.copy(), "S": r["S"].T.copy()}
+        ref = o.wgrad(X, dZ, dt, **kw)
+        return dict(ref, dW=r["dW"].T.copy(), S=r["S"].T.copy())
 
     for name, m in {"rows flipped": no_transpose_rows_flipped, "last row dropped": last_row_dropped,
                     "sign": sign}.items():
@@ -567,6 +570,7 @@ def test_wgrad_subsets_match_full(oracle_mod):
     full = oracle_mod.wgrad(X, dZ, 1)
     part = oracle_mod.wgrad(X, dZ, 1, rows=[0, 5, 23], cols=[1, 39])
     assert np.array_equal(part["dW"], full["dW"][np.ix_([0, 5, 23], [1, 39])])
+    assert np.array_equal(part["dbias"], full["dbias"][[0, 5, 23]])
     with pytest.raises(ValueError):
         oracle_mod.wgrad(X, dZ[:-1], 1)
 
@@ -596,3 +600,50 @@ def test_fp32_bias_values_are_taken_exactly(oracle_mod):
     assert np.array_equal(r["Y"], np.maximum(r["Z"], 0.0))
     with pytest.raises(ValueError):
         oracle_mod.linear_fwd(X, W, b32[:5], 1, "BIAS")
+
+
+# ------------------------------------------------------- NONE and the FFN step
+def test_none_epilog_is_the_plain_product(oracle_mod):
+    inp = synth.make_shape_inputs(6, 16, 24, "bf16", seed=44)
+    X, W, b = (synth.bits_u16(inp[k]) for k in ("X", "W", "bias"))
+    r = oracle_mod.linear_fwd(X, W, b, 1, "NONE")   # the bias is not used
+    zero = _bits([0.0] * 16, "bf16")
+    rz = oracle_mod.linear_fwd(X, W, zero, 1, "BIAS")
+    assert np.array_equal(r["Y"], rz["Y"]) and np.array_equal(r["S"], rz["S"])
+
+
+def test_encode_exact(oracle_mod):
+    v = np.array([0.0, -3.0, 256.0, 0.5, -65504.0])
+    assert np.array_equal(oracle_mod.decode(oracle_mod.encode_exact(v, 0), 0), v)
+    assert np.array_equal(oracle_mod.decode(oracle_mod.encode_exact(v[:4], 1), 1), v[:4])
+    with pytest.raises(ValueError):
+        oracle_mod.encode_exact(np.array([257.0]), 1)   # bf16 holds 8 significant bits
+    with pytest.raises(ValueError):
+        oracle_mod.encode_exact(np.array([2049.0]), 0)  # fp16 holds 11
+
+
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+def test_ffn_step_matches_float64_autograd(oracle_mod, dtype):
+    """The chained step against torch's float64 autograd of the same block
+    (exact on integer inputs): pins every transpose and orientation."""
+    T, D, F = 12, 16, 24
+    inp = synth.ffn_step_inputs(T, D, F, dtype, seed=3, kind="int")
+    bits = {k: synth.bits_u16(v) for k, v in inp.items()}
+    dt = DT[dtype]
+    r = oracle_mod.ffn_step(bits["X"], bits["W1"], bits["b1"], bits["W2"], bits["b2"], bits["dY"], dt)
+    t = {k: v.double().requires_grad_(k != "dY") for k, v in inp.items()}
+    h = torch.relu(t["X"] @ t["W1"].T + t["b1"])
+    y = h @ t["W2"].T + t["b2"]
+    y.backward(t["dY"])
+    assert np.array_equal(r["H"], h.detach().numpy()) and np.array_equal(r["Y"], y.detach().numpy())
+    for ours, theirs in (("dX", "X"), ("dW1", "W1"), ("db1", "b1"), ("dW2", "W2"), ("db2", "b2")):
+        assert np.array_equal(r[ours], t[theirs].grad.numpy()), ours
+    assert np.array_equal(r["bits"], h.detach().numpy() > 0)
+
+
+def test_ffn_step_refuses_inexact_intermediates(oracle_mod):
+    T, D, F = 4, 8, 8
+    inp = synth.ffn_step_inputs(T, D, F, "bf16", seed=1, kind="normal")
+    bits = {k: synth.bits_u16(v) for k, v in inp.items()}
+    with pytest.raises(ValueError):
+        oracle_mod.ffn_step(bits["X"], bits["W1"], bits["b1"], bits["W2"], bits["b2"], bits["dY"], 1)
