@@ -32,6 +32,7 @@ EXPORTED = ["gemm_epi_plan", "gemm_epi_execute", "drelu_bgrad_execute", "gemm_ep
             "gemm_epi_query", "gemm_epi_status", "gemm_epi_unfused_execute", "drelu_bgrad_unfused_execute",
             "drelu_bgrad_execute_noalloc", "gemm_epi_wgrad_execute", "gemm_epi_set_bias_f32", "gemm_epi_plan_ex"]
 FLAG_W_NK = 1  # GEMM_EPI_FLAG_W_NK
+FLAG_OUT_F32 = 2  # GEMM_EPI_FLAG_OUT_F32
 
 NOALLOC_SCRATCH_BYTES = 4 << 20  # GEMM_EPI_NOALLOC_SCRATCH_BYTES
 
@@ -164,15 +165,19 @@ def drelu_bgrad_execute_noalloc(dY2, W2, aux, dZ, dbias, stream=None):
 class Plan:
     """A plan for one (T, N, K, dtype, epilog); execute any number of times."""
 
-    def __init__(self, T: int, N: int, K: int, dtype: torch.dtype, epilog: str | int, w_nk: bool = False):
-        """w_nk: the weight (W, or W2 of DRELU_BGRAD) is N x K, K contiguous."""
+    def __init__(self, T: int, N: int, K: int, dtype: torch.dtype, epilog: str | int, w_nk: bool = False,
+                 out_f32: bool = False):
+        """w_nk: the weight (W, or W2 of DRELU_BGRAD) is N x K, K contiguous.
+        out_f32: the output (Y, dZ or dW) is fp32."""
         self.T, self.N, self.K = T, N, K
+        self.out_dtype = torch.float32 if out_f32 else dtype
         self.w_shape = (N, K) if w_nk else (K, N)
         self.dtype = dtype
         self.epilog = EPILOGS[epilog] if isinstance(epilog, str) else epilog
         self.aux_words = (N + 31) // 32
         self.bias_dtype = dtype
-        self.handle = gemm_epi_plan(T, N, K, dtype, self.epilog, FLAG_W_NK if w_nk else 0)
+        self.handle = gemm_epi_plan(T, N, K, dtype, self.epilog,
+                                    (FLAG_W_NK if w_nk else 0) | (FLAG_OUT_F32 if out_f32 else 0))
 
     def set_bias_f32(self, on: bool = True):
         """Read the forward bias as fp32 (True) or in the plan's 16-bit type (False)."""
@@ -210,27 +215,28 @@ class Plan:
     def gemm_epi_execute(self, X, W, bias, Y, aux=None, stream=None):
         T, N, K, dt = self.T, self.N, self.K, self.dtype
         args = (_ptr(X, (T, K), dt, "X"), _ptr(W, self.w_shape, dt, "W"), _ptr(bias, (N,), self.bias_dtype, "bias"),
-                _ptr(Y, (T, N), dt, "Y"), _ptr(aux, (T, self.aux_words), torch.int32, "aux"))
+                _ptr(Y, (T, N), self.out_dtype, "Y"), _ptr(aux, (T, self.aux_words), torch.int32, "aux"))
         _check(lib().gemm_epi_execute(self.handle, *args, _stream_ptr(stream)))
 
     def drelu_bgrad_execute(self, dY2, W2, aux, dZ, dbias, stream=None):
         T, N, K, dt = self.T, self.N, self.K, self.dtype
         args = (_ptr(dY2, (T, K), dt, "dY2"), _ptr(W2, self.w_shape, dt, "W2"),
-                _ptr(aux, (T, self.aux_words), torch.int32, "aux"), _ptr(dZ, (T, N), dt, "dZ"),
+                _ptr(aux, (T, self.aux_words), torch.int32, "aux"), _ptr(dZ, (T, N), self.out_dtype, "dZ"),
                 _ptr(dbias, (N,), torch.float32, "dbias"))
         _check(lib().drelu_bgrad_execute(self.handle, *args, _stream_ptr(stream)))
 
     def gemm_epi_wgrad_execute(self, X, dZ, dW, dbias=None, stream=None):
         """WGRAD plan: dW (K x N) = X^T . dZ; dbias (K floats, optional) = sum over t of X."""
         T, N, K, dt = self.T, self.N, self.K, self.dtype
-        args = (_ptr(X, (T, K), dt, "X"), _ptr(dZ, (T, N), dt, "dZ"), _ptr(dW, (K, N), dt, "dW"),
+        args = (_ptr(X, (T, K), dt, "X"), _ptr(dZ, (T, N), dt, "dZ"),
+                _ptr(dW, (K, N), self.out_dtype, "dW"),
                 _ptr(dbias, (K,), torch.float32, "dbias"))
         _check(lib().gemm_epi_wgrad_execute(self.handle, *args, _stream_ptr(stream)))
 
     def gemm_epi_unfused_execute(self, X, W, bias, T1, T2, Y, aux=None, stream=None):
         T, N, K, dt = self.T, self.N, self.K, self.dtype
         args = (_ptr(X, (T, K), dt, "X"), _ptr(W, self.w_shape, dt, "W"), _ptr(bias, (N,), self.bias_dtype, "bias"),
-                _ptr(T1, (T, N), dt, "T1"), _ptr(T2, (T, N), dt, "T2"), _ptr(Y, (T, N), dt, "Y"),
+                _ptr(T1, (T, N), dt, "T1"), _ptr(T2, (T, N), dt, "T2"), _ptr(Y, (T, N), self.out_dtype, "Y"),
                 _ptr(aux, (T, self.aux_words), torch.int32, "aux"))
         _check(lib().gemm_epi_unfused_execute(self.handle, *args, _stream_ptr(stream)))
 
@@ -238,7 +244,7 @@ class Plan:
         T, N, K, dt = self.T, self.N, self.K, self.dtype
         args = (_ptr(dY2, (T, K), dt, "dY2"), _ptr(W2, self.w_shape, dt, "W2"),
                 _ptr(aux, (T, self.aux_words), torch.int32, "aux"), _ptr(G, (T, N), dt, "G"),
-                _ptr(dZ, (T, N), dt, "dZ"), _ptr(dbias, (N,), torch.float32, "dbias"))
+                _ptr(dZ, (T, N), self.out_dtype, "dZ"), _ptr(dbias, (N,), torch.float32, "dbias"))
         _check(lib().drelu_bgrad_unfused_execute(self.handle, *args, _stream_ptr(stream)))
 
     # prebuilt calls: (fn, args) so that fn(*args) enqueues the C call with no
@@ -246,26 +252,27 @@ class Plan:
     def execute_call(self, X, W, bias, Y, aux=None, stream=None):
         T, N, K, dt = self.T, self.N, self.K, self.dtype
         args = (self.handle, _ptr(X, (T, K), dt, "X"), _ptr(W, self.w_shape, dt, "W"), _ptr(bias, (N,), self.bias_dtype, "bias"),
-                _ptr(Y, (T, N), dt, "Y"), _ptr(aux, (T, self.aux_words), torch.int32, "aux"), _stream_ptr(stream))
+                _ptr(Y, (T, N), self.out_dtype, "Y"), _ptr(aux, (T, self.aux_words), torch.int32, "aux"), _stream_ptr(stream))
         return lib().gemm_epi_execute, args
 
     def drelu_bgrad_call(self, dY2, W2, aux, dZ, dbias, stream=None):
         T, N, K, dt = self.T, self.N, self.K, self.dtype
         args = (self.handle, _ptr(dY2, (T, K), dt, "dY2"), _ptr(W2, self.w_shape, dt, "W2"),
-                _ptr(aux, (T, self.aux_words), torch.int32, "aux"), _ptr(dZ, (T, N), dt, "dZ"),
+                _ptr(aux, (T, self.aux_words), torch.int32, "aux"), _ptr(dZ, (T, N), self.out_dtype, "dZ"),
                 _ptr(dbias, (N,), torch.float32, "dbias"), _stream_ptr(stream))
         return lib().drelu_bgrad_execute, args
 
     def wgrad_call(self, X, dZ, dW, dbias=None, stream=None):
         T, N, K, dt = self.T, self.N, self.K, self.dtype
-        args = (self.handle, _ptr(X, (T, K), dt, "X"), _ptr(dZ, (T, N), dt, "dZ"), _ptr(dW, (K, N), dt, "dW"),
+        args = (self.handle, _ptr(X, (T, K), dt, "X"), _ptr(dZ, (T, N), dt, "dZ"),
+                _ptr(dW, (K, N), self.out_dtype, "dW"),
                 _ptr(dbias, (K,), torch.float32, "dbias"), _stream_ptr(stream))
         return lib().gemm_epi_wgrad_execute, args
 
     def unfused_call(self, X, W, bias, T1, T2, Y, aux=None, stream=None):
         T, N, K, dt = self.T, self.N, self.K, self.dtype
         args = (self.handle, _ptr(X, (T, K), dt, "X"), _ptr(W, self.w_shape, dt, "W"), _ptr(bias, (N,), self.bias_dtype, "bias"),
-                _ptr(T1, (T, N), dt, "T1"), _ptr(T2, (T, N), dt, "T2"), _ptr(Y, (T, N), dt, "Y"),
+                _ptr(T1, (T, N), dt, "T1"), _ptr(T2, (T, N), dt, "T2"), _ptr(Y, (T, N), self.out_dtype, "Y"),
                 _ptr(aux, (T, self.aux_words), torch.int32, "aux"), _stream_ptr(stream))
         return lib().gemm_epi_unfused_execute, args
 
@@ -273,26 +280,26 @@ class Plan:
         T, N, K, dt = self.T, self.N, self.K, self.dtype
         args = (self.handle, _ptr(dY2, (T, K), dt, "dY2"), _ptr(W2, self.w_shape, dt, "W2"),
                 _ptr(aux, (T, self.aux_words), torch.int32, "aux"), _ptr(G, (T, N), dt, "G"),
-                _ptr(dZ, (T, N), dt, "dZ"), _ptr(dbias, (N,), torch.float32, "dbias"), _stream_ptr(stream))
+                _ptr(dZ, (T, N), self.out_dtype, "dZ"), _ptr(dbias, (N,), torch.float32, "dbias"), _stream_ptr(stream))
         return lib().drelu_bgrad_unfused_execute, args
 
     # conveniences that allocate their outputs (allocation happens in torch,
     # outside the library; the library call itself allocates nothing)
     def forward(self, X, W, bias, stream=None):
-        Y = torch.empty((self.T, self.N), dtype=self.dtype, device=X.device)
+        Y = torch.empty((self.T, self.N), dtype=self.out_dtype, device=X.device)
         aux = (torch.empty((self.T, self.aux_words), dtype=torch.int32, device=X.device)
                if self.epilog == RELU_AUX_BIAS else None)
         self.gemm_epi_execute(X, W, bias, Y, aux, stream)
         return Y, aux
 
     def backward(self, dY2, W2, aux, stream=None):
-        dZ = torch.empty((self.T, self.N), dtype=self.dtype, device=dY2.device)
+        dZ = torch.empty((self.T, self.N), dtype=self.out_dtype, device=dY2.device)
         dbias = torch.empty((self.N,), dtype=torch.float32, device=dY2.device)
         self.drelu_bgrad_execute(dY2, W2, aux, dZ, dbias, stream)
         return dZ, dbias
 
     def wgrad(self, X, dZ, with_dbias=False, stream=None):
-        dW = torch.empty((self.K, self.N), dtype=self.dtype, device=X.device)
+        dW = torch.empty((self.K, self.N), dtype=self.out_dtype, device=X.device)
         dbias = torch.empty((self.K,), dtype=torch.float32, device=X.device) if with_dbias else None
         self.gemm_epi_wgrad_execute(X, dZ, dW, dbias, stream)
         return (dW, dbias) if with_dbias else dW

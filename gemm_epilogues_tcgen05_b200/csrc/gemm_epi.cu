@@ -88,6 +88,21 @@ int encode_out(CUtensorMap* map, const void* out, int64_t T, int64_t N) {
   return encode_2d(map, out, (uint64_t)N, (uint64_t)T, 32, 32, "the output", CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
+// fp32 output: 16 x 32 blocks (64-byte rows, the 16-bit blocks' staging layout)
+int encode_out_f32(CUtensorMap* map, const void* out, int64_t T, int64_t N) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(GEMM_EPI_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[2] = {(uint64_t)N, (uint64_t)T};
+  const cuuint64_t strides[1] = {(uint64_t)N * 4};
+  const cuuint32_t box[2] = {16, 32};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(out), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(GEMM_EPI_ERR_CUDA, "tensor map encode for the fp32 output failed (CUresult %d)", (int)r);
+  return GEMM_EPI_OK;
+}
+
 // the mask words as the tile kernels' TMA stores see them: per warp and tile
 // a block of BN/32 words x 32 rows. Usable when a row of words is a multiple
 // of 16 bytes and the pointer is 16-byte aligned; otherwise the kernels store
@@ -299,6 +314,7 @@ struct gemm_epi_plan_s {
   int tail_split = 1;    // GEMM_EPI_TAIL_SPLIT=0 keeps whole tiles in the pair kernel's last round
   int bias_f32 = 0;      // gemm_epi_set_bias_f32: the forward bias is fp32
   int w_nk = 0;          // GEMM_EPI_FLAG_W_NK: W / W2 given N x K (K contiguous)
+  int out_f32 = 0;       // GEMM_EPI_FLAG_OUT_F32: Y / dZ / dW written as fp32
   // tensor-map cache
   const void* a_ptr = nullptr;
   const void* b_ptr = nullptr;
@@ -382,12 +398,13 @@ ge::TileParams base_params(const gemm_epi_plan_s* p) {
   k.tail_split = p->tail_split;
   k.bias_f32 = p->bias_f32;
   k.b_kmajor = p->w_nk;
+  k.out_f32 = p->out_f32;
   return k;
 }
 
 int prepare_out_map(gemm_epi_plan_s* p, const void* out) {
   if (out != p->y_ptr) {
-    int rc = encode_out(&p->tmY, out, p->T, p->N);
+    int rc = p->out_f32 ? encode_out_f32(&p->tmY, out, p->T, p->N) : encode_out(&p->tmY, out, p->T, p->N);
     if (rc) return rc;
     p->y_ptr = out;
   }
@@ -479,6 +496,7 @@ ge::SkinnyParams skinny_params(const gemm_epi_plan_s* p) {
   k.status = p->status_dev;
   k.timeout_ns = p->timeout_ns;
   k.bias_f32 = p->bias_f32;
+  k.out_f32 = p->out_f32;
   return k;
 }
 
@@ -513,7 +531,7 @@ gemm_epi_plan_t gemm_epi_plan(int64_t T, int64_t N, int64_t K, gemm_epi_dtype dt
 
 gemm_epi_plan_t gemm_epi_plan_ex(int64_t T, int64_t N, int64_t K, gemm_epi_dtype dtype, gemm_epi_epilog epilog,
                                  uint32_t flags) {
-  if ((flags & ~(uint32_t)GEMM_EPI_FLAG_W_NK) != 0) {
+  if ((flags & ~(uint32_t)(GEMM_EPI_FLAG_W_NK | GEMM_EPI_FLAG_OUT_F32)) != 0) {
     fail(GEMM_EPI_ERR_INVALID_ARG, "unknown plan flags 0x%x", flags);
     return nullptr;
   }
@@ -573,6 +591,7 @@ gemm_epi_plan_t gemm_epi_plan_ex(int64_t T, int64_t N, int64_t K, gemm_epi_dtype
   p->dtype = dtype;
   p->epilog = epilog;
   p->w_nk = w_nk ? 1 : 0;
+  p->out_f32 = (flags & GEMM_EPI_FLAG_OUT_F32) ? 1 : 0;
   p->device = dev;
   p->num_sms = sms;
   const bool bf16 = dtype == GEMM_EPI_BF16;
@@ -827,6 +846,8 @@ int gemm_epi_unfused_execute(gemm_epi_plan_t plan, const void* X, const void* W,
   if (!p) return fail(GEMM_EPI_ERR_INVALID_ARG, "gemm_epi_unfused_execute: unknown plan");
   if (p->epilog == GEMM_EPI_DRELU_BGRAD || p->epilog == GEMM_EPI_WGRAD || p->epilog == GEMM_EPI_NONE)
     return fail(GEMM_EPI_ERR_EPILOG_MISMATCH, "gemm_epi_unfused_execute: the plan's epilog has nothing to unfuse");
+  if (p->out_f32)
+    return fail(GEMM_EPI_ERR_UNSUPPORTED, "the unfused path keeps 16-bit intermediates and outputs (no fp32 output)");
   if (!X || !W || !bias || !T1 || !T2 || !Y) return fail(GEMM_EPI_ERR_INVALID_ARG, "unfused: NULL pointer");
   if (p->epilog == GEMM_EPI_RELU_AUX_BIAS && !aux)
     return fail(GEMM_EPI_ERR_EPILOG_MISMATCH, "RELU_AUX_BIAS needs an aux buffer");
@@ -921,6 +942,8 @@ int drelu_bgrad_unfused_execute(gemm_epi_plan_t plan, const void* dY2, const voi
   if (!p) return fail(GEMM_EPI_ERR_INVALID_ARG, "drelu_bgrad_unfused_execute: unknown plan");
   if (p->epilog != GEMM_EPI_DRELU_BGRAD)
     return fail(GEMM_EPI_ERR_EPILOG_MISMATCH, "drelu_bgrad_unfused_execute called on a forward plan");
+  if (p->out_f32)
+    return fail(GEMM_EPI_ERR_UNSUPPORTED, "the unfused path keeps 16-bit intermediates and outputs (no fp32 output)");
   if (!dY2 || !W2 || !aux || !G || !dZ || !dbias) return fail(GEMM_EPI_ERR_INVALID_ARG, "unfused: NULL pointer");
   if (!aligned(dY2, 16) || !aligned(W2, 16) || !aligned(G, 16) || !aligned(dZ, 16) || !aligned(aux, 4) ||
       !aligned(dbias, 4))

@@ -40,6 +40,7 @@ struct SkinnyParams {
   int* status;
   uint64_t timeout_ns;
   int32_t bias_f32;                // the bias is N fp32 values (else the 16-bit type)
+  int32_t out_f32;                 // the output is fp32 (else the 16-bit type)
 };
 
 // A stage holds KPS consecutive 64-deep k-blocks: W as one box of 64 features
@@ -114,6 +115,15 @@ __device__ __forceinline__ void store_16(void* base, int64_t i, float v) {
     reinterpret_cast<__half*>(base)[i] = __float2half_rn(v);
 }
 
+// the output element i, fp32 or rounded to the 16-bit type
+template <bool BF16>
+__device__ __forceinline__ void store_out(const SkinnyParams& p, int64_t i, float v) {
+  if (p.out_f32)
+    reinterpret_cast<float*>(p.out)[i] = v;
+  else
+    store_16<BF16>(p.out, i, v);
+}
+
 // DRELU_BGRAD: the mask words of rows t0 .. t0+15 for this warp's 32
 // features (one word per row). Callers load them ahead of use -- before the
 // accumulator wait, or before the previous rows' stores -- so the loads are
@@ -144,7 +154,7 @@ __device__ __forceinline__ void skinny_finish16(const SkinnyParams& p, float (&v
       const int t = t0 + j;
       if (t < p.T) {
         const float dz = ((m[j] >> lane) & 1u) ? v[j] : 0.f;
-        if (n_ok) store_16<BF16>(p.out, static_cast<int64_t>(t) * p.N + n, dz);
+        if (n_ok) store_out<BF16>(p, static_cast<int64_t>(t) * p.N + n, dz);
         dbias_acc += dz;
       }
     }
@@ -163,7 +173,7 @@ __device__ __forceinline__ void skinny_finish16(const SkinnyParams& p, float (&v
         z = pos ? z : 0.f;
       }
       const int t = t0 + j;
-      if (t < p.T && n_ok) store_16<BF16>(p.out, static_cast<int64_t>(t) * p.N + n, z);
+      if (t < p.T && n_ok) store_out<BF16>(p, static_cast<int64_t>(t) * p.N + n, z);
     }
     if constexpr (EPI == EPI_RELU_AUX_BIAS) {
       const int t = t0 + static_cast<int>(lane);

@@ -102,6 +102,7 @@ struct TileParams {
   int32_t tail_split;       // pair kernel: split the last round's tiles into column halves
   int32_t bias_f32;         // the bias is N fp32 values (else the 16-bit type)
   int32_t b_kmajor;         // W is N x K (K contiguous): B is staged K-major, one box of BN rows per stage
+  int32_t out_f32;          // the output (Y, dZ or dW) is fp32 (else the 16-bit type)
 };
 
 constexpr int kBM = 128;
@@ -314,7 +315,31 @@ __device__ __forceinline__ void epi_rows(const TileParams& p, uint32_t tbase, in
         }
       }
     }
-    {
+    if (p.out_f32) {
+      // fp32 output: the chunk goes out as two 16-column blocks, whose 64-byte
+      // rows are staged and stored exactly like the 16-bit blocks below (a
+      // second block that would start at or past N is not stored)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        if (h == 1 && nc0 + 16 >= p.N) break;  // warp-uniform
+        uint8_t* buf = stg + (scount & 1u) * 2048;
+        if (lane == 0) bulk_wait_group_read<1>();
+        __syncwarp();
+        const uint32_t rbase = smem_u32(buf) + lane * 64;
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          st_shared_v4(rbase + ((q ^ ((lane >> 1) & 3u)) * 16),
+                       make_uint4(__float_as_uint(v[16 * h + 4 * q]), __float_as_uint(v[16 * h + 4 * q + 1]),
+                                  __float_as_uint(v[16 * h + 4 * q + 2]), __float_as_uint(v[16 * h + 4 * q + 3])));
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(tmY, buf, nc0 + 16 * h, wrow0);
+          bulk_commit_group();
+        }
+        ++scount;
+      }
+    } else {
       // Stage this warp's 32 x 32 block (row = lane, 64 bytes) with the
       // 64-byte swizzle -- 16-byte chunk q of row r at chunk q ^ ((r >> 1) & 3)
       // -- so the 16-byte shared stores are conflict-free, then one lane

@@ -115,7 +115,7 @@ GEMM_EPI_API gemm_epi_plan_t gemm_epi_plan(int64_t T, int64_t N, int64_t K, gemm
                               gemm_epi_epilog epilog);
 
 /* Flags of gemm_epi_plan_ex. */
-enum { GEMM_EPI_FLAG_W_NK = 1u };
+enum { GEMM_EPI_FLAG_W_NK = 1u, GEMM_EPI_FLAG_OUT_F32 = 2u };
 
 /*
  * gemm_epi_plan_ex: gemm_epi_plan with flags (gemm_epi_plan passes 0).
@@ -127,6 +127,12 @@ enum { GEMM_EPI_FLAG_W_NK = 1u };
  *   K x N); with this flag neither has to be transposed in memory. Such plans
  *   run on the one-CTA or CTA-pair kernels, never the few-row kernel. Not
  *   valid for WGRAD plans.
+ *   GEMM_EPI_FLAG_OUT_F32: the output -- Y, dZ or dW -- is written as fp32
+ *   (the accumulator, not rounded; 16-byte aligned) while the operands stay
+ *   16-bit ("Fusing bias addition into matrix multiplication with
+ *   nvmath-python", engineering checklist: operand and result types need
+ *   only be compatible). The mask words and dbias are unchanged. The unfused
+ *   entry points return GEMM_EPI_ERR_UNSUPPORTED on such a plan.
  * Returns a plan, or NULL with gemm_epi_last_error() set (unknown flags:
  * GEMM_EPI_ERR_INVALID_ARG).
  */

@@ -326,6 +326,49 @@ def test_ffn_step_chain_bit_exact(T, D, F, dtype):
     assert np.array_equal(oracle.relu_aux_bits(gpu["aux"].numpy().view(np.uint32), F), ref["bits"])
 
 
+@pytest.mark.parametrize("variant", VARIANTS)
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+@pytest.mark.parametrize("T,N,K", [(200, 264, 136), (16, 1032, 520), (600, 1024, 328), (1000, 5000, 72), (5, 40, 24)])
+def test_fp32_output(monkeypatch, T, N, K, dtype, variant):
+    """16-bit operands, fp32 Y / dZ / dW (GEMM_EPI_FLAG_OUT_F32): the accumulator itself."""
+    _force(monkeypatch, variant)
+    D2 = max(8, (K // 2) // 8 * 8)
+    inp = synth.make_shape_inputs(T, N, K, dtype, seed=19 * T + N + K, D2=D2)
+    for ep in FWD_EPILOGS:
+        gpu = run_forward(inp, ep, DT[dtype], out_f32=True)
+        assert gpu["Y"].dtype == torch.float32
+        check_forward(inp, ep, DT[dtype], gpu)
+    fwd = run_forward(inp, "RELU_AUX_BIAS", DT[dtype])
+    outs = run_backward(inp, fwd["aux"], DT[dtype], out_f32=True, repeats=2)
+    for gpu in outs:
+        assert gpu["dZ"].dtype == torch.float32
+        check_backward(inp, fwd["aux"], DT[dtype], gpu)
+    assert torch.equal(outs[0]["dbias"], outs[1]["dbias"])
+    if variant != "skinny":
+        winp = synth.make_shape_inputs(T, N, K, dtype, seed=T + 7 * N + K, D2=N)
+        check_wgrad(winp, DT[dtype], run_wgrad(winp, DT[dtype], out_f32=True))
+
+
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+def test_fp32_output_integer_inputs_exact(dtype):
+    T, N, K, D2 = 300, 1024, 64, 40
+    inp = synth.make_shape_inputs(T, N, K, dtype, seed=78, D2=D2, kind="int")
+    for ep in ("BIAS", "RELU_AUX_BIAS"):
+        check_forward(inp, ep, DT[dtype], run_forward(inp, ep, DT[dtype], out_f32=True), exact=True)
+    fwd = run_forward(inp, "RELU_AUX_BIAS", DT[dtype])
+    check_backward(inp, fwd["aux"], DT[dtype], run_backward(inp, fwd["aux"], DT[dtype], out_f32=True), exact=True)
+
+
+def test_fp32_output_unfused_is_refused():
+    h = binding.gemm_epi_plan(64, 64, 64, binding.F16, binding.RELU_BIAS, flags=binding.FLAG_OUT_F32)
+    try:
+        p = torch.zeros(64 * 64, dtype=torch.float32, device="cuda").data_ptr()
+        rc = binding.lib().gemm_epi_unfused_execute(h, p, p, p, p, p, p, None, None)
+        assert rc == binding.ERR_UNSUPPORTED
+    finally:
+        binding.gemm_epi_free(h)
+
+
 def test_plan_flags_are_checked():
     with pytest.raises(binding.GemmEpiError):
         binding.gemm_epi_plan(64, 64, 64, binding.F16, binding.RELU_BIAS, flags=2)
