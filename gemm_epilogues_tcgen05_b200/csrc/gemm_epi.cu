@@ -135,16 +135,21 @@ static_assert(static_cast<int>(GEMM_EPI_BIAS) == ge::EPI_BIAS && static_cast<int
                   static_cast<int>(GEMM_EPI_NONE) == ge::EPI_STORE,
               "the public epilog values are the kernels' epilog kinds");
 
-template <int BN, int ST, bool BF>
+// BK: the weight is given N x K (GEMM_EPI_FLAG_W_NK); never with WGRAD
+template <int BN, int ST, bool BF, bool BK>
 TileKernelFn pick_epi(int epi) {
   switch (epi) {
-    case ge::EPI_BIAS: return ge::tile_kernel<BN, ST, ge::EPI_BIAS, BF>;
-    case ge::EPI_RELU_BIAS: return ge::tile_kernel<BN, ST, ge::EPI_RELU_BIAS, BF>;
-    case ge::EPI_RELU_AUX_BIAS: return ge::tile_kernel<BN, ST, ge::EPI_RELU_AUX_BIAS, BF>;
-    case ge::EPI_DRELU_BGRAD: return ge::tile_kernel<BN, ST, ge::EPI_DRELU_BGRAD, BF>;
-    case ge::EPI_GELU_BIAS: return ge::tile_kernel<BN, ST, ge::EPI_GELU_BIAS, BF>;
-    case ge::EPI_WGRAD: return ge::tile_kernel<BN, ST, ge::EPI_WGRAD, BF>;
-    default: return ge::tile_kernel<BN, ST, ge::EPI_STORE, BF>;
+    case ge::EPI_BIAS: return ge::tile_kernel<BN, ST, ge::EPI_BIAS, BF, BK>;
+    case ge::EPI_RELU_BIAS: return ge::tile_kernel<BN, ST, ge::EPI_RELU_BIAS, BF, BK>;
+    case ge::EPI_RELU_AUX_BIAS: return ge::tile_kernel<BN, ST, ge::EPI_RELU_AUX_BIAS, BF, BK>;
+    case ge::EPI_DRELU_BGRAD: return ge::tile_kernel<BN, ST, ge::EPI_DRELU_BGRAD, BF, BK>;
+    case ge::EPI_GELU_BIAS: return ge::tile_kernel<BN, ST, ge::EPI_GELU_BIAS, BF, BK>;
+    case ge::EPI_WGRAD:
+      if constexpr (BK)
+        return nullptr;
+      else
+        return ge::tile_kernel<BN, ST, ge::EPI_WGRAD, BF>;
+    default: return ge::tile_kernel<BN, ST, ge::EPI_STORE, BF, BK>;
   }
 }
 
@@ -155,45 +160,58 @@ struct TileCfg {
   bool pair = false;  // CTA-pair kernel, launched in clusters of 2
 };
 
-template <bool BF>
+template <bool BF, bool BK>
 TileKernelFn pick_pair_epi(int epi) {
   switch (epi) {
-    case ge::EPI_BIAS: return ge::tile2_kernel<256, 6, ge::EPI_BIAS, BF>;
-    case ge::EPI_RELU_BIAS: return ge::tile2_kernel<256, 6, ge::EPI_RELU_BIAS, BF>;
-    case ge::EPI_RELU_AUX_BIAS: return ge::tile2_kernel<256, 6, ge::EPI_RELU_AUX_BIAS, BF>;
-    case ge::EPI_DRELU_BGRAD: return ge::tile2_kernel<256, 6, ge::EPI_DRELU_BGRAD, BF>;
-    case ge::EPI_GELU_BIAS: return ge::tile2_kernel<256, 6, ge::EPI_GELU_BIAS, BF>;
-    case ge::EPI_WGRAD: return ge::tile2_kernel<256, 6, ge::EPI_WGRAD, BF>;
-    default: return ge::tile2_kernel<256, 6, ge::EPI_STORE, BF>;
+    case ge::EPI_BIAS: return ge::tile2_kernel<256, 6, ge::EPI_BIAS, BF, BK>;
+    case ge::EPI_RELU_BIAS: return ge::tile2_kernel<256, 6, ge::EPI_RELU_BIAS, BF, BK>;
+    case ge::EPI_RELU_AUX_BIAS: return ge::tile2_kernel<256, 6, ge::EPI_RELU_AUX_BIAS, BF, BK>;
+    case ge::EPI_DRELU_BGRAD: return ge::tile2_kernel<256, 6, ge::EPI_DRELU_BGRAD, BF, BK>;
+    case ge::EPI_GELU_BIAS: return ge::tile2_kernel<256, 6, ge::EPI_GELU_BIAS, BF, BK>;
+    case ge::EPI_WGRAD:
+      if constexpr (BK)
+        return nullptr;
+      else
+        return ge::tile2_kernel<256, 6, ge::EPI_WGRAD, BF>;
+    default: return ge::tile2_kernel<256, 6, ge::EPI_STORE, BF, BK>;
   }
 }
 
-TileCfg pair_cfg(int epi, bool bf16) {
+template <int BN, int ST>
+TileKernelFn pick_tile(int epi, bool bf16, bool bk) {
+  if (bk) return bf16 ? pick_epi<BN, ST, true, true>(epi) : pick_epi<BN, ST, false, true>(epi);
+  return bf16 ? pick_epi<BN, ST, true, false>(epi) : pick_epi<BN, ST, false, false>(epi);
+}
+
+TileCfg pair_cfg(int epi, bool bf16, bool bk) {
   TileCfg c;
   c.BN = 256;
   c.stages = 6;
   c.smem = ge::Tile2Smem<256, 6>::BYTES;
-  c.fn = bf16 ? pick_pair_epi<true>(epi) : pick_pair_epi<false>(epi);
+  if (bk)
+    c.fn = bf16 ? pick_pair_epi<true, true>(epi) : pick_pair_epi<false, true>(epi);
+  else
+    c.fn = bf16 ? pick_pair_epi<true, false>(epi) : pick_pair_epi<false, false>(epi);
   c.pair = true;
   return c;
 }
 
-TileCfg tile_cfg(int BN, int epi, bool bf16) {
+TileCfg tile_cfg(int BN, int epi, bool bf16, bool bk) {
   TileCfg c;
   c.BN = BN;
   if (BN == 256) {
     c.stages = 4;
     c.smem = ge::TileSmem<256, 4>::BYTES;
-    c.fn = bf16 ? pick_epi<256, 4, true>(epi) : pick_epi<256, 4, false>(epi);
+    c.fn = pick_tile<256, 4>(epi, bf16, bk);
   } else if (BN == 128) {
     c.stages = 6;
     c.smem = ge::TileSmem<128, 6>::BYTES;
-    c.fn = bf16 ? pick_epi<128, 6, true>(epi) : pick_epi<128, 6, false>(epi);
+    c.fn = pick_tile<128, 6>(epi, bf16, bk);
   } else {
     c.BN = 64;
     c.stages = 8;
     c.smem = ge::TileSmem<64, 8>::BYTES;
-    c.fn = bf16 ? pick_epi<64, 8, true>(epi) : pick_epi<64, 8, false>(epi);
+    c.fn = pick_tile<64, 8>(epi, bf16, bk);
   }
   return c;
 }
@@ -315,6 +333,7 @@ struct gemm_epi_plan_s {
   int bias_f32 = 0;      // gemm_epi_set_bias_f32: the forward bias is fp32
   int w_nk = 0;          // GEMM_EPI_FLAG_W_NK: W / W2 given N x K (K contiguous)
   int out_f32 = 0;       // GEMM_EPI_FLAG_OUT_F32: Y / dZ / dW written as fp32
+  int cache_hints = 0;   // few-row kernel: L2 eviction policies on the operand loads (GEMM_EPI_CACHE_HINTS)
   // tensor-map cache
   const void* a_ptr = nullptr;
   const void* b_ptr = nullptr;
@@ -397,7 +416,6 @@ ge::TileParams base_params(const gemm_epi_plan_s* p) {
   k.inject_stall = p->inject_stall;
   k.tail_split = p->tail_split;
   k.bias_f32 = p->bias_f32;
-  k.b_kmajor = p->w_nk;
   k.out_f32 = p->out_f32;
   return k;
 }
@@ -497,6 +515,7 @@ ge::SkinnyParams skinny_params(const gemm_epi_plan_s* p) {
   k.timeout_ns = p->timeout_ns;
   k.bias_f32 = p->bias_f32;
   k.out_f32 = p->out_f32;
+  k.cache_hints = p->cache_hints;
   return k;
 }
 
@@ -597,8 +616,8 @@ gemm_epi_plan_t gemm_epi_plan_ex(int64_t T, int64_t N, int64_t K, gemm_epi_dtype
   const bool bf16 = dtype == GEMM_EPI_BF16;
   const bool pair = use_pair(T, N, K, sms);
   const int bn = pair ? 256 : choose_bn(T, N, sms);
-  p->cfg = pair ? pair_cfg((int)epilog, bf16) : tile_cfg(bn, (int)epilog, bf16);
-  p->cfg_store = pair ? pair_cfg(ge::EPI_STORE, bf16) : tile_cfg(bn, ge::EPI_STORE, bf16);
+  p->cfg = pair ? pair_cfg((int)epilog, bf16, w_nk) : tile_cfg(bn, (int)epilog, bf16, w_nk);
+  p->cfg_store = pair ? pair_cfg(ge::EPI_STORE, bf16, w_nk) : tile_cfg(bn, ge::EPI_STORE, bf16, w_nk);
   p->kernel = pair ? 2 : 0;
   p->m_tiles = ceil_div(T, ge::kBM);
   p->n_tiles = ceil_div(N, bn);
@@ -623,6 +642,7 @@ gemm_epi_plan_t gemm_epi_plan_ex(int64_t T, int64_t N, int64_t K, gemm_epi_dtype
   if (const char* f = getenv("GEMM_EPI_INJECT_STALL")) p->inject_stall = atoi(f) != 0;
   if (const char* f = getenv("GEMM_EPI_TAIL_SPLIT")) p->tail_split = atoi(f) != 0;
 
+
   auto cleanup = [&](int rc) {
     if (p->col_tickets) cudaFree(p->col_tickets);
     if (p->sk_partials) cudaFree(p->sk_partials);
@@ -638,8 +658,14 @@ gemm_epi_plan_t gemm_epi_plan_ex(int64_t T, int64_t N, int64_t K, gemm_epi_dtype
     e = cudaFuncSetAttribute(c->fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)c->smem);
     if (e != cudaSuccess) return cleanup(cuda_fail(e, "cudaFuncSetAttribute(max dynamic shared memory)"));
   }
+  // L2 eviction hints on the few-row kernel's operand loads (W evict_first, X
+  // evict_last), where W streams through L2 once (measured at N = 11008, K =
+  // 4096: T = 1 25.1 / 24.5 us against 27.3 / 26.8, T = 64 32.6 / 33.4 against
+  // 33.2 / 34.3). The tile kernels load without hints: there they did not help
+  // the FFN and square shapes and slowed the large one (17.6 against 16.8 ms).
   if (!pair && epilog != GEMM_EPI_WGRAD && !w_nk && use_skinny(T)) {
     p->kernel = 1;
+    p->cache_hints = 1;
     p->sk = skinny_cfg(T, (int)epilog, bf16);
     const int n_tiles = ceil_div(N, 128);
     p->sk_kbt = ceil_div(K, (int64_t)ge::kBK * p->sk.KPS);
@@ -705,6 +731,7 @@ gemm_epi_plan_t gemm_epi_plan_ex(int64_t T, int64_t N, int64_t K, gemm_epi_dtype
     e = cudaMalloc((void**)&p->partials, p->partial_bytes);
     if (e != cudaSuccess) return cleanup(cuda_fail(e, "cudaMalloc(workspace)"));
   }
+  if (const char* f = getenv("GEMM_EPI_CACHE_HINTS")) p->cache_hints = atoi(f) != 0;  // A/B override
   {
     std::lock_guard<std::mutex> g(g_mu);
     live_plans().insert(p);
@@ -1030,7 +1057,7 @@ int noalloc_setup(int dev, NoAllocDevice*& out) {
     d.scratch = static_cast<unsigned char*>(p);
     for (int bn : {64, 128, 256}) {
       for (bool bf16 : {false, true}) {
-        TileCfg c = tile_cfg(bn, ge::EPI_DRELU_BGRAD, bf16);
+        TileCfg c = tile_cfg(bn, ge::EPI_DRELU_BGRAD, bf16, false);
         d.err = cudaFuncSetAttribute(c.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)c.smem);
         if (d.err != cudaSuccess) {
           d.what = "cudaFuncSetAttribute(max dynamic shared memory)";
@@ -1085,7 +1112,7 @@ extern "C" int drelu_bgrad_execute_noalloc(int64_t T, int64_t N, int64_t K, gemm
   float* partials = reinterpret_cast<float*>(nd->scratch + kNoAllocStatusBytes);
 
   const int bn = choose_bn(T, N, sms);
-  const TileCfg cfg = tile_cfg(bn, ge::EPI_DRELU_BGRAD, dtype == GEMM_EPI_BF16);
+  const TileCfg cfg = tile_cfg(bn, ge::EPI_DRELU_BGRAD, dtype == GEMM_EPI_BF16, false);
   CUtensorMap tmA, tmB, tmY;
   rc = encode_2d(&tmA, dY2, (uint64_t)K, (uint64_t)T, ge::kBK, ge::kBM, "dY2");
   if (rc) return rc;

@@ -41,6 +41,7 @@ struct SkinnyParams {
   uint64_t timeout_ns;
   int32_t bias_f32;                // the bias is N fp32 values (else the 16-bit type)
   int32_t out_f32;                 // the output is fp32 (else the 16-bit type)
+  int32_t cache_hints;             // W streamed once: evict_first; X read by every CTA: evict_last
 };
 
 // A stage holds KPS consecutive 64-deep k-blocks: W as one box of 64 features
@@ -310,6 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       };
       int64_t gk = lo;  // global k-block index of the next load
+      const uint64_t pol_w = l2_policy_evict_first(), pol_x = l2_policy_evict_last();
       while (ok && skinny_segment(p, lo, hi, g, s)) {
         const int n0 = s.tile * 128;
         for (int kb = s.kb0; kb < s.kb1; ++kb, ++it, ++gk) {
@@ -321,11 +323,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           mbar_arrive_expect_tx(&full[st], L::STAGE);
-          tma_load_2d(sA + st * L::A_BYTES, &tmW, &full[st], n0, kb * L::BK);
-          tma_load_2d(sA + st * L::A_BYTES + L::A_CHUNK, &tmW, &full[st], n0 + 64, kb * L::BK);
+          if (p.cache_hints) {
+            tma_load_2d_hint(sA + st * L::A_BYTES, &tmW, &full[st], n0, kb * L::BK, pol_w);
+            tma_load_2d_hint(sA + st * L::A_BYTES + L::A_CHUNK, &tmW, &full[st], n0 + 64, kb * L::BK, pol_w);
 #pragma unroll
-          for (int j = 0; j < KPS; ++j)
-            tma_load_2d(sB + st * L::B_BYTES + j * L::B_SUB, &tmX, &full[st], kb * L::BK + j * kBK, 0);
+            for (int j = 0; j < KPS; ++j)
+              tma_load_2d_hint(sB + st * L::B_BYTES + j * L::B_SUB, &tmX, &full[st], kb * L::BK + j * kBK, 0, pol_x);
+          } else {
+            tma_load_2d(sA + st * L::A_BYTES, &tmW, &full[st], n0, kb * L::BK);
+            tma_load_2d(sA + st * L::A_BYTES + L::A_CHUNK, &tmW, &full[st], n0 + 64, kb * L::BK);
+#pragma unroll
+            for (int j = 0; j < KPS; ++j)
+              tma_load_2d(sB + st * L::B_BYTES + j * L::B_SUB, &tmX, &full[st], kb * L::BK + j * kBK, 0);
+          }
         }
       }
       const uint32_t inflight = it < STAGES ? it : STAGES;

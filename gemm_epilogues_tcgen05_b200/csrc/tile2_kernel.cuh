@@ -77,7 +77,7 @@ struct PairSchedule {
   }
 };
 
-template <int BN, int STAGES, int EPI, bool BF16>
+template <int BN, int STAGES, int EPI, bool BF16, bool BK = false>
 __global__ void __launch_bounds__(kThreads, 1)
     tile2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmAux,
@@ -144,8 +144,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int m2_tiles = (p.m_tiles + 1) / 2;  // 256-row tiles
-  // half units need a 64-row box of a K-major W: with b_kmajor every unit is a whole tile
-  const PairSchedule sched(m2_tiles * p.n_tiles, npairs, p.tail_split != 0 && p.b_kmajor == 0);
+  // half units would need a 64-row box of a K-major W: with BK every unit is a whole tile
+  const PairSchedule sched(m2_tiles * p.n_tiles, npairs, p.tail_split != 0 && !BK);
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -174,7 +174,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             tma_load_2d_pair(sA + s * L::A_BYTES, &tmA, fbar, kb * kBK, m0);
           }
-          if (p.b_kmajor) {  // this CTA's 128 rows of the N x K weight in one box
+          if constexpr (BK) {  // this CTA's 128 rows of the N x K weight in one box
             tma_load_2d_pair(sB + s * L::B_BYTES, &tmB, fbar, kb * kBK, nh0);
           } else {
             for (int j = 0; j < nchunks; ++j)
@@ -196,7 +196,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         for (int u = pair; ok && u < sched.num_units; u += npairs, ++tcount) {
           const PairUnit w = sched.unit(u, m2_tiles, p.n_tiles, p.group_m);
-          const uint32_t idesc = p.b_kmajor ? IDESC_BK : w.half < 0 ? IDESC : IDESC_HALF;
+          const uint32_t idesc = BK ? IDESC_BK : w.half < 0 ? IDESC : IDESC_HALF;
           const uint32_t buf = tcount & 1u;
           const uint32_t tph = (tcount >> 1) & 1u;
           if (!wait_bounded(&tempty[buf], tph ^ 1u, p, abort_flag, 3)) break;
@@ -215,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int kk = 0; kk < kBK / 16; ++kk) {
               const uint64_t adesc = a_desc<A_MN>(a0, kk);
-              const uint64_t bdesc = b_desc(b0, kk, p.b_kmajor != 0, L::B_CHUNK);
+              const uint64_t bdesc = b_desc(b0, kk, BK, L::B_CHUNK);
               umma_f16_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
             }
             umma_commit_pair(&empty[s], BOTH);

@@ -101,7 +101,6 @@ struct TileParams {
   float* dbias;             // DRELU_BGRAD: written by the tile that takes a column block's last ticket
   int32_t tail_split;       // pair kernel: split the last round's tiles into column halves
   int32_t bias_f32;         // the bias is N fp32 values (else the 16-bit type)
-  int32_t b_kmajor;         // W is N x K (K contiguous): B is staged K-major, one box of BN rows per stage
   int32_t out_f32;          // the output (Y, dZ or dW) is fp32 (else the 16-bit type)
 };
 
@@ -432,7 +431,10 @@ __device__ __forceinline__ void epi_finish_dbias(const TileParams& p, int nb, in
   named_bar_sync(1, 128);  // the flag word is reused by the next tile
 }
 
-template <int BN, int STAGES, int EPI, bool BF16>
+// BK: the weight is N x K (K contiguous) and B is staged K-major; a template
+// parameter, not a runtime flag -- a branch on it in the producer and MMA
+// loops cost 3-4 % on the FFN shape (their issue path is latency-critical)
+template <int BN, int STAGES, int EPI, bool BF16, bool BK = false>
 __global__ void __launch_bounds__(kThreads, 1)
     tile_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmAux,
@@ -516,7 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             tma_load_2d(sA + s * L::A_BYTES, &tmA, &full[s], kb * kBK, m0);
           }
-          if (p.b_kmajor) {
+          if constexpr (BK) {
             tma_load_2d(sB + s * L::B_BYTES, &tmB, &full[s], kb * kBK, n0);
           } else {
 #pragma unroll
@@ -536,8 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t it = 0, tcount = 0;
       bool ok = true;
-      const bool bk = p.b_kmajor != 0;
-      const uint32_t idesc = bk ? IDESC_BK : IDESC;
+      constexpr uint32_t idesc = BK ? IDESC_BK : IDESC;
       for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++tcount) {
         const uint32_t buf = tcount & 1u;
         const uint32_t tph = (tcount >> 1) & 1u;
@@ -557,7 +558,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
             const uint64_t adesc = a_desc<A_MN>(a0, kk);
-            const uint64_t bdesc = b_desc(b0, kk, bk, L::B_CHUNK);
+            const uint64_t bdesc = b_desc(b0, kk, BK, L::B_CHUNK);
             umma_f16(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
           umma_commit(&empty[s]);

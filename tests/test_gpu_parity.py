@@ -371,7 +371,7 @@ def test_fp32_output_unfused_is_refused():
 
 def test_plan_flags_are_checked():
     with pytest.raises(binding.GemmEpiError):
-        binding.gemm_epi_plan(64, 64, 64, binding.F16, binding.RELU_BIAS, flags=2)
+        binding.gemm_epi_plan(64, 64, 64, binding.F16, binding.RELU_BIAS, flags=4)  # no such flag
     with pytest.raises(binding.GemmEpiError):
         binding.gemm_epi_plan(64, 64, 64, binding.F16, binding.WGRAD, flags=binding.FLAG_W_NK)
 
