@@ -48,6 +48,11 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// Fault injection for the host tests: GEMM_EPI_INJECT_ENCODE_FAILURE makes every
+// tensor-map encode fail, so an execute call must return GEMM_EPI_ERR_CUDA
+// before it launches anything.
+bool inject_encode_failure() { return getenv("GEMM_EPI_INJECT_ENCODE_FAILURE") != nullptr; }
+
 EncodeTiledFn encode_fn() {
   static EncodeTiledFn fn = nullptr;
   static std::once_flag once;
@@ -69,6 +74,7 @@ int encode_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer
               CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(GEMM_EPI_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  if (inject_encode_failure()) return fail(GEMM_EPI_ERR_CUDA, "injected tensor map encode failure");
   const cuuint64_t dims[2] = {inner, outer};
   const cuuint64_t strides[1] = {inner * 2};
   const cuuint32_t box[2] = {box_inner, box_outer};
@@ -92,6 +98,7 @@ int encode_out(CUtensorMap* map, const void* out, int64_t T, int64_t N) {
 int encode_out_f32(CUtensorMap* map, const void* out, int64_t T, int64_t N) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(GEMM_EPI_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  if (inject_encode_failure()) return fail(GEMM_EPI_ERR_CUDA, "injected tensor map encode failure");
   const cuuint64_t dims[2] = {(uint64_t)N, (uint64_t)T};
   const cuuint64_t strides[1] = {(uint64_t)N * 4};
   const cuuint32_t box[2] = {16, 32};
@@ -115,6 +122,7 @@ bool aux_tma_ok(const void* aux, int64_t N, int bn) {
 int encode_aux(CUtensorMap* map, const void* aux, int64_t T, int64_t N, int bn) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(GEMM_EPI_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  if (inject_encode_failure()) return fail(GEMM_EPI_ERR_CUDA, "injected tensor map encode failure");
   const uint64_t words = (uint64_t)((N + 31) / 32);
   const cuuint64_t dims[2] = {words, (uint64_t)T};
   const cuuint64_t strides[1] = {words * 4};

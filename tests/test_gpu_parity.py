@@ -428,6 +428,26 @@ def test_wgrad_plan_rejects_other_calls():
         binding.gemm_epi_free(hf)
 
 
+def test_injected_encode_failure_returns_error_without_launch(monkeypatch):
+    """A failing tensor-map encode (forced on the host) is reported by execute
+    as GEMM_EPI_ERR_CUDA; the output stays untouched (nothing was launched)."""
+    T, N, K = 128, 128, 64
+    inp = synth.make_shape_inputs(T, N, K, "bf16", seed=2)
+    g = {k: v.cuda() for k, v in inp.items()}
+    with binding.Plan(T, N, K, torch.bfloat16, "RELU_BIAS") as plan:
+        Y = torch.full((T, N), 7.0, dtype=torch.bfloat16, device="cuda")
+        monkeypatch.setenv("GEMM_EPI_INJECT_ENCODE_FAILURE", "1")
+        with pytest.raises(binding.GemmEpiError) as e:
+            plan.gemm_epi_execute(g["X"], g["W"], g["bias"], Y)
+        assert e.value.code == binding.ERR_CUDA and "injected" in str(e.value)
+        torch.cuda.synchronize()
+        assert torch.all(Y == 7.0)
+        monkeypatch.delenv("GEMM_EPI_INJECT_ENCODE_FAILURE")
+        plan.gemm_epi_execute(g["X"], g["W"], g["bias"], Y)  # the plan still works afterwards
+        torch.cuda.synchronize()
+        assert plan.status() == 0 and not torch.all(Y == 7.0)
+
+
 def test_unknown_epilog_values_rejected():
     for bad in (-1, 7, 99):
         with pytest.raises(binding.GemmEpiError):
