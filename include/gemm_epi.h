@@ -140,14 +140,20 @@ GEMM_EPI_API gemm_epi_plan_t gemm_epi_plan_ex(int64_t T, int64_t N, int64_t K, g
                                               gemm_epi_epilog epilog, uint32_t flags);
 
 /*
- * gemm_epi_execute: the forward epilogs (BIAS, RELU_BIAS, RELU_AUX_BIAS).
- *   X, W, Y: device pointers, 16-byte aligned. bias: device pointer, 2-byte
- *   aligned, never NULL. aux: device pointer, 4-byte aligned, required for
- *   RELU_AUX_BIAS and ignored (may be NULL) otherwise.
+ * gemm_epi_execute: the forward epilogs (BIAS, RELU_BIAS, RELU_AUX_BIAS,
+ * GELU_BIAS) and the plain product (NONE).
+ *   X, W, Y: device pointers, 16-byte aligned (W is K x N, or N x K with
+ *   GEMM_EPI_FLAG_W_NK; Y is fp32 with GEMM_EPI_FLAG_OUT_F32). bias: device
+ *   pointer, 2-byte aligned (4-byte for an fp32 bias, gemm_epi_set_bias_f32),
+ *   never NULL except for NONE, where it is ignored. aux: device pointer,
+ *   4-byte aligned, required for RELU_AUX_BIAS and ignored (may be NULL)
+ *   otherwise.
  * Returns GEMM_EPI_OK once the work is enqueued on `stream`;
- * GEMM_EPI_ERR_EPILOG_MISMATCH on a DRELU_BGRAD plan or a missing aux;
- * GEMM_EPI_ERR_TIMEOUT if an earlier call on this plan reported a watchdog
- * expiry (the report is cleared by reading it).
+ * GEMM_EPI_ERR_EPILOG_MISMATCH on a DRELU_BGRAD or WGRAD plan or a missing
+ * aux; GEMM_EPI_ERR_MISALIGNED for a misaligned pointer; GEMM_EPI_ERR_CUDA if
+ * a tensor map cannot be encoded or the launch fails (nothing is launched
+ * then); GEMM_EPI_ERR_TIMEOUT if an earlier call on this plan reported a
+ * watchdog expiry (the report is cleared by reading it).
  */
 GEMM_EPI_API int gemm_epi_execute(gemm_epi_plan_t plan, const void* X, const void* W, const void* bias, void* Y,
                      uint32_t* aux, cudaStream_t stream);
@@ -220,11 +226,15 @@ GEMM_EPI_API int gemm_epi_status(gemm_epi_plan_t plan);
  * MatMul writes an intermediate, BiasAdd reads it and writes another, ReLU
  * reads that and writes the output).
  *   gemm_epi_unfused_execute: GEMM -> T1 (T x N, dtype), T1 + bias -> T2,
- *   relu(T2) -> Y (and, for RELU_AUX_BIAS, the mask from T2 > 0 -> aux).
- *   For BIAS the ReLU kernel is skipped and T2 is the output: pass Y as T2.
+ *   relu(T2) -> Y (and, for RELU_AUX_BIAS, the mask from T2 > 0 -> aux), or
+ *   gelu(T2) -> Y for GELU_BIAS. For BIAS the activation kernel is skipped
+ *   and T2 is the output: pass Y as T2.
  *   drelu_bgrad_unfused_execute: GEMM -> G (dtype), mask apply -> dZ,
  *   column sum of dZ -> dbias (fixed order).
  * T1, T2, G: caller-owned device scratch of T x N dtype, 16-byte aligned.
+ * Plans with epilog NONE or WGRAD return GEMM_EPI_ERR_EPILOG_MISMATCH, plans
+ * with GEMM_EPI_FLAG_OUT_F32 GEMM_EPI_ERR_UNSUPPORTED (the unfused path
+ * keeps 16-bit intermediates).
  */
 GEMM_EPI_API int gemm_epi_unfused_execute(gemm_epi_plan_t plan, const void* X, const void* W, const void* bias,
                              void* T1, void* T2, void* Y, uint32_t* aux, cudaStream_t stream);
