@@ -176,6 +176,50 @@ class ClockSampler:
                 "power_w_max": max((num(p[4]) or 0.0) for p in inside)}
 
 
+def roofline(w, fwd_epi, res, peaks, peak_src):
+    """The JSON line's roofline object for the dominant call (the slower of
+    the two): HBM-bound for the few-row workloads, tensor-bound otherwise,
+    against the measured peak that fits the run's regime."""
+    alg = res["alg"]
+    # dominant kernel: the one of the two calls that takes longer
+    part = "fwd" if res["fwd_ms"] >= res["bwd_ms"] else "bwd"
+    part_ms = res[f"{part}_ms"]
+    skinny = w.name.startswith("skinny")
+    if skinny:
+        achieved = alg[part]["bytes"] / (part_ms / 1e3) / 1e9
+        peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak}
+    else:
+        achieved = alg[part]["flops"] / (part_ms / 1e3) / 1e12
+        # fp16 dense peak = bf16 dense peak. The burst figure is for a kernel
+        # that runs before the 1 kW power cap settles the clocks; a launch of
+        # a millisecond or more, or a timed region during which the sampled
+        # clocks report the power cap active (back-to-back steps), is a
+        # sustained load and is measured against the sustained figure.
+        burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+        long_launch = part_ms >= 1.0
+        capped = "sw_power_cap" in ((res.get("clocks") or {}).get("reasons") or [])
+        peak = sustained if (long_launch or capped) else burst
+        kind = ("sustained (launch >= 1 ms)" if long_launch else
+                "sustained (power cap active in the timed region)" if capped else "burst (launch < 1 ms)")
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "frac_of_burst": achieved / burst, "peak_kind": kind}
+    kname = {0: "tile_kernel", 1: "skinny_kernel", 2: "tile2_kernel (CTA pair)"}[res["kernel"]]
+    roof["kernel"] = f"{part}: {kname} " + (fwd_epi if part == "fwd" else "DRELU_BGRAD" +
+                                              (" + dbias finish" if res["kernel"] != 1 else ""))
+    if fwd_epi == "FFN_STEP":
+        roof["kernel"] = (f"{part}: " + ("layer 1 RELU_AUX_BIAS + layer 2 BIAS" if part == "fwd" else
+                                         "DRELU_BGRAD, WGRAD (+db2), WGRAD, NONE") + f" ({kname} kernels)")
+    roof["peak_source"] = "measured (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
+    roof["traffic"] = measured_traffic(w, part, fwd_epi)
+    # roofline time of the whole step: slower of FLOPs at the tensor peak and bytes at HBM
+    t_roof = sum(max(v["flops"] / (float(peaks.get("bf16_tflops", 1590.0)) * 1e12),
+                     v["bytes"] / (float(peaks.get("hbm_gbs", 6650.0)) * 1e9)) for v in alg.values())
+    roof["step_roofline_frac"] = t_roof * 1e3 / res["step_ms"]
+    return roof
+
+
 # ------------------------------------------------------- across the ranks
 def max_over_ranks(values, device, world: int) -> list[float]:
     """Each entry's maximum over all ranks (the slowest rank's time): an
@@ -593,44 +637,8 @@ def main():
     if rank != 0:
         return
 
-    alg = res["alg"]
     value = whole_job_tflops(res["flops_step"], world, res["step_ms"])
-    # dominant kernel: the one of the two calls that takes longer
-    part = "fwd" if res["fwd_ms"] >= res["bwd_ms"] else "bwd"
-    part_ms = res[f"{part}_ms"]
-    skinny = w.name.startswith("skinny")
-    if skinny:
-        achieved = alg[part]["bytes"] / (part_ms / 1e3) / 1e9
-        peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak}
-    else:
-        achieved = alg[part]["flops"] / (part_ms / 1e3) / 1e12
-        # fp16 dense peak = bf16 dense peak. The burst figure is for a kernel
-        # that runs before the 1 kW power cap settles the clocks; a launch of
-        # a millisecond or more, or a timed region during which the sampled
-        # clocks report the power cap active (back-to-back steps), is a
-        # sustained load and is measured against the sustained figure.
-        burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-        sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
-        long_launch = part_ms >= 1.0
-        capped = "sw_power_cap" in ((res.get("clocks") or {}).get("reasons") or [])
-        peak = sustained if (long_launch or capped) else burst
-        kind = ("sustained (launch >= 1 ms)" if long_launch else
-                "sustained (power cap active in the timed region)" if capped else "burst (launch < 1 ms)")
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                "frac_of_burst": achieved / burst, "peak_kind": kind}
-    kname = {0: "tile_kernel", 1: "skinny_kernel", 2: "tile2_kernel (CTA pair)"}[res["kernel"]]
-    roof["kernel"] = f"{part}: {kname} " + (fwd_epi if part == "fwd" else "DRELU_BGRAD" +
-                                              (" + dbias finish" if res["kernel"] != 1 else ""))
-    if fwd_epi == "FFN_STEP":
-        roof["kernel"] = (f"{part}: " + ("layer 1 RELU_AUX_BIAS + layer 2 BIAS" if part == "fwd" else
-                                         "DRELU_BGRAD, WGRAD (+db2), WGRAD, NONE") + f" ({kname} kernels)")
-    roof["peak_source"] = "measured (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
-    roof["traffic"] = measured_traffic(w, part, fwd_epi)
-    # roofline time of the whole step: slower of FLOPs at the tensor peak and bytes at HBM
-    t_roof = sum(max(v["flops"] / (float(peaks.get("bf16_tflops", 1590.0)) * 1e12),
-                     v["bytes"] / (float(peaks.get("hbm_gbs", 6650.0)) * 1e9)) for v in alg.values())
-    roof["step_roofline_frac"] = t_roof * 1e3 / res["step_ms"]
+    roof = roofline(w, fwd_epi, res, peaks, peak_src)
 
     line = {"metric": metric_name(w), "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": res["step_ms"], "higher_is_better": True, "scaling": "weak",

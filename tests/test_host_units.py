@@ -109,3 +109,42 @@ def test_sample_indices_distinct_and_seeded():
     a = synth.sample_indices(4096, 256, seed=7)
     assert len(set(a)) == 256 and all(0 <= x < 4096 for x in a)
     assert a == synth.sample_indices(4096, 256, seed=7)
+
+
+# ------------------------------------------------------------ roofline object
+PEAKS = {"hbm_gbs": 6542.1, "bf16_tflops": 1671.6, "bf16_tflops_sustained": 1407.4}
+
+
+def _res(w, fwd_epi, fwd_ms, bwd_ms, reasons=(), kernel=2):
+    alg = bench.algorithmic(w, fwd_epi, bwd_ms > 0)
+    return {"alg": alg, "fwd_ms": fwd_ms, "bwd_ms": bwd_ms, "step_ms": fwd_ms + bwd_ms, "kernel": kernel,
+            "clocks": {"reasons": list(reasons)}}
+
+
+def test_roofline_takes_the_slower_call_and_the_burst_peak():
+    w = W["ffn"]
+    r = bench.roofline(w, "RELU_AUX_BIAS", _res(w, "RELU_AUX_BIAS", 0.270, 0.280), PEAKS, "measured")
+    assert r["bound"] == "tensor" and r["kernel"].startswith("bwd: tile2_kernel")
+    assert r["achieved"] == pytest.approx(369.4e9 / 0.280e-3 / 1e12, rel=1e-3)
+    assert r["peak"] == 1671.6 and r["peak_kind"].startswith("burst")
+    assert r["frac"] == pytest.approx(r["achieved"] / 1671.6)
+    # the whole step against its roofline time (FLOPs at the tensor peak for both calls)
+    assert r["step_roofline_frac"] == pytest.approx(2 * 369.4e9 / 1671.6e12 / 0.550e-3, rel=2e-3)
+
+
+def test_roofline_uses_the_sustained_peak_under_the_power_cap_or_for_long_launches():
+    w = W["ffn"]
+    capped = bench.roofline(w, "RELU_AUX_BIAS", _res(w, "RELU_AUX_BIAS", 0.27, 0.28, ["sw_power_cap"]), PEAKS, "measured")
+    assert capped["peak"] == 1407.4 and "power cap" in capped["peak_kind"]
+    assert capped["frac_of_burst"] == pytest.approx(capped["achieved"] / 1671.6)
+    big = W["large"]
+    long_ = bench.roofline(big, "RELU_AUX_BIAS", _res(big, "RELU_AUX_BIAS", 15.0, 0.0, kernel=0), PEAKS, "measured")
+    assert long_["peak"] == 1407.4 and "1 ms" in long_["peak_kind"] and long_["kernel"].startswith("fwd: tile_kernel")
+
+
+def test_roofline_is_hbm_bound_for_the_few_row_workloads():
+    w = W["skinny-1"]
+    r = bench.roofline(w, "RELU_BIAS", _res(w, "RELU_BIAS", 0.0246, 0.0227, kernel=1), PEAKS, "measured")
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s" and r["peak"] == 6542.1
+    assert r["achieved"] == pytest.approx(bench.algorithmic(w, "RELU_BIAS", True)["fwd"]["bytes"] / 0.0246e-3 / 1e9)
+    assert r["frac"] == pytest.approx(r["achieved"] / 6542.1)
