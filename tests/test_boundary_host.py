@@ -56,6 +56,13 @@ def test_plan_rejects_bad_enums(L):
     assert "epilog" in binding.gemm_epi_last_error()
 
 
+def test_plan_flags_are_checked_before_the_device(L):
+    assert not L.gemm_epi_plan_ex(64, 64, 64, 0, 0, 8)  # no such flag
+    assert "flags" in binding.gemm_epi_last_error()
+    assert not L.gemm_epi_plan_ex(64, 64, 64, 0, binding.WGRAD, binding.FLAG_W_NK)
+    assert "W_NK" in binding.gemm_epi_last_error()
+
+
 def test_unknown_plan_handles_are_rejected_not_dereferenced(L):
     bogus = ctypes.c_void_p(0x12345678)
     rc = L.gemm_epi_execute(bogus, 16, 16, 16, 16, 16, None)
