@@ -22,6 +22,13 @@ their order and notation:
   GELU(z) = z * Phi(z), Phi the standard normal CDF, i.e.
   z/2 * (1 + erf(z / sqrt 2)), with scipy's double-precision erf as the
   library primitive.
+* GELU_AUX_BIAS -- GELU_BIAS that also returns an auxiliary output for the
+  backward pass, as RELU_AUX_BIAS does for ReLU. The pages describe
+  RELU_AUX_BIAS's auxiliary output (the mask, for the backward epilog) but
+  not GELU's; the derivative of GELU depends on the pre-activation z itself,
+  not only on its sign, so the auxiliary output is read as that
+  pre-activation Z = X.W + bias (``pre``), which the library stores in its
+  16-bit type.
 * ``wgrad`` -- the weight gradient dW = X^T . dZ of the linear layer, the
   part of the backward pass that "nvmath-python fused epilogs for linear
   layers" (FAQ) says DRELU_BGRAD does not cover. The plain definition:
@@ -62,6 +69,7 @@ EPILOG_BIAS = "BIAS"
 EPILOG_RELU_BIAS = "RELU_BIAS"
 EPILOG_RELU_AUX_BIAS = "RELU_AUX_BIAS"
 EPILOG_GELU_BIAS = "GELU_BIAS"
+EPILOG_GELU_AUX_BIAS = "GELU_AUX_BIAS"
 EPILOG_NONE = "NONE"
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -187,11 +195,14 @@ def linear_fwd(X, W, bias, dtype: int, epilog: str, rows=None, cols=None, thread
     Returns a dict with
       Z     the pre-activation X.W + bias (fp64, exact up to binary64 rounding)
       S     the error scale sum_k |x w| + |b|
-      Y     Z for BIAS; max(Z, 0) for RELU_BIAS / RELU_AUX_BIAS; gelu(Z) for GELU_BIAS
+      Y     Z for BIAS; max(Z, 0) for RELU_BIAS / RELU_AUX_BIAS; gelu(Z) for GELU_BIAS and
+            GELU_AUX_BIAS
       bits  Z > 0 (strict: a zero pre-activation gives bit 0), for RELU_AUX_BIAS
       aux   the packed words (only when every column was computed)
+      pre   GELU_AUX_BIAS's auxiliary output: the pre-activation Z
     """
-    if epilog not in (EPILOG_BIAS, EPILOG_RELU_BIAS, EPILOG_RELU_AUX_BIAS, EPILOG_GELU_BIAS, EPILOG_NONE):
+    if epilog not in (EPILOG_BIAS, EPILOG_RELU_BIAS, EPILOG_RELU_AUX_BIAS, EPILOG_GELU_BIAS, EPILOG_GELU_AUX_BIAS,
+                      EPILOG_NONE):
         raise ValueError(f"unknown forward epilog {epilog}")
     if epilog == EPILOG_NONE:
         bias = None  # the plain product
@@ -211,8 +222,10 @@ def linear_fwd(X, W, bias, dtype: int, epilog: str, rows=None, cols=None, thread
     out = {"Z": Z, "S": S}
     if epilog in (EPILOG_BIAS, EPILOG_NONE):
         out["Y"] = Z.copy()
-    elif epilog == EPILOG_GELU_BIAS:
+    elif epilog in (EPILOG_GELU_BIAS, EPILOG_GELU_AUX_BIAS):
         out["Y"] = gelu(Z)
+        if epilog == EPILOG_GELU_AUX_BIAS:
+            out["pre"] = Z.copy()
     else:
         out["Y"] = np.maximum(Z, 0.0)
     if epilog == EPILOG_RELU_AUX_BIAS:

@@ -503,6 +503,69 @@ def test_gelu_epilog_is_bias_then_gelu(oracle_mod):
     assert np.max(np.abs(rg["Y"] - z * 0.5 * (1 + np.vectorize(math.erf)(z / math.sqrt(2))))) < 1e-15
 
 
+# ------------------------------------------------------------ GELU_AUX_BIAS
+def pin_gelu_aux(fwd, gelu):
+    """GELU_AUX_BIAS's auxiliary output is the pre-activation Z = X.W + bias and
+    Y = gelu(Z). Pinned to the hand-worked forward example (Z worked out by
+    hand there), to the X = I closed form (Z = W + bias), and to GELU's own
+    pins through ``gelu``."""
+    fails = []
+    g = _load("linear_fwd_hand.json")
+    for dt in ("fp16", "bf16"):
+        r = fwd(_bits(g["X"], dt), _bits(g["W"], dt), _bits(g["bias"], dt), DT[dt], "GELU_AUX_BIAS")
+        if not np.array_equal(r["pre"], np.array(g["Z"], dtype=np.float64)):
+            fails.append(f"hand-worked Z ({dt})")
+        if np.max(np.abs(r["Y"] - gelu(np.array(g["Z"], dtype=np.float64)))) > 0.0:
+            fails.append(f"hand-worked Y ({dt})")
+    rng = np.random.default_rng(3)
+    n = 6
+    Wv = (rng.integers(-64, 64, size=(n, 10)) / 16.0)
+    bv = (rng.integers(-64, 64, size=10) / 32.0)
+    r = fwd(_bits(np.eye(n).tolist(), "bf16"), _bits(Wv.tolist(), "bf16"), _bits(bv.tolist(), "bf16"), 1,
+            "GELU_AUX_BIAS")
+    if not np.array_equal(r["pre"], Wv + bv[None, :]):
+        fails.append("closed form X = I")
+    return fails
+
+
+def test_gelu_aux_pins(oracle_mod):
+    fails = pin_gelu_aux(oracle_mod.linear_fwd, oracle_mod.gelu)
+    assert not fails, fails
+
+
+def test_gelu_aux_planted_mistakes_are_caught(oracle_mod):
+    o = oracle_mod
+
+    def mutant(change):
+        def fwd(X, W, b, dt, ep, **kw):
+            r = o.linear_fwd(X, W, b, dt, "GELU_AUX_BIAS", **kw)
+            change(r, X, W, b, dt)
+            return r
+        return fwd
+
+    def no_bias(r, X, W, b, dt):
+        r["pre"] = o.linear_fwd(X, W, None, dt, "NONE")["Y"]
+
+    mutants = {
+        "aux holds gelu(Z)": lambda r, *a: r.__setitem__("pre", o.gelu(r["Z"])),
+        "aux holds X.W without the bias": no_bias,
+        "aux holds relu(Z)": lambda r, *a: r.__setitem__("pre", np.maximum(r["Z"], 0.0)),
+        "Y is relu(Z)": lambda r, *a: r.__setitem__("Y", np.maximum(r["Z"], 0.0)),
+        "aux transposed": lambda r, *a: r.__setitem__("pre", r["Z"].T.copy() if r["Z"].shape[0] == r["Z"].shape[1]
+                                                        else r["Z"][::-1].copy()),
+    }
+    for name, change in mutants.items():
+        assert pin_gelu_aux(mutant(change), o.gelu), f"pins did not catch: {name}"
+
+
+def test_gelu_aux_is_gelu_bias_plus_its_pre_activation(oracle_mod):
+    inp = synth.make_shape_inputs(9, 24, 40, "bf16", seed=43)
+    X, W, b = (synth.bits_u16(inp[k]) for k in ("X", "W", "bias"))
+    rg = oracle_mod.linear_fwd(X, W, b, 1, "GELU_BIAS")
+    ra = oracle_mod.linear_fwd(X, W, b, 1, "GELU_AUX_BIAS")
+    assert np.array_equal(ra["Y"], rg["Y"]) and np.array_equal(ra["pre"], rg["Z"]) and "pre" not in rg
+
+
 # ------------------------------------------------------------------ WGRAD
 def pin_wgrad(wg):
     fails = []
