@@ -91,6 +91,8 @@ def algorithmic(w: synth.Workload, fwd_epi: str, bwd: bool):
     aux_bytes = w.T * math.ceil(w.N / 32) * 4
     f_fwd = 2.0 * w.T * w.N * w.K
     b_fwd = e * (w.T * w.K + w.K * w.N + w.N + w.T * w.N) + (aux_bytes if fwd_epi == "RELU_AUX_BIAS" else 0)
+    if fwd_epi == "GELU_AUX_BIAS":  # the pre-activation written as the auxiliary output
+        b_fwd += e * w.T * w.N
     if fwd_epi == "WGRAD":  # dW = X^T dZ: reads X and dZ, writes dW
         b_fwd = e * (w.T * w.K + w.T * w.N + w.K * w.N)
     if fwd_epi == "FFN_STEP":  # two-layer block, D = K, F = N: 2 forward and 4 backward products
@@ -110,70 +112,119 @@ def algorithmic(w: synth.Workload, fwd_epi: str, bwd: bool):
 
 
 # ----------------------------------------------------------------- clocks
+REASON_BITS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20, "sw_power_cap": 0x4}
+
+
+def summarise_clock_samples(samples, t0, t1, t_warm0=None):
+    """samples: (time, sm_mhz, max_mhz, power_w, reasons bitmask). Median SM
+    clock and the active reasons inside [t0, t1] (the timed region), and over
+    [t_warm0, t1] (warm-up and timed region) when given; falls back to every
+    sample if none falls inside."""
+    def stats(lo, hi):
+        inside = [x for x in samples if lo <= x[0] <= hi]
+        return inside
+
+    inside = stats(t0, t1)
+    wide = stats(t_warm0, t1) if t_warm0 is not None else inside
+    use = inside or wide or list(samples)
+    if not use:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+    reasons = sorted({n for x in use for n, b in REASON_BITS.items() if x[4] & b})
+    out = {"sm_mhz": statistics.median(x[1] for x in use), "sm_max_mhz": max(x[2] for x in use),
+           "samples": len(inside), "reasons": reasons, "power_w_max": max(x[3] for x in use)}
+    if t_warm0 is not None and wide:
+        out["warmup_and_timed"] = {
+            "samples": len(wide), "sm_mhz": statistics.median(x[1] for x in wide),
+            "sm_mhz_min": min(x[1] for x in wide),
+            "reasons": sorted({n for x in wide for n, b in REASON_BITS.items() if x[4] & b})}
+    return out
+
+
 class ClockSampler:
+    """Polls the GPU's SM clock, power and clock-event reasons through NVML
+    every 5 ms in a thread (reads only; no setting is changed), from before
+    the warm-up to the end of the timed region. Falls back to nvidia-smi at
+    its shortest period when NVML cannot be loaded."""
     FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    PERIOD_S = 0.005
 
     def __init__(self, uuid: str | None):
         self.uuid = uuid
-        self.proc = None
-        self.lines = []
+        self.samples = []
+        self.stop_flag = threading.Event()
         self.t = None
+        self.proc = None
+        self.source = None
 
     def start(self):
         try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            h = None
+            if self.uuid:
+                try:
+                    u = self.uuid if self.uuid.startswith("GPU-") else "GPU-" + self.uuid
+                    h = pynvml.nvmlDeviceGetHandleByUUID(u)
+                except Exception:
+                    h = None
+            if h is None:
+                h = pynvml.nvmlDeviceGetHandleByIndex(0)
+            self.source = "nvml, 5 ms"
+            self.t = threading.Thread(target=self._poll_nvml, args=(pynvml, h), daemon=True)
+            self.t.start()
+            return
+        except Exception:
+            pass
+        try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                                          "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                                          "-lms", "20"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.source = "nvidia-smi, 20 ms"
+            self.t = threading.Thread(target=self._read_smi, daemon=True)
+            self.t.start()
         except Exception:
             self.proc = None
-            return
-        self.t = threading.Thread(target=self._read, daemon=True)
-        self.t.start()
 
-    def _read(self):
+    def _poll_nvml(self, nv, h):
+        clk = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        while not self.stop_flag.is_set():
+            try:
+                self.samples.append((time.time(), float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)), float(mx),
+                                     nv.nvmlDeviceGetPowerUsage(h) / 1000.0, int(clk(h))))
+            except Exception:
+                pass
+            time.sleep(self.PERIOD_S)
+
+    def _read_smi(self):
         for line in self.proc.stdout:
-            self.lines.append((time.time(), line.strip()))
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10 or (self.uuid and self.uuid not in parts[1]):
+                continue
+            try:
+                bits = sum(b for n, b in REASON_BITS.items()
+                           if parts[6 + list(REASON_BITS).index(n)].lower().startswith("active"))
+                self.samples.append((time.time(), float(parts[2]), float(parts[3]), float(parts[4]), bits))
+            except ValueError:
+                continue
 
-    def stop(self, t0, t1):
-        if not self.proc:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
+    def stop(self, t0, t1, t_warm0=None):
+        self.stop_flag.set()
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
         if self.t:
             self.t.join(timeout=2)
-        rows = []
-        for ts, line in self.lines:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 10:
-                continue
-            if self.uuid and self.uuid not in parts[1]:
-                continue
-            rows.append((ts, parts))
-        if not rows and self.lines:  # uuid did not match: take the first GPU
-            rows = [(ts, [p.strip() for p in line.split(",")]) for ts, line in self.lines]
-            idx0 = rows[0][1][0]
-            rows = [r for r in rows if len(r[1]) >= 10 and r[1][0] == idx0]
-        inside = [p for ts, p in rows if t0 <= ts <= t1] or [p for _, p in rows]
-        if not inside:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-
-        def num(x):
-            try:
-                return float(x)
-            except ValueError:
-                return None
-
-        sm = [num(p[2]) for p in inside if num(p[2]) is not None]
-        mx = [num(p[3]) for p in inside if num(p[3]) is not None]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for p in inside for i in range(4) if p[6 + i].lower().startswith("active")})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "samples": len(inside), "reasons": reasons,
-                "power_w_max": max((num(p[4]) or 0.0) for p in inside)}
+        if self.source is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no clock source"]}
+        out = summarise_clock_samples(self.samples, t0, t1, t_warm0)
+        out["source"] = self.source
+        return out
 
 
 def roofline(w, fwd_epi, res, peaks, peak_src):
@@ -272,7 +323,8 @@ def run_ours(args, w: synth.Workload, rank: int, world: int, dev: torch.device):
         G = torch.empty((w.T, w.N), dtype=dt, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-    fwd_aux = aux if fwd_epi == "RELU_AUX_BIAS" else None
+    fwd_aux = (aux if fwd_epi == "RELU_AUX_BIAS" else
+               torch.empty((w.T, w.N), dtype=dt, device=dev) if fwd_epi == "GELU_AUX_BIAS" else None)
 
     # prebuilt C calls: the timed loop does no per-call argument checking
     step_plans = None
@@ -343,12 +395,6 @@ def run_ours(args, w: synth.Workload, rank: int, world: int, dev: torch.device):
                 flush.zero_()
                 step(ev)
 
-    run_steps([new_events() for _ in range(args.warmup)])
-    torch.cuda.synchronize(dev)
-    for p in (step_plans if args.ffn_step else (fplan, bplan)):
-        if p is not None and p.status() != 0:
-            raise RuntimeError("watchdog fired during warm-up")
-
     uuid = None
     try:
         uuid = str(torch.cuda.get_device_properties(dev).uuid)
@@ -357,7 +403,15 @@ def run_ours(args, w: synth.Workload, rank: int, world: int, dev: torch.device):
     sampler = ClockSampler(uuid) if rank == 0 else None
     if sampler:
         sampler.start()
-        time.sleep(0.3)
+        time.sleep(0.05)
+    torch.cuda.synchronize(dev)
+    warm0 = time.time()
+    run_steps([new_events() for _ in range(args.warmup)])
+    torch.cuda.synchronize(dev)
+    for p in (step_plans if args.ffn_step else (fplan, bplan)):
+        if p is not None and p.status() != 0:
+            raise RuntimeError("watchdog fired during warm-up")
+
     evs = [new_events() for _ in range(args.steps)]
     if world > 1:
         torch.distributed.barrier()
@@ -368,7 +422,7 @@ def run_ours(args, w: synth.Workload, rank: int, world: int, dev: torch.device):
     wall1 = time.time()
     if world > 1:
         torch.distributed.barrier()
-    clocks = sampler.stop(wall0, wall1) if sampler else None
+    clocks = sampler.stop(wall0, wall1, warm0) if sampler else None
     for p in (step_plans if args.ffn_step else (fplan, bplan)):
         if p is not None and p.status() != 0:
             raise RuntimeError("watchdog fired during the timed region")
@@ -602,7 +656,8 @@ def main():
                     help="time a whole two-layer block step (2 forward, 4 backward products) on the workload's shape")
     ap.add_argument("--wgrad", action="store_true",
                     help="time the weight gradient dW = X^T dZ alone on the workload's shape")
-    ap.add_argument("--fwd-epilog", choices=["BIAS", "RELU_BIAS", "RELU_AUX_BIAS", "GELU_BIAS"], default=None,
+    ap.add_argument("--fwd-epilog", choices=["BIAS", "RELU_BIAS", "RELU_AUX_BIAS", "GELU_BIAS", "GELU_AUX_BIAS"],
+                    default=None,
                     help="time this forward epilog alone on the workload's shape instead of its own step")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -13,9 +13,9 @@ import os
 import torch
 
 F16, BF16 = 0, 1
-BIAS, RELU_BIAS, RELU_AUX_BIAS, DRELU_BGRAD, GELU_BIAS, WGRAD, NONE = 0, 1, 2, 3, 4, 5, 6
+BIAS, RELU_BIAS, RELU_AUX_BIAS, DRELU_BGRAD, GELU_BIAS, WGRAD, NONE, GELU_AUX_BIAS = 0, 1, 2, 3, 4, 5, 6, 7
 EPILOGS = {"BIAS": BIAS, "RELU_BIAS": RELU_BIAS, "RELU_AUX_BIAS": RELU_AUX_BIAS, "DRELU_BGRAD": DRELU_BGRAD,
-           "GELU_BIAS": GELU_BIAS, "WGRAD": WGRAD, "NONE": NONE}
+           "GELU_BIAS": GELU_BIAS, "WGRAD": WGRAD, "NONE": NONE, "GELU_AUX_BIAS": GELU_AUX_BIAS}
 DTYPES = {torch.float16: F16, torch.bfloat16: BF16}
 
 OK = 0
@@ -179,6 +179,20 @@ class Plan:
         self.handle = gemm_epi_plan(T, N, K, dtype, self.epilog,
                                     (FLAG_W_NK if w_nk else 0) | (FLAG_OUT_F32 if out_f32 else 0))
 
+    def aux_spec(self):
+        """Shape and dtype of the forward's auxiliary output: the mask words
+        (T x ceil(N/32) int32) for RELU_AUX_BIAS, the pre-activation (T x N,
+        the plan's 16-bit type) for GELU_AUX_BIAS, None otherwise."""
+        if self.epilog == RELU_AUX_BIAS:
+            return (self.T, self.aux_words), torch.int32
+        if self.epilog == GELU_AUX_BIAS:
+            return (self.T, self.N), self.dtype
+        return None
+
+    def _aux(self, aux):
+        spec = self.aux_spec() or ((self.T, self.aux_words), torch.int32)
+        return _ptr(aux, spec[0], spec[1], "aux")
+
     def set_bias_f32(self, on: bool = True):
         """Read the forward bias as fp32 (True) or in the plan's 16-bit type (False)."""
         _check(lib().gemm_epi_set_bias_f32(self.handle, 1 if on else 0))
@@ -215,7 +229,7 @@ class Plan:
     def gemm_epi_execute(self, X, W, bias, Y, aux=None, stream=None):
         T, N, K, dt = self.T, self.N, self.K, self.dtype
         args = (_ptr(X, (T, K), dt, "X"), _ptr(W, self.w_shape, dt, "W"), _ptr(bias, (N,), self.bias_dtype, "bias"),
-                _ptr(Y, (T, N), self.out_dtype, "Y"), _ptr(aux, (T, self.aux_words), torch.int32, "aux"))
+                _ptr(Y, (T, N), self.out_dtype, "Y"), self._aux(aux))
         _check(lib().gemm_epi_execute(self.handle, *args, _stream_ptr(stream)))
 
     def drelu_bgrad_execute(self, dY2, W2, aux, dZ, dbias, stream=None):
@@ -237,7 +251,7 @@ class Plan:
         T, N, K, dt = self.T, self.N, self.K, self.dtype
         args = (_ptr(X, (T, K), dt, "X"), _ptr(W, self.w_shape, dt, "W"), _ptr(bias, (N,), self.bias_dtype, "bias"),
                 _ptr(T1, (T, N), dt, "T1"), _ptr(T2, (T, N), dt, "T2"), _ptr(Y, (T, N), self.out_dtype, "Y"),
-                _ptr(aux, (T, self.aux_words), torch.int32, "aux"))
+                self._aux(aux))
         _check(lib().gemm_epi_unfused_execute(self.handle, *args, _stream_ptr(stream)))
 
     def drelu_bgrad_unfused_execute(self, dY2, W2, aux, G, dZ, dbias, stream=None):
@@ -252,7 +266,7 @@ class Plan:
     def execute_call(self, X, W, bias, Y, aux=None, stream=None):
         T, N, K, dt = self.T, self.N, self.K, self.dtype
         args = (self.handle, _ptr(X, (T, K), dt, "X"), _ptr(W, self.w_shape, dt, "W"), _ptr(bias, (N,), self.bias_dtype, "bias"),
-                _ptr(Y, (T, N), self.out_dtype, "Y"), _ptr(aux, (T, self.aux_words), torch.int32, "aux"), _stream_ptr(stream))
+                _ptr(Y, (T, N), self.out_dtype, "Y"), self._aux(aux), _stream_ptr(stream))
         return lib().gemm_epi_execute, args
 
     def drelu_bgrad_call(self, dY2, W2, aux, dZ, dbias, stream=None):
@@ -273,7 +287,7 @@ class Plan:
         T, N, K, dt = self.T, self.N, self.K, self.dtype
         args = (self.handle, _ptr(X, (T, K), dt, "X"), _ptr(W, self.w_shape, dt, "W"), _ptr(bias, (N,), self.bias_dtype, "bias"),
                 _ptr(T1, (T, N), dt, "T1"), _ptr(T2, (T, N), dt, "T2"), _ptr(Y, (T, N), self.out_dtype, "Y"),
-                _ptr(aux, (T, self.aux_words), torch.int32, "aux"), _stream_ptr(stream))
+                self._aux(aux), _stream_ptr(stream))
         return lib().gemm_epi_unfused_execute, args
 
     def drelu_bgrad_unfused_call(self, dY2, W2, aux, G, dZ, dbias, stream=None):
@@ -287,8 +301,8 @@ class Plan:
     # outside the library; the library call itself allocates nothing)
     def forward(self, X, W, bias, stream=None):
         Y = torch.empty((self.T, self.N), dtype=self.out_dtype, device=X.device)
-        aux = (torch.empty((self.T, self.aux_words), dtype=torch.int32, device=X.device)
-               if self.epilog == RELU_AUX_BIAS else None)
+        spec = self.aux_spec()
+        aux = torch.empty(spec[0], dtype=spec[1], device=X.device) if spec else None
         self.gemm_epi_execute(X, W, bias, Y, aux, stream)
         return Y, aux
 

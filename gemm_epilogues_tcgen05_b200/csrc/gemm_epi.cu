@@ -14,6 +14,7 @@
 
 #include "../../include/gemm_epi.h"
 #include "aux_kernels.cuh"
+#include "kernel_table.h"
 #include "skinny_kernel.cuh"
 #include "tile2_kernel.cuh"
 #include "tile_kernel.cuh"
@@ -48,10 +49,41 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-// Fault injection for the host tests: GEMM_EPI_INJECT_ENCODE_FAILURE makes every
-// tensor-map encode fail, so an execute call must return GEMM_EPI_ERR_CUDA
-// before it launches anything.
-bool inject_encode_failure() { return getenv("GEMM_EPI_INJECT_ENCODE_FAILURE") != nullptr; }
+// Fault-injection hooks for the tests take effect only while
+// GEMM_EPI_TEST_HOOKS=1 is set as well, so that one stray variable inherited
+// by a production process cannot make its plans stall or fail.
+bool test_hooks_on() {
+  const char* f = getenv("GEMM_EPI_TEST_HOOKS");
+  return f && atoi(f) == 1;
+}
+bool test_hook(const char* name) {
+  const char* f = test_hooks_on() ? getenv(name) : nullptr;
+  return f && atoi(f) != 0;
+}
+
+// GEMM_EPI_INJECT_ENCODE_FAILURE makes every tensor-map encode fail, so an
+// execute call must return GEMM_EPI_ERR_CUDA before it launches anything.
+bool inject_encode_failure() { return test_hook("GEMM_EPI_INJECT_ENCODE_FAILURE"); }
+
+// The watchdog settings a launch carries: the limit of each bounded wait
+// (2 s; GEMM_EPI_WAIT_TIMEOUT_MS overrides) and, for the watchdog tests,
+// GEMM_EPI_INJECT_STALL -- the MMA issuer withholds its first tile's
+// completion signal, so the epilogue's wait runs out and the kernel reports
+// ERR_TIMEOUT. Read when a plan is created and on every call of the
+// allocation-free entry point.
+struct WatchdogEnv {
+  uint64_t timeout_ns = 2000000000ull;
+  int inject_stall = 0;
+};
+WatchdogEnv watchdog_env() {
+  WatchdogEnv w;
+  if (const char* t = getenv("GEMM_EPI_WAIT_TIMEOUT_MS")) {
+    const long long ms = atoll(t);
+    if (ms > 0) w.timeout_ns = (uint64_t)ms * 1000000ull;
+  }
+  w.inject_stall = test_hook("GEMM_EPI_INJECT_STALL") ? 1 : 0;
+  return w;
+}
 
 EncodeTiledFn encode_fn() {
   static EncodeTiledFn fn = nullptr;
@@ -86,7 +118,8 @@ int encode_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer
   return GEMM_EPI_OK;
 }
 
-using TileKernelFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, ge::TileParams);
+using ge_inst::SkinnyKernelFn;
+using ge_inst::TileKernelFn;
 
 // the output (Y, dZ or an unfused intermediate) as the tile kernels' TMA
 // stores see it: 32 x 32 blocks, 64-byte swizzle
@@ -140,26 +173,9 @@ static_assert(static_cast<int>(GEMM_EPI_BIAS) == ge::EPI_BIAS && static_cast<int
                   static_cast<int>(GEMM_EPI_DRELU_BGRAD) == ge::EPI_DRELU_BGRAD &&
                   static_cast<int>(GEMM_EPI_GELU_BIAS) == ge::EPI_GELU_BIAS &&
                   static_cast<int>(GEMM_EPI_WGRAD) == ge::EPI_WGRAD &&
-                  static_cast<int>(GEMM_EPI_NONE) == ge::EPI_STORE,
+                  static_cast<int>(GEMM_EPI_NONE) == ge::EPI_STORE &&
+                  static_cast<int>(GEMM_EPI_GELU_AUX_BIAS) == ge::EPI_GELU_AUX_BIAS,
               "the public epilog values are the kernels' epilog kinds");
-
-// BK: the weight is given N x K (GEMM_EPI_FLAG_W_NK); never with WGRAD
-template <int BN, int ST, bool BF, bool BK>
-TileKernelFn pick_epi(int epi) {
-  switch (epi) {
-    case ge::EPI_BIAS: return ge::tile_kernel<BN, ST, ge::EPI_BIAS, BF, BK>;
-    case ge::EPI_RELU_BIAS: return ge::tile_kernel<BN, ST, ge::EPI_RELU_BIAS, BF, BK>;
-    case ge::EPI_RELU_AUX_BIAS: return ge::tile_kernel<BN, ST, ge::EPI_RELU_AUX_BIAS, BF, BK>;
-    case ge::EPI_DRELU_BGRAD: return ge::tile_kernel<BN, ST, ge::EPI_DRELU_BGRAD, BF, BK>;
-    case ge::EPI_GELU_BIAS: return ge::tile_kernel<BN, ST, ge::EPI_GELU_BIAS, BF, BK>;
-    case ge::EPI_WGRAD:
-      if constexpr (BK)
-        return nullptr;
-      else
-        return ge::tile_kernel<BN, ST, ge::EPI_WGRAD, BF>;
-    default: return ge::tile_kernel<BN, ST, ge::EPI_STORE, BF, BK>;
-  }
-}
 
 struct TileCfg {
   int BN = 256, stages = 4;
@@ -168,77 +184,65 @@ struct TileCfg {
   bool pair = false;  // CTA-pair kernel, launched in clusters of 2
 };
 
-template <bool BF, bool BK>
-TileKernelFn pick_pair_epi(int epi) {
-  switch (epi) {
-    case ge::EPI_BIAS: return ge::tile2_kernel<256, 6, ge::EPI_BIAS, BF, BK>;
-    case ge::EPI_RELU_BIAS: return ge::tile2_kernel<256, 6, ge::EPI_RELU_BIAS, BF, BK>;
-    case ge::EPI_RELU_AUX_BIAS: return ge::tile2_kernel<256, 6, ge::EPI_RELU_AUX_BIAS, BF, BK>;
-    case ge::EPI_DRELU_BGRAD: return ge::tile2_kernel<256, 6, ge::EPI_DRELU_BGRAD, BF, BK>;
-    case ge::EPI_GELU_BIAS: return ge::tile2_kernel<256, 6, ge::EPI_GELU_BIAS, BF, BK>;
-    case ge::EPI_WGRAD:
-      if constexpr (BK)
-        return nullptr;
-      else
-        return ge::tile2_kernel<256, 6, ge::EPI_WGRAD, BF>;
-    default: return ge::tile2_kernel<256, 6, ge::EPI_STORE, BF, BK>;
-  }
-}
-
-template <int BN, int ST>
-TileKernelFn pick_tile(int epi, bool bf16, bool bk) {
-  if (bk) return bf16 ? pick_epi<BN, ST, true, true>(epi) : pick_epi<BN, ST, false, true>(epi);
-  return bf16 ? pick_epi<BN, ST, true, false>(epi) : pick_epi<BN, ST, false, false>(epi);
-}
-
-TileCfg pair_cfg(int epi, bool bf16, bool bk) {
+// bk: the weight is given N x K (GEMM_EPI_FLAG_W_NK); never with WGRAD
+TileCfg pair_cfg(int epi, bool bf16, bool bk, bool split = false) {
   TileCfg c;
   c.BN = 256;
   c.stages = 6;
   c.smem = ge::Tile2Smem<256, 6>::BYTES;
-  if (bk)
-    c.fn = bf16 ? pick_pair_epi<true, true>(epi) : pick_pair_epi<false, true>(epi);
+  if (split)
+    c.fn = bf16 ? ge_inst::pair_split_bf16(epi, bk) : ge_inst::pair_split_f16(epi, bk);
   else
-    c.fn = bf16 ? pick_pair_epi<true, false>(epi) : pick_pair_epi<false, false>(epi);
+    c.fn = bf16 ? ge_inst::pair_bf16(epi, bk) : ge_inst::pair_f16(epi, bk);
   c.pair = true;
   return c;
 }
 
+// How many CTA pairs of this kernel the device holds at once (clusters of
+// two must sit in one GPC); one pair per two SMs if the query fails.
+int max_resident_pairs(const TileCfg& c, int sms) {
+  if (cudaFuncSetAttribute(c.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)c.smem) != cudaSuccess) {
+    cudaGetLastError();
+    return sms / 2;
+  }
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3((unsigned)(sms / 2 * 2), 1, 1);
+  lc.blockDim = dim3(ge::kThreads, 1, 1);
+  lc.dynamicSmemBytes = c.smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, (const void*)c.fn, &lc) != cudaSuccess || n < 1) {
+    cudaGetLastError();
+    return sms / 2;
+  }
+  return n < sms / 2 ? n : sms / 2;
+}
+
 TileCfg tile_cfg(int BN, int epi, bool bf16, bool bk) {
   TileCfg c;
-  c.BN = BN;
-  if (BN == 256) {
+  c.BN = BN == 256 || BN == 128 ? BN : 64;
+  if (c.BN == 256) {
     c.stages = 4;
     c.smem = ge::TileSmem<256, 4>::BYTES;
-    c.fn = pick_tile<256, 4>(epi, bf16, bk);
-  } else if (BN == 128) {
+  } else if (c.BN == 128) {
     c.stages = 6;
     c.smem = ge::TileSmem<128, 6>::BYTES;
-    c.fn = pick_tile<128, 6>(epi, bf16, bk);
   } else {
-    c.BN = 64;
     c.stages = 8;
     c.smem = ge::TileSmem<64, 8>::BYTES;
-    c.fn = pick_tile<64, 8>(epi, bf16, bk);
   }
+  c.fn = bk ? (bf16 ? ge_inst::tile_bf16_nk(c.BN, epi) : ge_inst::tile_f16_nk(c.BN, epi))
+            : (bf16 ? ge_inst::tile_bf16_mn(c.BN, epi) : ge_inst::tile_f16_mn(c.BN, epi));
   return c;
 }
 
 int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
-
-using SkinnyKernelFn = void (*)(CUtensorMap, CUtensorMap, ge::SkinnyParams);
-
-template <int TP, int KPS, bool BF>
-SkinnyKernelFn pick_skinny_epi(int epi) {
-  switch (epi) {
-    case ge::EPI_BIAS: return ge::skinny_kernel<TP, KPS, ge::EPI_BIAS, BF>;
-    case ge::EPI_RELU_BIAS: return ge::skinny_kernel<TP, KPS, ge::EPI_RELU_BIAS, BF>;
-    case ge::EPI_RELU_AUX_BIAS: return ge::skinny_kernel<TP, KPS, ge::EPI_RELU_AUX_BIAS, BF>;
-    case ge::EPI_GELU_BIAS: return ge::skinny_kernel<TP, KPS, ge::EPI_GELU_BIAS, BF>;
-    case ge::EPI_STORE: return ge::skinny_kernel<TP, KPS, ge::EPI_STORE, BF>;
-    default: return ge::skinny_kernel<TP, KPS, ge::EPI_DRELU_BGRAD, BF>;
-  }
-}
 
 struct SkinnyCfg {
   int TP = 16;
@@ -253,7 +257,10 @@ SkinnyCfg skinny_cfg_kps(int epi, bool bf16) {
   SkinnyCfg c;
   c.TP = TP;
   c.KPS = KPS;
-  c.fn = bf16 ? pick_skinny_epi<TP, KPS, true>(epi) : pick_skinny_epi<TP, KPS, false>(epi);
+  if constexpr (KPS == 2)
+    c.fn = bf16 ? ge_inst::skinny_bf16_kps2(TP, epi) : ge_inst::skinny_f16_kps2(TP, epi);
+  else
+    c.fn = bf16 ? ge_inst::skinny_bf16_kps1(TP, epi) : ge_inst::skinny_f16_kps1(TP, epi);
   c.smem = ge::SkinnySmem<TP, KPS>::BYTES;
   c.stages = ge::SkinnySmem<TP, KPS>::STAGES;
   return c;
@@ -327,6 +334,13 @@ struct gemm_epi_plan_s {
   int dtype, epilog;
   int device, num_sms;
   int m_tiles, n_tiles, k_blocks, num_tiles, aux_words, grid, group_m;
+  int raster_n = 0;  // tile order by column groups (see choose_raster)
+  int pair_split = 0;        // CTA pairs in stream-K mode
+  int pair_max_segs = 1;
+  float* pair_slots = nullptr;  // stream-K fp32 partials
+  int* pair_flags = nullptr;    // stream-K segment counters, zero between launches
+  int n_pair_flags = 0;
+  size_t pair_bytes = 0;
   TileCfg cfg;       // fused kernel
   TileCfg cfg_store; // unfused GEMM (plain store)
   float* partials = nullptr;  // DRELU_BGRAD: m_tiles x N
@@ -378,6 +392,7 @@ int take_status(gemm_epi_plan_s* p) {
     // an interrupted launch may have left split-tile tickets counted
     if (p->sk_tickets) cudaMemset(p->sk_tickets, 0, sizeof(int) * (size_t)ceil_div(p->N, 128));
     if (p->col_tickets) cudaMemset(p->col_tickets, 0, sizeof(int) * (size_t)p->n_tickets);
+    if (p->pair_flags) cudaMemset(p->pair_flags, 0, sizeof(int) * (size_t)p->n_pair_flags);
     return fail(GEMM_EPI_ERR_TIMEOUT, "a kernel of this plan gave up waiting (watchdog code 0x%x)", v);
   }
   return GEMM_EPI_OK;
@@ -419,6 +434,10 @@ ge::TileParams base_params(const gemm_epi_plan_s* p) {
   k.num_tiles = p->num_tiles;
   k.aux_words = p->aux_words;
   k.group_m = p->group_m;
+  k.raster_n = p->raster_n;
+  k.sk_slots = p->pair_slots;
+  k.sk_flags = p->pair_flags;
+  k.sk_max_segs = p->pair_max_segs;
   k.status = p->status_dev;
   k.timeout_ns = p->timeout_ns;
   k.inject_stall = p->inject_stall;
@@ -442,7 +461,16 @@ int launch_tile(gemm_epi_plan_s* p, const TileCfg& c, const ge::TileParams& k_in
   int rc = prepare_out_map(p, k.out);
   if (rc) return rc;
   k.aux_tma = 0;
-  if (k.aux_out && aux_tma_ok(k.aux_out, p->N, c.BN)) {
+  if (p->epilog == GEMM_EPI_GELU_AUX_BIAS && k.aux_out) {
+    // the pre-activation Z, T x N in the 16-bit type, stored like Y
+    if (k.aux_out != p->aux_ptr) {
+      rc = encode_2d(&p->tmAux, k.aux_out, (uint64_t)p->N, (uint64_t)p->T, 32, 32, "the GELU auxiliary output",
+                     CU_TENSOR_MAP_SWIZZLE_64B);
+      if (rc) return rc;
+      p->aux_ptr = k.aux_out;
+    }
+    k.aux_tma = 1;
+  } else if (k.aux_out && aux_tma_ok(k.aux_out, p->N, c.BN)) {
     if (k.aux_out != p->aux_ptr) {
       rc = encode_aux(&p->tmAux, k.aux_out, p->T, p->N, c.BN);
       if (rc) return rc;
@@ -474,21 +502,46 @@ int launch_tile(gemm_epi_plan_s* p, const TileCfg& c, const ge::TileParams& k_in
   return GEMM_EPI_OK;
 }
 
-// Raster group (in row tiles of `tile_rows`): the group's block of X --
-// group rows x K x 2 bytes -- is kept to about 48 MB, a little under half of
-// the 126 MB L2, so it stays resident while the group sweeps every column
-// block of W. When all of X fits, one group spans every row tile and each
-// column block of W is streamed from HBM once.
-int choose_group_m(int64_t T, int64_t K, int tile_rows) {
-  const int m_tiles = (int)((T + tile_rows - 1) / tile_rows);
-  const int64_t block = (int64_t)tile_rows * K * 2;
-  int64_t g = ((int64_t)48 << 20) / block;
-  if (const char* f = getenv("GEMM_EPI_GROUP_M")) {  // tuning override
-    const int v = atoi(f);
-    if (v >= 1) g = v;
+// Raster: which operand's block stays in L2 while the other streams past
+// it. Holding a group of R row tiles of X (R x tile_rows x K x 2 bytes) while
+// the group sweeps every column block streams W from HBM once per group;
+// holding C column tiles of W streams X once per group. The estimate of the
+// HBM reads of each -- X + ceil(m_tiles / R) W, or W + ceil(n_tiles / C) X --
+// picks the order, with the held block kept to about 48 MB, a little under
+// half of the 126 MB L2 (when all of X fits, W is streamed once). The column
+// order wins only when X is much larger than W (the 65536 x 16384 x 8192
+// problem: X 2 GiB, W 256 MiB). GEMM_EPI_RASTER=m|n and GEMM_EPI_GROUP_M (the
+// group size in tiles) override, for measurement.
+struct Raster {
+  int group = 1;
+  int by_n = 0;
+};
+
+Raster choose_raster(int64_t T, int64_t N, int64_t K, int tile_rows, int tile_cols) {
+  const int64_t m_tiles = (T + tile_rows - 1) / tile_rows, n_tiles = (N + tile_cols - 1) / tile_cols;
+  const double budget = double(48 << 20);
+  const double x_bytes = 2.0 * T * K, w_bytes = 2.0 * K * N;
+  int64_t R = (int64_t)(budget / (2.0 * tile_rows * K)), C = (int64_t)(budget / (2.0 * tile_cols * K));
+  R = R < 1 ? 1 : R > m_tiles ? m_tiles : R;
+  C = C < 1 ? 1 : C > n_tiles ? n_tiles : C;
+  const double by_m = x_bytes + double((m_tiles + R - 1) / R) * w_bytes;
+  const double by_n = w_bytes + double((n_tiles + C - 1) / C) * x_bytes;
+  Raster r;
+  r.by_n = by_n < 0.9 * by_m ? 1 : 0;
+  r.group = (int)(r.by_n ? C : R);
+  if (const char* f = getenv("GEMM_EPI_RASTER")) {  // tuning override
+    if (!strcmp(f, "m") || !strcmp(f, "n")) {
+      r.by_n = f[0] == 'n';
+      r.group = (int)(r.by_n ? C : R);
+    }
   }
-  if (g < 1) g = 1;
-  return g >= m_tiles ? m_tiles : (int)g;
+  if (const char* f = getenv("GEMM_EPI_GROUP_M")) {  // tuning override: the group size in tiles
+    const int v = atoi(f);
+    if (v >= 1) r.group = v;
+  }
+  const int64_t outer = r.by_n ? n_tiles : m_tiles;
+  if (r.group > outer) r.group = (int)outer;
+  return r;
 }
 
 int prepare_skinny_maps(gemm_epi_plan_s* p, const void* A, const void* B) {
@@ -524,6 +577,7 @@ ge::SkinnyParams skinny_params(const gemm_epi_plan_s* p) {
   k.bias_f32 = p->bias_f32;
   k.out_f32 = p->out_f32;
   k.cache_hints = p->cache_hints;
+  k.inject_stall = p->inject_stall;
   return k;
 }
 
@@ -580,7 +634,7 @@ gemm_epi_plan_t gemm_epi_plan_ex(int64_t T, int64_t N, int64_t K, gemm_epi_dtype
     fail(GEMM_EPI_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
     return nullptr;
   }
-  if (epilog < GEMM_EPI_BIAS || epilog > GEMM_EPI_NONE) {
+  if (epilog < GEMM_EPI_BIAS || epilog > GEMM_EPI_GELU_AUX_BIAS) {
     fail(GEMM_EPI_ERR_INVALID_ARG, "unknown epilog %d", (int)epilog);
     return nullptr;
   }
@@ -632,26 +686,19 @@ gemm_epi_plan_t gemm_epi_plan_ex(int64_t T, int64_t N, int64_t K, gemm_epi_dtype
   p->k_blocks = ceil_div(K, ge::kBK);
   p->num_tiles = p->m_tiles * p->n_tiles;
   p->aux_words = ceil_div(N, 32);
-  p->group_m = choose_group_m(T, K, pair ? 2 * ge::kBM : ge::kBM);
+  const Raster raster = choose_raster(T, N, K, pair ? 2 * ge::kBM : ge::kBM, bn);
+  p->group_m = raster.group;
+  p->raster_n = raster.by_n;
   p->grid = p->num_tiles < sms ? p->num_tiles : sms;
-  if (pair) {  // one cluster of two CTAs per 256-row x 256-column tile, up to one CTA per SM
-    const int pair_tiles = ceil_div(T, 256) * p->n_tiles;
-    const int pairs = pair_tiles < sms / 2 ? pair_tiles : sms / 2;
-    p->grid = 2 * pairs;
-  }
-  p->timeout_ns = 2000000000ull;  // 2 s per wait
-  if (const char* t = getenv("GEMM_EPI_WAIT_TIMEOUT_MS")) {
-    long long ms = atoll(t);
-    if (ms > 0) p->timeout_ns = (uint64_t)ms * 1000000ull;
-  }
-  // Fault injection for the watchdog tests (one-CTA tile kernel only): the
-  // MMA warp withholds its first tile's completion signal, so the epilogue's
-  // bounded wait runs out and the kernel reports ERR_TIMEOUT.
-  if (const char* f = getenv("GEMM_EPI_INJECT_STALL")) p->inject_stall = atoi(f) != 0;
+  const WatchdogEnv wd = watchdog_env();
+  p->timeout_ns = wd.timeout_ns;
+  p->inject_stall = wd.inject_stall;
   if (const char* f = getenv("GEMM_EPI_TAIL_SPLIT")) p->tail_split = atoi(f) != 0;
 
 
   auto cleanup = [&](int rc) {
+    if (p->pair_slots) cudaFree(p->pair_slots);
+    if (p->pair_flags) cudaFree(p->pair_flags);
     if (p->col_tickets) cudaFree(p->col_tickets);
     if (p->sk_partials) cudaFree(p->sk_partials);
     if (p->sk_tickets) cudaFree(p->sk_tickets);
@@ -662,7 +709,50 @@ gemm_epi_plan_t gemm_epi_plan_ex(int64_t T, int64_t N, int64_t K, gemm_epi_dtype
     return nullptr;
   };
 
+  if (pair) {
+    // One cluster of two CTAs per 256-row x 256-column tile, up to the number
+    // of clusters the device can hold at once (a GPC with an odd number of
+    // free SMs cannot place a pair on its last one). With fewer tiles than
+    // that, stream-K: every pair takes an equal share of the tiles' k-blocks
+    // (at least 8), so the idle pairs stream W too.
+    const int pair_tiles = ceil_div(T, 256) * p->n_tiles;
+    const int max_pairs = max_resident_pairs(p->cfg, sms);
+    int pairs = pair_tiles < max_pairs ? pair_tiles : max_pairs;
+    bool split = pair_tiles < max_pairs && p->k_blocks >= 16;
+    if (const char* f = getenv("GEMM_EPI_PAIR_SPLIT")) split = split && atoi(f) != 0;  // A/B override
+    if (split) {
+      const int64_t want = (int64_t)pair_tiles * p->k_blocks / 8;
+      const int sp = (int)(want < max_pairs ? want : max_pairs);
+      split = sp > pair_tiles;
+      if (split) pairs = sp;
+    }
+    p->grid = 2 * pairs;
+    if (split) {
+      p->pair_split = 1;
+      p->cfg = pair_cfg((int)epilog, bf16, w_nk, true);
+      p->cfg_store = pair_cfg(ge::EPI_STORE, bf16, w_nk, true);
+      const int64_t total = (int64_t)pair_tiles * p->k_blocks;
+      p->pair_max_segs = 1;
+      for (int t = 0; t < pair_tiles; ++t) {
+        const int64_t a = ge::pair_owner((int64_t)t * p->k_blocks, pairs, total);
+        const int64_t b = ge::pair_owner((int64_t)(t + 1) * p->k_blocks - 1, pairs, total);
+        if (b - a + 1 > p->pair_max_segs) p->pair_max_segs = (int)(b - a + 1);
+      }
+      p->pair_bytes = (size_t)pair_tiles * (p->pair_max_segs - 1) * 2 * ge::kBM * 256 * sizeof(float);
+      if (p->pair_bytes) {
+        e = cudaMalloc((void**)&p->pair_slots, p->pair_bytes);
+        if (e != cudaSuccess) return cleanup(cuda_fail(e, "cudaMalloc(stream-K partials)"));
+      }
+      e = cudaMalloc((void**)&p->pair_flags, sizeof(int) * 2 * (size_t)pair_tiles);
+      if (e != cudaSuccess) return cleanup(cuda_fail(e, "cudaMalloc(stream-K flags)"));
+      e = cudaMemset(p->pair_flags, 0, sizeof(int) * 2 * (size_t)pair_tiles);
+      if (e != cudaSuccess) return cleanup(cuda_fail(e, "cudaMemset(stream-K flags)"));
+      p->n_pair_flags = 2 * pair_tiles;
+      p->pair_bytes += sizeof(int) * 2 * (size_t)pair_tiles;
+    }
+  }
   for (const TileCfg* c : {&p->cfg, &p->cfg_store}) {
+    if (!c->fn) return cleanup(fail(GEMM_EPI_ERR_INVALID_ARG, "no kernel instance for this epilog and layout"));
     e = cudaFuncSetAttribute(c->fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)c->smem);
     if (e != cudaSuccess) return cleanup(cuda_fail(e, "cudaFuncSetAttribute(max dynamic shared memory)"));
   }
@@ -723,7 +813,7 @@ gemm_epi_plan_t gemm_epi_plan_ex(int64_t T, int64_t N, int64_t K, gemm_epi_dtype
   // the column partials are needed by the fused and the unfused backward
   p->partial_bytes = (size_t)p->m_tiles * (size_t)N * sizeof(float);
   if (epilog == GEMM_EPI_DRELU_BGRAD) {
-    if (getenv("GEMM_EPI_INJECT_PLAN_ALLOC_FAILURE"))
+    if (test_hook("GEMM_EPI_INJECT_PLAN_ALLOC_FAILURE"))
       return cleanup(fail(GEMM_EPI_ERR_CUDA, "injected workspace allocation failure"));
     e = cudaMalloc((void**)&p->partials, p->partial_bytes);
     if (e != cudaSuccess) return cleanup(cuda_fail(e, "cudaMalloc(workspace)"));
@@ -759,6 +849,8 @@ void gemm_epi_free(gemm_epi_plan_t plan) {
   }
   if (plan->partials) cudaFree(plan->partials);
   if (plan->col_tickets) cudaFree(plan->col_tickets);
+  if (plan->pair_slots) cudaFree(plan->pair_slots);
+  if (plan->pair_flags) cudaFree(plan->pair_flags);
   if (plan->sk_partials) cudaFree(plan->sk_partials);
   if (plan->sk_tickets) cudaFree(plan->sk_tickets);
   if (plan->status_host) cudaFreeHost(plan->status_host);
@@ -792,12 +884,13 @@ int gemm_epi_query(gemm_epi_plan_t plan, gemm_epi_info* info) {
     info->tile_n = p->cfg.BN;
     info->tile_k = ge::kBK;
     info->stages = p->cfg.stages;
-    info->split_k = 1;
+    info->split_k = p->pair_split ? p->pair_max_segs : 1;
     info->grid = p->grid;
     info->launches = 1;
-    info->workspace_bytes = p->epilog == GEMM_EPI_DRELU_BGRAD ? p->partial_bytes + sizeof(int) * (size_t)p->n_tickets
-                            : p->epilog == GEMM_EPI_WGRAD    ? p->partial_bytes
-                                                             : 0;
+    info->workspace_bytes = p->pair_bytes +
+                            (p->epilog == GEMM_EPI_DRELU_BGRAD ? p->partial_bytes + sizeof(int) * (size_t)p->n_tickets
+                             : p->epilog == GEMM_EPI_WGRAD     ? p->partial_bytes
+                                                               : 0);
   }
   return GEMM_EPI_OK;
 }
@@ -817,11 +910,13 @@ int gemm_epi_execute(gemm_epi_plan_t plan, const void* X, const void* W, const v
                 p->epilog == GEMM_EPI_WGRAD ? "WGRAD" : "DRELU_BGRAD");
   if (!X || !W || !Y || (!bias && p->epilog != GEMM_EPI_NONE))
     return fail(GEMM_EPI_ERR_INVALID_ARG, "gemm_epi_execute: NULL X, W, bias or Y");
-  if (p->epilog == GEMM_EPI_RELU_AUX_BIAS && !aux)
-    return fail(GEMM_EPI_ERR_EPILOG_MISMATCH, "RELU_AUX_BIAS needs an aux buffer");
+  const bool gelu_aux = p->epilog == GEMM_EPI_GELU_AUX_BIAS;
+  if ((p->epilog == GEMM_EPI_RELU_AUX_BIAS || gelu_aux) && !aux)
+    return fail(GEMM_EPI_ERR_EPILOG_MISMATCH, "%s needs an aux buffer", gelu_aux ? "GELU_AUX_BIAS" : "RELU_AUX_BIAS");
   if (!aligned(X, 16) || !aligned(W, 16) || !aligned(Y, 16) || !aligned(bias, p->bias_f32 ? 4 : 2) ||
-      (p->epilog == GEMM_EPI_RELU_AUX_BIAS && !aligned(aux, 4)))
-    return fail(GEMM_EPI_ERR_MISALIGNED, "gemm_epi_execute: X, W, Y need 16-byte, bias 2-byte, aux 4-byte alignment");
+      (p->epilog == GEMM_EPI_RELU_AUX_BIAS && !aligned(aux, 4)) || (gelu_aux && !aligned(aux, 16)))
+    return fail(GEMM_EPI_ERR_MISALIGNED,
+                "gemm_epi_execute: X, W, Y need 16-byte, bias 2-byte, aux 4-byte (GELU_AUX_BIAS: 16-byte) alignment");
   int rc = take_status(p);
   if (rc) return rc;
   if (p->kernel == 1) {
@@ -883,9 +978,11 @@ int gemm_epi_unfused_execute(gemm_epi_plan_t plan, const void* X, const void* W,
     return fail(GEMM_EPI_ERR_EPILOG_MISMATCH, "gemm_epi_unfused_execute: the plan's epilog has nothing to unfuse");
   if (p->out_f32)
     return fail(GEMM_EPI_ERR_UNSUPPORTED, "the unfused path keeps 16-bit intermediates and outputs (no fp32 output)");
+  const bool gelu_aux = p->epilog == GEMM_EPI_GELU_AUX_BIAS;
+  if ((p->epilog == GEMM_EPI_RELU_AUX_BIAS || gelu_aux) && !aux)
+    return fail(GEMM_EPI_ERR_EPILOG_MISMATCH, "%s needs an aux buffer", gelu_aux ? "GELU_AUX_BIAS" : "RELU_AUX_BIAS");
+  if (gelu_aux) T2 = aux;  // the bias kernel's output is the auxiliary output Z itself
   if (!X || !W || !bias || !T1 || !T2 || !Y) return fail(GEMM_EPI_ERR_INVALID_ARG, "unfused: NULL pointer");
-  if (p->epilog == GEMM_EPI_RELU_AUX_BIAS && !aux)
-    return fail(GEMM_EPI_ERR_EPILOG_MISMATCH, "RELU_AUX_BIAS needs an aux buffer");
   if (!aligned(X, 16) || !aligned(W, 16) || !aligned(T1, 16) || !aligned(T2, 16) || !aligned(Y, 16) ||
       !aligned(bias, p->bias_f32 ? 4 : 2) || (aux && !aligned(aux, 4)))
     return fail(GEMM_EPI_ERR_MISALIGNED, "unfused: misaligned pointer");
@@ -905,7 +1002,7 @@ int gemm_epi_unfused_execute(gemm_epi_plan_t plan, const void* X, const void* W,
   else
     ge::bias_add_kernel<false><<<blocks, 256, 0, stream>>>((const uint4*)T1, bias, (uint4*)T2, p->T, (int)p->N,
                                                            p->bias_f32);
-  if (p->epilog == GEMM_EPI_GELU_BIAS) {
+  if (p->epilog == GEMM_EPI_GELU_BIAS || gelu_aux) {
     const int64_t n_vec = p->T * p->N / 8;
     if (bf16)
       ge::gelu_kernel<true><<<blocks, 256, 0, stream>>>((const uint4*)T2, (uint4*)Y, n_vec);
@@ -1030,9 +1127,8 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocStatusB
 constexpr int kNoAllocMaxDevices = 64;
 
 struct NoAllocDevice {
-  std::once_flag once;
-  cudaError_t err = cudaSuccess;
-  const char* what = "";
+  std::mutex mu;
+  bool ready = false;                // set only once the set-up below succeeded
   unsigned char* scratch = nullptr;  // device address of g_noalloc_scratch on this device
 };
 NoAllocDevice g_noalloc_dev[kNoAllocMaxDevices];
@@ -1052,29 +1148,28 @@ __global__ void noalloc_dbias_finish_kernel(const float* __restrict__ partials, 
   dbias[n] = s;
 }
 
+// Once per device, with that device current: the scratch array's device
+// address and the kernels' shared-memory limit. A failed attempt (for
+// instance one made during a stream capture) leaves the device not ready, so
+// the next call tries again.
 int noalloc_setup(int dev, NoAllocDevice*& out) {
   if (dev < 0 || dev >= kNoAllocMaxDevices) return fail(GEMM_EPI_ERR_UNSUPPORTED, "device index %d out of range", dev);
   NoAllocDevice& d = g_noalloc_dev[dev];
-  std::call_once(d.once, [&d] {
+  std::lock_guard<std::mutex> g(d.mu);
+  if (!d.ready) {
     void* p = nullptr;
-    d.err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (d.err != cudaSuccess) {
-      d.what = "cudaGetSymbolAddress(scratch)";
-      return;
-    }
-    d.scratch = static_cast<unsigned char*>(p);
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
     for (int bn : {64, 128, 256}) {
       for (bool bf16 : {false, true}) {
         TileCfg c = tile_cfg(bn, ge::EPI_DRELU_BGRAD, bf16, false);
-        d.err = cudaFuncSetAttribute(c.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)c.smem);
-        if (d.err != cudaSuccess) {
-          d.what = "cudaFuncSetAttribute(max dynamic shared memory)";
-          return;
-        }
+        e = cudaFuncSetAttribute(c.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)c.smem);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(max dynamic shared memory)");
       }
     }
-  });
-  if (d.err != cudaSuccess) return cuda_fail(d.err, d.what);
+    d.scratch = static_cast<unsigned char*>(p);
+    d.ready = true;
+  }
   out = &d;
   return GEMM_EPI_OK;
 }
@@ -1138,12 +1233,16 @@ extern "C" int drelu_bgrad_execute_noalloc(int64_t T, int64_t N, int64_t K, gemm
   k.k_blocks = ceil_div(K, ge::kBK);
   k.num_tiles = k.m_tiles * k.n_tiles;
   k.aux_words = ceil_div(N, 32);
-  k.group_m = choose_group_m(T, K, ge::kBM);
+  const Raster raster = choose_raster(T, N, K, ge::kBM, bn);
+  k.group_m = raster.group;
+  k.raster_n = raster.by_n;
   k.out = dZ;
   k.aux_in = aux;
   k.partials = partials;
   k.status = status;
-  k.timeout_ns = 2000000000ull;
+  const WatchdogEnv wd = watchdog_env();  // the same limit (and test hook) as a plan's
+  k.timeout_ns = wd.timeout_ns;
+  k.inject_stall = wd.inject_stall;
   const int grid = k.num_tiles < sms ? k.num_tiles : sms;
 
   // the status word must start each call at zero; the partials are fully

@@ -32,7 +32,7 @@ struct SkinnyParams {
   int32_t prefetch;                // k-blocks of W prefetched into L2 ahead of the ring (0 = none)
   const void* bias;
   void* out;                       // Y or dZ, T x N
-  uint32_t* aux_out;
+  uint32_t* aux_out;               // RELU_AUX_BIAS mask words; GELU_AUX_BIAS: T x N 16-bit Z
   const uint32_t* aux_in;
   float* dbias;
   float* partials;                 // [n_tiles][max_segs][TP][128] fp32
@@ -42,6 +42,7 @@ struct SkinnyParams {
   int32_t bias_f32;                // the bias is N fp32 values (else the 16-bit type)
   int32_t out_f32;                 // the output is fp32 (else the 16-bit type)
   int32_t cache_hints;             // W streamed once: evict_first; X read by every CTA: evict_last
+  int32_t inject_stall;            // fault injection for tests: withhold the first segment's tfull commit
 };
 
 // A stage holds KPS consecutive 64-deep k-blocks: W as one box of 64 features
@@ -164,7 +165,10 @@ __device__ __forceinline__ void skinny_finish16(const SkinnyParams& p, float (&v
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       float z = v[j] + bias_n;
-      if constexpr (EPI == EPI_GELU_BIAS) z = gelu_erf(z);
+      const int t = t0 + j;
+      if constexpr (EPI == EPI_GELU_AUX_BIAS)  // the pre-activation, 16-bit, before GELU
+        if (t < p.T && n_ok) store_16<BF16>(p.aux_out, static_cast<int64_t>(t) * p.N + n, z);
+      if constexpr (AppliesGelu<EPI>::value) z = gelu_erf(z);
       if constexpr (EPI == EPI_RELU_BIAS || EPI == EPI_RELU_AUX_BIAS) {
         const bool pos = z > 0.f;
         if constexpr (EPI == EPI_RELU_AUX_BIAS) {
@@ -173,7 +177,6 @@ __device__ __forceinline__ void skinny_finish16(const SkinnyParams& p, float (&v
         }
         z = pos ? z : 0.f;
       }
-      const int t = t0 + j;
       if (t < p.T && n_ok) store_out<BF16>(p, static_cast<int64_t>(t) * p.N + n, z);
     }
     if constexpr (EPI == EPI_RELU_AUX_BIAS) {
@@ -381,7 +384,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_commit(&empty[st]);
         }
         if (!ok) break;
-        umma_commit(&tfull[buf]);
+        // (fault injection: the epilogue then waits on a barrier nothing arrives on)
+        if (!(p.inject_stall && scount == 1)) umma_commit(&tfull[buf]);
       }
       umma_commit(drain);
       wait_bounded(drain, 0, wp, abort_flag, 5, /*honour_abort=*/false);

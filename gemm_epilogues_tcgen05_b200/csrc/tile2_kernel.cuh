@@ -24,6 +24,18 @@
 // Tail split: when the tiles left for the last round fill at most half of
 // the pairs, each of them is processed as two 128-column halves (MMA N =
 // 128), so the last round takes half a tile's time instead of a whole one.
+//
+// Stream-K (SPLIT): with fewer tiles than pairs (the few-row problems, e.g.
+// 256 rows x 43 column tiles for 74 pairs), the (tile, k-block) space is cut
+// into one contiguous k-range per pair, so every pair streams the same share
+// of W. A tile covered by several pairs has one segment per pair; segment 0
+// (the one that starts at k-block 0) finishes the tile. The others write
+// their fp32 accumulator (each CTA its 128 rows) to a workspace slot and
+// count themselves on the tile's flag; segment 0 waits (bounded) until all
+// are in, adds them to its own in segment order (so the sum is the same on
+// every run) and runs the epilogue. Only segment 0 waits, and it waits only
+// on segments that never wait, and every pair is resident (one CTA per SM),
+// so the waits always end.
 #pragma once
 
 #include "tile_kernel.cuh"
@@ -49,11 +61,18 @@ struct Tile2Smem {
 };
 
 // Work unit u of the pair schedule: a whole tile, or (in the split tail) one
-// column half of a tile.
+// column half of a tile; under stream-K, one k-range of a tile.
 struct PairUnit {
   int mb, nb;
-  int half;  // -1 for a whole tile, else 0 or 1
+  int half;          // -1 for a whole tile, else 0 or 1
+  int kb0, kb1;      // k-blocks [kb0, kb1)
+  int tile, seg, nsegs;  // stream-K: the tile's index, this pair's segment of it, their count
 };
+
+// largest pair whose stream-K range starts at or before k-block x
+__device__ __host__ __forceinline__ int64_t pair_owner(int64_t x, int64_t npairs, int64_t total) {
+  return ((x + 1) * npairs - 1) / total;
+}
 
 struct PairSchedule {
   int num_tiles, full_units, num_units;
@@ -64,7 +83,7 @@ struct PairSchedule {
     full_units = split ? tiles - tail : tiles;
     num_units = split ? tiles + tail : tiles;
   }
-  __device__ __forceinline__ PairUnit unit(int u, int m2_tiles, int n_tiles, int group_m) const {
+  __device__ __forceinline__ PairUnit unit(int u, int m2_tiles, int n_tiles, int group, int by_n) const {
     PairUnit r;
     int t = u;
     r.half = -1;
@@ -72,12 +91,63 @@ struct PairSchedule {
       t = full_units + (u - full_units) / 2;
       r.half = (u - full_units) & 1;
     }
-    tile_coords(t, m2_tiles, n_tiles, group_m, r.mb, r.nb);
+    tile_coords(t, m2_tiles, n_tiles, group, by_n, r.mb, r.nb);
+    r.tile = t;
+    r.seg = 0;
+    r.nsegs = 1;
     return r;
   }
 };
 
-template <int BN, int STAGES, int EPI, bool BF16, bool BK = false>
+// The sequence of units of one pair. Without SPLIT: units pair, pair +
+// npairs, ... of the schedule, each over every k-block. With SPLIT: the
+// pieces of the pair's contiguous range [lo, hi) of the flattened (tile,
+// k-block) space, tile by tile.
+template <bool SPLIT>
+struct PairWork {
+  PairSchedule sched;
+  int pair, npairs, m2_tiles, n_tiles, group, by_n, k_blocks;
+  int64_t total, hi, cur;
+  __device__ __forceinline__ PairWork(const TileParams& p, int pair_, int npairs_, int m2)
+      : sched(m2 * p.n_tiles, npairs_, !SPLIT && p.tail_split != 0),
+        pair(pair_), npairs(npairs_), m2_tiles(m2), n_tiles(p.n_tiles), group(p.group_m), by_n(p.raster_n),
+        k_blocks(p.k_blocks) {
+    total = static_cast<int64_t>(m2) * p.n_tiles * p.k_blocks;
+    if constexpr (SPLIT) {
+      cur = static_cast<int64_t>(pair) * total / npairs;
+      hi = static_cast<int64_t>(pair + 1) * total / npairs;
+    } else {
+      cur = pair;
+      hi = sched.num_units;
+    }
+  }
+  __device__ __forceinline__ bool next(PairUnit& w) {
+    if (cur >= hi) return false;
+    if constexpr (SPLIT) {
+      const int t = static_cast<int>(cur / k_blocks);
+      const int64_t tb = static_cast<int64_t>(t) * k_blocks;
+      const int64_t end = hi < tb + k_blocks ? hi : tb + k_blocks;
+      w.mb = t % m2_tiles;
+      w.nb = t / m2_tiles;
+      w.half = -1;
+      w.kb0 = static_cast<int>(cur - tb);
+      w.kb1 = static_cast<int>(end - tb);
+      w.tile = t;
+      const int64_t first = pair_owner(tb, npairs, total);
+      w.nsegs = static_cast<int>(pair_owner(tb + k_blocks - 1, npairs, total) - first + 1);
+      w.seg = static_cast<int>(pair - first);
+      cur = end;
+    } else {
+      w = sched.unit(static_cast<int>(cur), m2_tiles, n_tiles, group, by_n);
+      w.kb0 = 0;
+      w.kb1 = k_blocks;
+      cur += npairs;
+    }
+    return true;
+  }
+};
+
+template <int BN, int STAGES, int EPI, bool BF16, bool BK = false, bool SPLIT = false>
 __global__ void __launch_bounds__(kThreads, 1)
     tile2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmAux,
@@ -110,6 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* stg_s = smem + L::OFF_STG;                             // [4 warps][2][2 KB]
   uint8_t* auxstg_s = smem + L::OFF_AUXSTG;                       // [4 warps][1 KB]
   volatile int* dflag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 8);
+  volatile int* sflag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 12);  // stream-K wait result
 
   const uint32_t warp = threadIdx.x >> 5;
   const uint32_t lane = lane_id();
@@ -145,7 +216,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   const int m2_tiles = (p.m_tiles + 1) / 2;  // 256-row tiles
   // half units would need a 64-row box of a K-major W: with BK every unit is a whole tile
-  const PairSchedule sched(m2_tiles * p.n_tiles, npairs, p.tail_split != 0 && !BK);
+  TileParams pw = p;
+  if constexpr (BK) pw.tail_split = 0;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -153,13 +225,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t it = 0;
       bool ok = true;
       const uint32_t full0 = mapa_shared(smem_u32(&full[0]), 0);
-      for (int u = pair; ok && u < sched.num_units; u += npairs) {
-        const PairUnit w = sched.unit(u, m2_tiles, p.n_tiles, p.group_m);
+      PairWork<SPLIT> work(pw, pair, npairs, m2_tiles);
+      PairUnit w;
+      while (ok && work.next(w)) {
         const int m0 = w.mb * 2 * kBM + static_cast<int>(rank) * kBM;
         // this CTA's columns: half of the tile (two 64-wide chunks), or half of a half (one chunk)
         const int nchunks = w.half < 0 ? BN / 128 : 1;
         const int nh0 = w.nb * BN + (w.half < 0 ? 0 : w.half * (BN / 2)) + static_cast<int>(rank) * nchunks * 64;
-        for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+        for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
           const uint32_t s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
           if (!wait_bounded(&empty[s], ph ^ 1u, p, abort_flag, 1)) {
@@ -194,15 +267,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (rank == 0) {
         uint32_t it = 0, tcount = 0;
         bool ok = true;
-        for (int u = pair; ok && u < sched.num_units; u += npairs, ++tcount) {
-          const PairUnit w = sched.unit(u, m2_tiles, p.n_tiles, p.group_m);
+        PairWork<SPLIT> work(pw, pair, npairs, m2_tiles);
+        PairUnit w;
+        for (; ok && work.next(w); ++tcount) {
           const uint32_t idesc = BK ? IDESC_BK : w.half < 0 ? IDESC : IDESC_HALF;
           const uint32_t buf = tcount & 1u;
           const uint32_t tph = (tcount >> 1) & 1u;
           if (!wait_bounded(&tempty[buf], tph ^ 1u, p, abort_flag, 3)) break;
           tc_fence_after();
           const uint32_t d_tmem = tmem_base + buf * BN;
-          for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+          for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
             const uint32_t s = it % STAGES;
             const uint32_t ph = (it / STAGES) & 1u;
             if (!wait_bounded(&full[s], ph, p, abort_flag, 4)) {
@@ -216,12 +290,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kk = 0; kk < kBK / 16; ++kk) {
               const uint64_t adesc = a_desc<A_MN>(a0, kk);
               const uint64_t bdesc = b_desc(b0, kk, BK, L::B_CHUNK);
-              umma_f16_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+              umma_f16_pair(d_tmem, adesc, bdesc, idesc, (kb > w.kb0 || kk != 0) ? 1u : 0u);
             }
             umma_commit_pair(&empty[s], BOTH);
           }
           if (!ok) break;
-          umma_commit_pair(&tfull[buf], BOTH);
+          // (fault injection: both CTAs' epilogues then wait on a barrier nothing arrives on)
+          if (!(p.inject_stall && tcount == 0)) umma_commit_pair(&tfull[buf], BOTH);
         }
         umma_commit_pair(drain, BOTH);
       }
@@ -238,8 +313,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t tcount = 0;
     bool ok = true;
     const uint32_t tempty0 = mapa_shared(smem_u32(&tempty[0]), 0);
-    for (int u = pair; u < sched.num_units; u += npairs, ++tcount) {
-      const PairUnit w = sched.unit(u, m2_tiles, p.n_tiles, p.group_m);
+    PairWork<SPLIT> work(pw, pair, npairs, m2_tiles);
+    PairUnit w;
+    for (; work.next(w); ++tcount) {
       const int prow = w.mb * 2 + static_cast<int>(rank);  // this CTA's 128-row block
       const int m0 = prow * kBM;
       const int n0 = w.nb * BN + (w.half < 0 ? 0 : w.half * (BN / 2));
@@ -254,11 +330,67 @@ __global__ void __launch_bounds__(kThreads, 1)
       named_bar_sync(1, 128);
       if (ok) ok = wait_bounded(&tfull[buf], tph, p, abort_flag, 6);
       ok = __all_sync(0xffffffffu, ok);
+      const uint32_t trow = tmem_base + ((ew * 32u) << 16) + buf * BN;
+      const int r = static_cast<int>(ew * 32 + lane);  // this thread's row of the CTA's 128
+      // stream-K slots of this tile and CTA: segment s >= 1 at slot (s - 1)
+      const int64_t slot_stride = 2 * kBM * BN;
+      float* slot0 = SPLIT ? p.sk_slots + (static_cast<int64_t>(w.tile) * (p.sk_max_segs - 1) * 2 + rank) * (kBM * BN)
+                           : nullptr;
+      int* flag = SPLIT ? p.sk_flags + w.tile * 2 + rank : nullptr;
+      if (SPLIT && w.seg > 0) {
+        // a later segment: hand the fp32 accumulator to segment 0 and count it in
+        if (ok) {
+          tc_fence_after();
+          float* dst = slot0 + (w.seg - 1) * slot_stride + r * BN;
+#pragma unroll 1
+          for (int c = 0; c < BN / 32; ++c) {
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(trow + c * 32, v);
+            tmem_wait_ld();
+            float4* q = reinterpret_cast<float4*>(dst + c * 32);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              __stcg(q + i, make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                        __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3])));
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(tempty0 + buf * 8);
+        }
+        __threadfence();
+        named_bar_sync(1, 128);
+        if (et == 0 && ok) atomicAdd(flag, 1);
+        continue;
+      }
+      int nadd = 0;
+      if (SPLIT && w.nsegs > 1) {
+        // segment 0: wait until the other segments' partials are in (bounded)
+        if (et == 0) {
+          int got = ok ? 1 : 0;
+          if (got) {
+            const uint64_t t0 = globaltimer_ns();
+            while (*reinterpret_cast<volatile int*>(flag) < w.nsegs - 1) {
+              __nanosleep(100);
+              if (*abort_flag || globaltimer_ns() - t0 > p.timeout_ns) {
+                report_timeout(p.status, abort_flag, 7);
+                got = 0;
+                break;
+              }
+            }
+            if (got) *flag = 0;  // ready for the next launch
+          }
+          __threadfence();
+          *sflag = got;
+        }
+        named_bar_sync(1, 128);
+        ok = ok && *sflag != 0;
+        nadd = w.nsegs - 1;
+      }
       if (ok) {
         tc_fence_after();
-        epi_rows<BN, EPI, BF16>(p, tmem_base + ((ew * 32u) << 16) + buf * BN, m0 + static_cast<int>(ew * 32 + lane), n0,
-                                bs, cp + ew * BN, &tmY, stg, scount, m0 + static_cast<int>(ew * 32), &tmAux,
-                                auxstg_s + ew * kAuxStageBytesPerWarp, mw, ncols, w.half < 0);
+        epi_rows<BN, EPI, BF16>(p, trow, m0 + r, n0, bs, cp + ew * BN, &tmY, stg, scount, m0 + static_cast<int>(ew * 32),
+                                &tmAux, auxstg_s + ew * kAuxStageBytesPerWarp, mw, ncols, w.half < 0,
+                                SPLIT ? slot0 + r * BN : nullptr, nadd, slot_stride);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(tempty0 + buf * 8);

@@ -26,8 +26,8 @@
 
 namespace ge {
 
-// The first six match gemm_epi_epilog; EPI_STORE (plain store of X.W) is the
-// unfused ablation's GEMM.
+// The values match gemm_epi_epilog; EPI_STORE (plain store of X.W) is the
+// public NONE and the unfused ablation's GEMM.
 enum EpiKind : int {
   EPI_BIAS = 0,
   EPI_RELU_BIAS = 1,
@@ -35,7 +35,14 @@ enum EpiKind : int {
   EPI_DRELU_BGRAD = 3,
   EPI_GELU_BIAS = 4,
   EPI_WGRAD = 5,
-  EPI_STORE = 6
+  EPI_STORE = 6,
+  EPI_GELU_AUX_BIAS = 7  // GELU_BIAS, and the pre-activation Z stored (16-bit) as the auxiliary output
+};
+
+// Epilogs that apply GELU.
+template <int EPI>
+struct AppliesGelu {
+  static constexpr bool value = EPI == EPI_GELU_BIAS || EPI == EPI_GELU_AUX_BIAS;
 };
 
 // The weight gradient dW = X^T dZ reads its A operand (X^T, M = the features
@@ -77,7 +84,8 @@ __device__ __forceinline__ uint64_t a_desc(uint32_t a0, int kk) {
 template <int EPI>
 struct AddsBias {
   static constexpr bool value =
-      EPI == EPI_BIAS || EPI == EPI_RELU_BIAS || EPI == EPI_RELU_AUX_BIAS || EPI == EPI_GELU_BIAS;
+      EPI == EPI_BIAS || EPI == EPI_RELU_BIAS || EPI == EPI_RELU_AUX_BIAS || EPI == EPI_GELU_BIAS ||
+      EPI == EPI_GELU_AUX_BIAS;
 };
 
 // GELU(z) = z * Phi(z), Phi the standard normal CDF, through CUDA's erff.
@@ -87,21 +95,28 @@ struct TileParams {
   int32_t T, N, K;
   int32_t m_tiles, n_tiles, k_blocks, num_tiles;
   int32_t aux_words;        // ceil(N / 32)
-  int32_t group_m;          // row tiles per raster group (see tile_coords)
+  int32_t group_m;          // row (or, with raster_n, column) tiles per raster group (see tile_coords)
   const void* bias;         // N values of the 16-bit type (forward)
   void* out;                // T x N, 16-bit: Y, dZ, or the unfused intermediate
-  uint32_t* aux_out;        // RELU_AUX_BIAS mask words
+  uint32_t* aux_out;        // RELU_AUX_BIAS mask words (GELU_AUX_BIAS: T x N 16-bit Z, stored through tmAux)
   const uint32_t* aux_in;   // DRELU_BGRAD mask words
   float* partials;          // DRELU_BGRAD: m_tiles x N column partial sums
   int* status;              // watchdog report (host-visible)
   uint64_t timeout_ns;
   int32_t inject_stall;     // fault injection for tests: withhold the first tile's tmem_full commit
+                            // (one-CTA kernel: the CTA's first tile; CTA pairs: the leader's first unit)
   int32_t aux_tma;          // RELU_AUX_BIAS: mask words go out by TMA store (see AuxByTma)
   int* col_tickets;         // DRELU_BGRAD: per column block, zero between launches; null = no in-kernel finish
   float* dbias;             // DRELU_BGRAD: written by the tile that takes a column block's last ticket
   int32_t tail_split;       // pair kernel: split the last round's tiles into column halves
   int32_t bias_f32;         // the bias is N fp32 values (else the 16-bit type)
   int32_t out_f32;          // the output (Y, dZ or dW) is fp32 (else the 16-bit type)
+  int32_t raster_n;         // tile order by column groups (see tile_coords)
+  // CTA-pair stream-K (few tiles): the k-blocks of all tiles are cut into one
+  // contiguous range per pair; a tile's later segments leave fp32 partials
+  float* sk_slots;          // [tiles][max_segs - 1][2 ranks][128 rows][256 cols]
+  int* sk_flags;            // [tiles][2 ranks] segments written, zero between launches
+  int32_t sk_max_segs;
 };
 
 constexpr int kBM = 128;
@@ -131,21 +146,28 @@ struct TileSmem {
   static constexpr uint32_t BYTES = END + 1024;               // + alignment slack
 };
 
-// Tile order: groups of `group_m` row tiles; inside a group the row tile
-// varies fastest, then the column tile. Consecutive CTAs therefore share
-// W's column block and the group's rows of X stay in L2 while the group
-// sweeps all column blocks.
-__device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, int group_m, int& mb, int& nb) {
-  const int per_group = group_m * n_tiles;
+// Tile order (raster). By rows (by_n = 0): groups of `group` row tiles;
+// inside a group the row tile varies fastest, then the column tile, so
+// consecutive CTAs share W's column block and the group's rows of X stay in
+// L2 while the group sweeps every column block. By columns (by_n = 1): the
+// same with the roles swapped -- groups of `group` column tiles whose block
+// of W stays in L2 while the group sweeps every row tile of X; the better
+// order when X is much larger than W.
+__device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, int group, int by_n, int& mb,
+                                            int& nb) {
+  const int outer = by_n ? n_tiles : m_tiles;  // the dimension that is grouped
+  const int inner = by_n ? m_tiles : n_tiles;
+  const int per_group = group * inner;
   const int g = tile / per_group;
-  const int first_m = g * group_m;
-  const int gsize = min(m_tiles - first_m, group_m);
+  const int first = g * group;
+  const int gsize = min(outer - first, group);
   const int r = tile - g * per_group;
-  mb = first_m + r % gsize;
-  nb = r / gsize;
+  const int a = first + r % gsize, b = r / gsize;
+  mb = by_n ? b : a;
+  nb = by_n ? a : b;
 }
 
-__device__ __noinline__ void report_timeout(int* status, volatile int* abort_flag, int site) {
+static __device__ __noinline__ void report_timeout(int* status, volatile int* abort_flag, int site) {
   *abort_flag = 1;
   if (status) {
     *reinterpret_cast<volatile int*>(status) = 0x7100 | site;
@@ -261,11 +283,44 @@ __device__ __forceinline__ MaskWords<BN> load_mask_words(const TileParams& p, in
   return m;
 }
 
+// Stage a warp's 32 x 32 block of 16-bit values (row = lane, 64 bytes) with
+// the 64-byte swizzle -- 16-byte chunk q of row r at chunk q ^ ((r >> 1) & 3)
+// -- so the 16-byte shared stores are conflict-free, then one lane writes the
+// block with a TMA store at column x, row y (rows and columns past the
+// tensor's extent are clipped by the tensor map). The buffer used two blocks
+// ago must have been read by its store before it is overwritten.
+template <bool BF16>
+__device__ __forceinline__ void store_block16(const float (&v)[32], const CUtensorMap* map, uint8_t* stg,
+                                              uint32_t& scount, int x, int y) {
+  const uint32_t lane = lane_id();
+  uint8_t* buf = stg + (scount & 1u) * 2048;
+  if (lane == 0) bulk_wait_group_read<1>();
+  __syncwarp();
+  const uint32_t rbase = smem_u32(buf) + lane * 64;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 w;
+    w.x = pack2<BF16>(v[8 * q + 0], v[8 * q + 1]);
+    w.y = pack2<BF16>(v[8 * q + 2], v[8 * q + 3]);
+    w.z = pack2<BF16>(v[8 * q + 4], v[8 * q + 5]);
+    w.w = pack2<BF16>(v[8 * q + 6], v[8 * q + 7]);
+    st_shared_v4(rbase + ((q ^ ((lane >> 1) & 3u)) * 16), w);
+  }
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(map, buf, x, y);
+    bulk_commit_group();
+  }
+  ++scount;
+}
+
 template <int BN, int EPI, bool BF16>
 __device__ __forceinline__ void epi_rows(const TileParams& p, uint32_t tbase, int row, int n0, const float* bs,
                                          float* cpw, const CUtensorMap* tmY, uint8_t* stg, uint32_t& scount,
                                          int wrow0, const CUtensorMap* tmAux, uint8_t* auxstg,
-                                         const MaskWords<BN>& mw, int ncols = BN, bool aux_block = true) {
+                                         const MaskWords<BN>& mw, int ncols = BN, bool aux_block = true,
+                                         const float* addp = nullptr, int nadd = 0, int64_t add_stride = 0) {
   const uint32_t lane = lane_id();
   const bool row_ok = row < p.T;
   constexpr bool kAuxTma = EPI == EPI_RELU_AUX_BIAS && AuxByTma<BN>::value;
@@ -285,6 +340,19 @@ __device__ __forceinline__ void epi_rows(const TileParams& p, uint32_t tbase, in
     float v[32];
 #pragma unroll
     for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+    // stream-K: this thread's row of the other k-segments' fp32 partial
+    // accumulators (written by other CTA pairs), added in segment order
+    for (int sg = 0; sg < nadd; ++sg) {
+      const float4* q = reinterpret_cast<const float4*>(addp + sg * add_stride + c * 32);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float4 x = __ldcg(q + i);
+        v[4 * i] += x.x;
+        v[4 * i + 1] += x.y;
+        v[4 * i + 2] += x.z;
+        v[4 * i + 3] += x.w;
+      }
+    }
     if constexpr (EPI == EPI_DRELU_BGRAD) {
       const uint32_t m = mw.w[c];
 #pragma unroll
@@ -292,7 +360,9 @@ __device__ __forceinline__ void epi_rows(const TileParams& p, uint32_t tbase, in
     } else if constexpr (!PlainStore<EPI>::value) {
 #pragma unroll
       for (int j = 0; j < 32; ++j) v[j] += bs[c * 32 + j];
-      if constexpr (EPI == EPI_GELU_BIAS) {
+      // GELU_AUX_BIAS: the pre-activation Z goes out (16-bit) before GELU
+      if constexpr (EPI == EPI_GELU_AUX_BIAS) store_block16<BF16>(v, tmAux, stg, scount, nc0, wrow0);
+      if constexpr (AppliesGelu<EPI>::value) {
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = gelu_erf(v[j]);
       }
@@ -339,32 +409,7 @@ __device__ __forceinline__ void epi_rows(const TileParams& p, uint32_t tbase, in
         ++scount;
       }
     } else {
-      // Stage this warp's 32 x 32 block (row = lane, 64 bytes) with the
-      // 64-byte swizzle -- 16-byte chunk q of row r at chunk q ^ ((r >> 1) & 3)
-      // -- so the 16-byte shared stores are conflict-free, then one lane
-      // writes the block with a TMA store (rows and columns past T and N are
-      // clipped by the tensor map). The buffer used two blocks ago must have
-      // been read by its store before it is overwritten.
-      uint8_t* buf = stg + (scount & 1u) * 2048;
-      if (lane == 0) bulk_wait_group_read<1>();
-      __syncwarp();
-      const uint32_t rbase = smem_u32(buf) + lane * 64;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint4 w;
-        w.x = pack2<BF16>(v[8 * q + 0], v[8 * q + 1]);
-        w.y = pack2<BF16>(v[8 * q + 2], v[8 * q + 3]);
-        w.z = pack2<BF16>(v[8 * q + 4], v[8 * q + 5]);
-        w.w = pack2<BF16>(v[8 * q + 6], v[8 * q + 7]);
-        st_shared_v4(rbase + ((q ^ ((lane >> 1) & 3u)) * 16), w);
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        tma_store_2d(tmY, buf, nc0, wrow0);
-        bulk_commit_group();
-      }
-      ++scount;
+      store_block16<BF16>(v, tmY, stg, scount, nc0, wrow0);
     }
     if constexpr (EPI == EPI_DRELU_BGRAD) {
       warp_transpose_reduce32(v);
@@ -502,7 +547,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
         int mb, nb;
-        tile_coords(tile, p.m_tiles, p.n_tiles, p.group_m, mb, nb);
+        tile_coords(tile, p.m_tiles, p.n_tiles, p.group_m, p.raster_n, mb, nb);
         const int m0 = mb * kBM, n0 = nb * BN;
         for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
           const uint32_t s = it % STAGES;
@@ -582,7 +627,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tcount) {
       int mb, nb;
-      tile_coords(tile, p.m_tiles, p.n_tiles, p.group_m, mb, nb);
+      tile_coords(tile, p.m_tiles, p.n_tiles, p.group_m, p.raster_n, mb, nb);
       const int m0 = mb * kBM, n0 = nb * BN;
       const uint32_t buf = tcount & 1u;
       const uint32_t tph = (tcount >> 1) & 1u;

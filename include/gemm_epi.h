@@ -36,6 +36,21 @@
  * Errors: functions return GEMM_EPI_OK (0) or a negative code; a message is
  * kept per thread and read with gemm_epi_last_error(). Argument errors are
  * detected before anything is launched.
+ *
+ * Environment variables, read when a plan is created (and by every call of
+ * drelu_bgrad_execute_noalloc); none is needed in normal use:
+ *   GEMM_EPI_WAIT_TIMEOUT_MS      limit of each bounded wait inside a kernel
+ *                                 (default 2000 ms; see GEMM_EPI_ERR_TIMEOUT)
+ *   tuning overrides of the plan's choices, for measurement and tests:
+ *   GEMM_EPI_FORCE_KERNEL=tile|pair|skinny, GEMM_EPI_FORCE_BN=64|128|256,
+ *   GEMM_EPI_RASTER=m|n, GEMM_EPI_GROUP_M, GEMM_EPI_SKINNY_GRID, GEMM_EPI_SKINNY_KPS=1|2,
+ *   GEMM_EPI_SKINNY_PREFETCH, GEMM_EPI_TAIL_SPLIT=0|1, GEMM_EPI_CACHE_HINTS=0|1
+ *   fault injection for the library's own tests, honoured only while
+ *   GEMM_EPI_TEST_HOOKS=1 is also set: GEMM_EPI_INJECT_STALL (a kernel
+ *   withholds its first tile's completion signal, so its watchdog fires),
+ *   GEMM_EPI_INJECT_ENCODE_FAILURE (every tensor-map encode fails),
+ *   GEMM_EPI_INJECT_PLAN_ALLOC_FAILURE (the DRELU_BGRAD workspace
+ *   allocation fails).
  */
 #ifndef GEMM_EPI_H
 #define GEMM_EPI_H
@@ -72,8 +87,16 @@ typedef enum {
   GEMM_EPI_DRELU_BGRAD = 3,   /* dZ = (dY2.W2) masked by aux, dbias = sum_t dZ */
   GEMM_EPI_GELU_BIAS = 4,     /* Y = gelu(X.W + bias); aux is ignored         */
   GEMM_EPI_WGRAD = 5,         /* dW = X^T . dZ, see gemm_epi_wgrad_execute    */
-  GEMM_EPI_NONE = 6           /* Y = X.W, no bias (may be NULL) or activation */
+  GEMM_EPI_NONE = 6,          /* Y = X.W, no bias (may be NULL) or activation */
+  GEMM_EPI_GELU_AUX_BIAS = 7  /* Y = gelu(Z), aux = Z = X.W + bias (16-bit)   */
 } gemm_epi_epilog;
+
+/* GELU_AUX_BIAS is to GELU_BIAS what RELU_AUX_BIAS is to RELU_BIAS: it also
+ * returns what the backward pass of the activation needs. The pages define
+ * that auxiliary output only for ReLU (the mask); GELU's derivative depends
+ * on the pre-activation itself, not only on its sign, so this library
+ * returns Z = X.W + bias, rounded to the plan's 16-bit type (round to
+ * nearest even), T x N row-major in the aux buffer. */
 
 enum {
   GEMM_EPI_OK = 0,
@@ -141,13 +164,15 @@ GEMM_EPI_API gemm_epi_plan_t gemm_epi_plan_ex(int64_t T, int64_t N, int64_t K, g
 
 /*
  * gemm_epi_execute: the forward epilogs (BIAS, RELU_BIAS, RELU_AUX_BIAS,
- * GELU_BIAS) and the plain product (NONE).
+ * GELU_BIAS, GELU_AUX_BIAS) and the plain product (NONE).
  *   X, W, Y: device pointers, 16-byte aligned (W is K x N, or N x K with
  *   GEMM_EPI_FLAG_W_NK; Y is fp32 with GEMM_EPI_FLAG_OUT_F32). bias: device
  *   pointer, 2-byte aligned (4-byte for an fp32 bias, gemm_epi_set_bias_f32),
  *   never NULL except for NONE, where it is ignored. aux: device pointer,
- *   4-byte aligned, required for RELU_AUX_BIAS and ignored (may be NULL)
- *   otherwise.
+ *   required for RELU_AUX_BIAS (the mask words, 4-byte aligned) and for
+ *   GELU_AUX_BIAS (T x N values of the plan's 16-bit type even with
+ *   GEMM_EPI_FLAG_OUT_F32, 16-byte aligned; pass it cast to uint32_t*), and
+ *   ignored (may be NULL) otherwise.
  * Returns GEMM_EPI_OK once the work is enqueued on `stream`;
  * GEMM_EPI_ERR_EPILOG_MISMATCH on a DRELU_BGRAD or WGRAD plan or a missing
  * aux; GEMM_EPI_ERR_MISALIGNED for a misaligned pointer; GEMM_EPI_ERR_CUDA if
@@ -227,8 +252,10 @@ GEMM_EPI_API int gemm_epi_status(gemm_epi_plan_t plan);
  * reads that and writes the output).
  *   gemm_epi_unfused_execute: GEMM -> T1 (T x N, dtype), T1 + bias -> T2,
  *   relu(T2) -> Y (and, for RELU_AUX_BIAS, the mask from T2 > 0 -> aux), or
- *   gelu(T2) -> Y for GELU_BIAS. For BIAS the activation kernel is skipped
- *   and T2 is the output: pass Y as T2.
+ *   gelu(T2) -> Y for GELU_BIAS. For GELU_AUX_BIAS the bias kernel writes
+ *   into aux (the auxiliary output Z; T2 is ignored and may be NULL), and
+ *   gelu(aux) -> Y. For BIAS the activation kernel is skipped and T2 is the
+ *   output: pass Y as T2.
  *   drelu_bgrad_unfused_execute: GEMM -> G (dtype), mask apply -> dZ,
  *   column sum of dZ -> dbias (fixed order).
  * T1, T2, G: caller-owned device scratch of T x N dtype, 16-byte aligned.
@@ -276,10 +303,14 @@ GEMM_EPI_API int drelu_bgrad_unfused_execute(gemm_epi_plan_t plan, const void* d
  * DRELU_BGRAD; the pointers, alignment and layouts as drelu_bgrad_execute.
  * First call on a device: it looks up the scratch array's device address
  * and sets the kernel's shared-memory limit for that device, once; make
- * that first call before any stream capture begins. Each call clears the
- * status block, then launches two kernels on `stream` and returns without
- * synchronising. If a kernel wait expires (the watchdog), every dbias entry
- * is written as NaN instead of a sum.
+ * that first call before any stream capture begins (a set-up that fails is
+ * tried again by the next call). Each call clears the status block, then
+ * launches two kernels on `stream` and returns without synchronising. The
+ * product always runs on the one-CTA tile kernel: at few-row shapes
+ * (T <= 256), where a plan picks the few-row kernel, this entry point is
+ * slower than drelu_bgrad_execute. Its waits are bounded like a plan's
+ * (GEMM_EPI_WAIT_TIMEOUT_MS); if one expires (the watchdog), every dbias
+ * entry is written as NaN instead of a sum, and dZ may be incomplete.
  */
 GEMM_EPI_API int drelu_bgrad_execute_noalloc(int64_t T, int64_t N, int64_t K, gemm_epi_dtype dtype,
                                              const void* dY2, const void* W2, const uint32_t* aux, void* dZ,

@@ -19,3 +19,18 @@ def oracle_mod():
 
     oracle.build()
     return oracle
+
+
+def pytest_sessionfinish(session, exitstatus):
+    """With GEMM_EPI_DBIAS_LOG=<path>, write the worst dbias error ratios the
+    parity checks saw (against the stated bound and against the full bound)."""
+    path = os.environ.get("GEMM_EPI_DBIAS_LOG")
+    if not path:
+        return
+    mod = sys.modules.get("_parity")
+    if mod is None or not getattr(mod, "DBIAS_RATIOS", None):
+        return
+    import json
+
+    with open(path, "w") as f:
+        json.dump(mod.DBIAS_RATIOS, f, indent=1, sort_keys=True)

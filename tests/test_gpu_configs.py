@@ -13,7 +13,7 @@ import torch
 import oracle
 from gemm_epilogues_tcgen05_b200 import Plan, synth
 
-from _parity import (Y_REL, assert_dbias_is_column_sum, assert_within, check_wgrad, dbias_scale, odt, run_wgrad,
+from _parity import (Y_REL, assert_dbias, assert_dbias_is_column_sum, assert_within, check_wgrad, odt, run_wgrad,
                      unit_roundoff)
 
 pytestmark = pytest.mark.gpu
@@ -102,7 +102,7 @@ def _run(w, full: bool):
     if full:
         rb = oracle.drelu_bgrad(bits(inp["dY2"]), bits(inp["W2"]), aux_np, odt(dt), w.N)
         assert_within(dZ.double().cpu().numpy(), rb["dZ"], rb["S"], Y_REL, f"{w.name} dZ", u)
-        assert_within(dbias.double().cpu().numpy(), rb["dbias"], dbias_scale(rb), 1.0, f"{w.name} dbias")
+        assert_dbias(dbias.double().cpu().numpy(), rb, w.D2, f"{w.name} (full size, every column)")
         assert_dbias_is_column_sum(dbias.cpu(), dZ.cpu(), dt)
     else:
         rr = oracle.drelu_bgrad(bits(inp["dY2"]), bits(inp["W2"]), aux_np, odt(dt), w.N, rows=rows)
@@ -110,7 +110,7 @@ def _run(w, full: bool):
         rc = oracle.drelu_bgrad(bits(inp["dY2"]), bits(inp["W2"]), aux_np, odt(dt), w.N, cols=cols)
         assert_within(take(dZ, None, cols).double().cpu().numpy(), rc["dZ"], rc["S"], Y_REL, f"{w.name} dZ cols", u)
         ci = torch.tensor(cols, device=dev)
-        assert_within(dbias[ci].double().cpu().numpy(), rc["dbias"], dbias_scale(rc), 1.0, f"{w.name} dbias")
+        assert_dbias(dbias[ci].double().cpu().numpy(), rc, w.D2, f"{w.name} (full size, {len(cols)} sampled columns)")
         assert_dbias_is_column_sum(dbias[ci].cpu(), dZ[:, ci].cpu(), dt)
 
 

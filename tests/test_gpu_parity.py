@@ -19,7 +19,7 @@ SHAPES = [(1, 8, 8), (5, 40, 24), (130, 72, 136), (200, 264, 200), (257, 520, 32
 # few-row shapes whose feature tiles are split over several CTAs (stream-K
 # segments), with ragged K and N, and one where every CTA owns whole tiles
 SKINNY_SHAPES = [(16, 1032, 2048), (100, 264, 1000), (256, 4104, 520), (40, 2056, 64), (1, 11008, 4096)]
-FWD_EPILOGS = ["BIAS", "RELU_BIAS", "RELU_AUX_BIAS", "GELU_BIAS"]
+FWD_EPILOGS = ["BIAS", "RELU_BIAS", "RELU_AUX_BIAS", "GELU_BIAS", "GELU_AUX_BIAS"]
 # CTA-pair shapes: T not a multiple of 256 (the peer CTA's rows partly or
 # wholly past T), N not a multiple of 256 (the peer's columns past N)
 PAIR_SHAPES = [(300, 264, 136), (600, 520, 328), (1000, 1032, 264), (257, 8, 64), (600, 1024, 328),
@@ -120,6 +120,70 @@ def test_skinny_split_tiles(monkeypatch, T, N, K, dtype):
         assert gpu["info"]["kernel"] == 1
         check_backward(inp, fwd["aux"], DT[dtype], gpu)
     assert torch.equal(outs[0]["dbias"], outs[1]["dbias"])
+
+
+@pytest.mark.parametrize("variant", ["tile128", "pair"])
+@pytest.mark.parametrize("raster,group", [("n", 1), ("n", 3), ("m", 2)])
+def test_raster_orders(monkeypatch, variant, raster, group):
+    """Tile order by column groups (W's block held in L2, X streamed) and small
+    row groups: every tile is computed exactly once whatever the order
+    (ragged T and N, more tiles than CTAs, DRELU_BGRAD tickets included)."""
+    _force(monkeypatch, variant)
+    monkeypatch.setenv("GEMM_EPI_RASTER", raster)
+    monkeypatch.setenv("GEMM_EPI_GROUP_M", str(group))
+    T, N, K = 1800, 3000, 72
+    inp = synth.make_shape_inputs(T, N, K, "bf16", seed=61 + group, D2=40)
+    for ep in ("RELU_AUX_BIAS", "GELU_AUX_BIAS"):
+        gpu = run_forward(inp, ep, torch.bfloat16)
+        _expect_variant(gpu["info"], variant, T)
+        check_forward(inp, ep, torch.bfloat16, gpu)
+    fwd = run_forward(inp, "RELU_AUX_BIAS", torch.bfloat16)
+    outs = run_backward(inp, fwd["aux"], torch.bfloat16, repeats=2)
+    for gpu in outs:
+        check_backward(inp, fwd["aux"], torch.bfloat16, gpu)
+    assert torch.equal(outs[0]["dbias"], outs[1]["dbias"])
+
+
+# CTA pairs in stream-K mode (fewer 256 x 256 tiles than pairs, K of at least
+# 16 k-blocks): tiles split over 2 to 9 pairs, ragged T and N, rows of the
+# peer CTA past T
+PAIR_SPLIT_SHAPES = [(300, 520, 2048), (200, 1032, 1024), (1000, 264, 4096), (256, 2056, 1096)]
+
+
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+@pytest.mark.parametrize("T,N,K", PAIR_SPLIT_SHAPES)
+def test_pair_stream_k(monkeypatch, T, N, K, dtype):
+    """Every epilog and DRELU_BGRAD (twice: the segment counters start from
+    zero again) through the CTA-pair kernel's stream-K mode; the unfused GEMM
+    and integer inputs (bit-exact whatever the split) too."""
+    _force(monkeypatch, "pair")
+    inp = synth.make_shape_inputs(T, N, K, dtype, seed=T + 5 * N + K, D2=K)
+    for ep in FWD_EPILOGS:
+        gpu = run_forward(inp, ep, DT[dtype])
+        assert gpu["info"]["kernel"] == 2 and gpu["info"]["split_k"] > 1, gpu["info"]
+        check_forward(inp, ep, DT[dtype], gpu)
+    fwd = run_forward(inp, "RELU_AUX_BIAS", DT[dtype])
+    outs = run_backward(inp, fwd["aux"], DT[dtype], repeats=2)
+    for gpu in outs:
+        assert gpu["info"]["split_k"] > 1
+        check_backward(inp, fwd["aux"], DT[dtype], gpu)
+    assert torch.equal(outs[0]["dbias"], outs[1]["dbias"])
+    assert torch.equal(outs[0]["dZ"].view(torch.int16), outs[1]["dZ"].view(torch.int16))
+    check_forward(inp, "RELU_BIAS", DT[dtype], run_forward(inp, "RELU_BIAS", DT[dtype], unfused=True), stored_xw=True)
+    iinp = synth.make_shape_inputs(T, N, K, dtype, seed=T + N, D2=K, kind="int")
+    check_forward(iinp, "RELU_AUX_BIAS", DT[dtype], run_forward(iinp, "RELU_AUX_BIAS", DT[dtype]), exact=True)
+    ifwd = run_forward(iinp, "RELU_AUX_BIAS", DT[dtype])
+    check_backward(iinp, ifwd["aux"], DT[dtype], run_backward(iinp, ifwd["aux"], DT[dtype]), exact=True)
+
+
+def test_pair_stream_k_can_be_switched_off(monkeypatch):
+    _force(monkeypatch, "pair")
+    monkeypatch.setenv("GEMM_EPI_PAIR_SPLIT", "0")
+    T, N, K = 300, 520, 2048
+    inp = synth.make_shape_inputs(T, N, K, "bf16", seed=5, D2=K)
+    gpu = run_forward(inp, "RELU_AUX_BIAS", torch.bfloat16)
+    assert gpu["info"]["kernel"] == 2 and gpu["info"]["split_k"] == 1
+    check_forward(inp, "RELU_AUX_BIAS", torch.bfloat16, gpu)
 
 
 # k per pipeline stage (64·KPS): K ragged against 128, K below one k-block
@@ -436,6 +500,7 @@ def test_injected_encode_failure_returns_error_without_launch(monkeypatch):
     g = {k: v.cuda() for k, v in inp.items()}
     with binding.Plan(T, N, K, torch.bfloat16, "RELU_BIAS") as plan:
         Y = torch.full((T, N), 7.0, dtype=torch.bfloat16, device="cuda")
+        monkeypatch.setenv("GEMM_EPI_TEST_HOOKS", "1")
         monkeypatch.setenv("GEMM_EPI_INJECT_ENCODE_FAILURE", "1")
         with pytest.raises(binding.GemmEpiError) as e:
             plan.gemm_epi_execute(g["X"], g["W"], g["bias"], Y)
@@ -449,34 +514,49 @@ def test_injected_encode_failure_returns_error_without_launch(monkeypatch):
 
 
 def test_unknown_epilog_values_rejected():
-    for bad in (-1, 7, 99):
+    for bad in (-1, 8, 99):
         with pytest.raises(binding.GemmEpiError):
             binding.gemm_epi_plan(64, 64, 64, binding.F16, bad)
 
 
 def test_injected_workspace_allocation_failure(monkeypatch):
     monkeypatch.setenv("GEMM_EPI_INJECT_PLAN_ALLOC_FAILURE", "1")
+    binding.gemm_epi_free(binding.gemm_epi_plan(256, 256, 256, binding.BF16, binding.DRELU_BGRAD))  # hooks off
+    monkeypatch.setenv("GEMM_EPI_TEST_HOOKS", "1")
     with pytest.raises(binding.GemmEpiError) as e:
         binding.gemm_epi_plan(256, 256, 256, binding.BF16, binding.DRELU_BGRAD)
     assert "injected" in str(e.value)
 
 
+# (kernel variant, T, N, K): the one-CTA kernel (BN = 64), the CTA pair (the
+# peer's epilogue waits on a commit from the leader and both drain through the
+# final cluster barrier; the second shape gives each pair two or three units,
+# so the leader's MMA issuer must give up on a later unit; the third runs in
+# stream-K mode, where a tile's segment 0 waits on the other segments'
+# partials) and the few-row kernel (a tile split into stream-K
+# segments, whose tickets must be reset after the abort)
+WATCHDOG_CASES = [("tile64", 512, 512, 256), ("pair", 512, 512, 256), ("pair", 2048, 5120, 64),
+                  ("pair", 300, 520, 2048), ("skinny", 16, 1032, 2048)]
+
+
+@pytest.mark.parametrize("variant,T,N,K", WATCHDOG_CASES)
 @pytest.mark.parametrize("epilog", ["RELU_AUX_BIAS", "DRELU_BGRAD"])
-def test_watchdog_reports_timeout_and_context_stays_usable(monkeypatch, epilog):
-    """Fault injection without a GPU fault: the MMA warp withholds the first
+def test_watchdog_reports_timeout_and_context_stays_usable(monkeypatch, epilog, variant, T, N, K):
+    """Fault injection without a GPU fault: the MMA issuer withholds the first
     tile's completion signal, the epilogue's bounded wait (200 ms here) runs
-    out, the kernel frees its tensor memory and returns, and the host reads
-    ERR_TIMEOUT. A fresh plan afterwards must compute correctly."""
-    T, N, K = 512, 512, 256
-    monkeypatch.setenv("GEMM_EPI_FORCE_KERNEL", "tile")
-    monkeypatch.setenv("GEMM_EPI_FORCE_BN", "64")
+    out, the kernel drains its copies and MMAs, frees its tensor memory and
+    returns, and the host reads ERR_TIMEOUT. The same plan and a fresh one
+    afterwards must compute correctly."""
+    _force(monkeypatch, variant)
     monkeypatch.setenv("GEMM_EPI_WAIT_TIMEOUT_MS", "200")
     monkeypatch.setenv("GEMM_EPI_INJECT_STALL", "1")
+    monkeypatch.setenv("GEMM_EPI_TEST_HOOKS", "1")
     inp = synth.make_shape_inputs(T, N, K, "bf16", seed=17, D2=K)
     g = {k: v.cuda() for k, v in inp.items()}
     dt = torch.bfloat16
     aux = torch.zeros((T, (N + 31) // 32), dtype=torch.int32, device="cuda")
     with binding.Plan(T, N, K, dt, epilog) as plan:
+        _expect_variant(plan.info(), variant, T)
         if epilog == "DRELU_BGRAD":
             plan.backward(g["dY2"], g["W2"], aux)
         else:
@@ -487,6 +567,18 @@ def test_watchdog_reports_timeout_and_context_stays_usable(monkeypatch, epilog):
         assert plan.status() == binding.OK  # the report is cleared by reading it
     monkeypatch.delenv("GEMM_EPI_INJECT_STALL")
     gpu = run_forward(inp, "RELU_AUX_BIAS", dt)
+    _expect_variant(gpu["info"], variant, T)
     check_forward(inp, "RELU_AUX_BIAS", dt, gpu)
-    out = run_backward(inp, gpu["aux"], dt)
-    check_backward(inp, gpu["aux"], dt, out)
+    outs = run_backward(inp, gpu["aux"], dt, repeats=2)  # split-tile and column tickets start from zero again
+    for out in outs:
+        check_backward(inp, gpu["aux"], dt, out)
+
+
+def test_stall_hook_needs_the_test_switch(monkeypatch):
+    """GEMM_EPI_INJECT_STALL alone (without GEMM_EPI_TEST_HOOKS=1) changes nothing."""
+    _force(monkeypatch, "tile64")
+    monkeypatch.setenv("GEMM_EPI_WAIT_TIMEOUT_MS", "200")
+    monkeypatch.setenv("GEMM_EPI_INJECT_STALL", "1")
+    monkeypatch.delenv("GEMM_EPI_TEST_HOOKS", raising=False)
+    inp = synth.make_shape_inputs(256, 256, 128, "bf16", seed=23)
+    check_forward(inp, "RELU_AUX_BIAS", torch.bfloat16, run_forward(inp, "RELU_AUX_BIAS", torch.bfloat16))
