@@ -78,7 +78,7 @@ def step_spec(w: synth.Workload, args=None):
         return "RELU_AUX_BIAS", True
     if w.name == "square":
         return "RELU_BIAS", False
-    if w.name == "large":
+    if w.name in ("large", "large-proxy"):
         return "RELU_AUX_BIAS", False
     if w.name.startswith("skinny"):
         return "RELU_BIAS", True

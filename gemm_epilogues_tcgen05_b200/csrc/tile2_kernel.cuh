@@ -127,8 +127,7 @@ struct PairWork {
       const int t = static_cast<int>(cur / k_blocks);
       const int64_t tb = static_cast<int64_t>(t) * k_blocks;
       const int64_t end = hi < tb + k_blocks ? hi : tb + k_blocks;
-      w.mb = t % m2_tiles;
-      w.nb = t / m2_tiles;
+      tile_coords(t, m2_tiles, n_tiles, group, by_n, w.mb, w.nb);
       w.half = -1;
       w.kb0 = static_cast<int>(cur - tb);
       w.kb1 = static_cast<int>(end - tb);

@@ -62,6 +62,10 @@ WORKLOADS = {
     "ffn": Workload("ffn", "bf16", 4096, 4096, 11008, 4096, 1.0 / 11008, seed=1236),
     "large": Workload("large", "fp16", 65536, 16384, 8192, seed=1237),
 }
+# a same-K slice of the large shape (8192 of its 65536 rows, ~0.7 GB on the
+# device), small enough for multi-pass profiler captures of the large
+# shape's kernel
+WORKLOADS["large-proxy"] = Workload("large-proxy", "fp16", 8192, 16384, 8192, seed=1237)
 for _t in (1, 8, 64, 256):
     WORKLOADS[f"skinny-{_t}"] = Workload(f"skinny-{_t}", "bf16", _t, 4096, 11008, 4096, 1.0 / 11008,
                                          seed=1238)
