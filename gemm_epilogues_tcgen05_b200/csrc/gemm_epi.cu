@@ -149,7 +149,7 @@ int encode_out_f32(CUtensorMap* map, const void* out, int64_t T, int64_t N) {
 // the words directly.
 bool aux_tma_ok(const void* aux, int64_t N, int bn) {
   const int64_t words = (N + 31) / 32;
-  return bn >= 128 && (words % 4) == 0 && (reinterpret_cast<uintptr_t>(aux) & 15) == 0;
+  return (bn == 128 || bn == 256) && (words % 4) == 0 && (reinterpret_cast<uintptr_t>(aux) & 15) == 0;
 }
 
 int encode_aux(CUtensorMap* map, const void* aux, int64_t T, int64_t N, int bn) {
@@ -226,10 +226,13 @@ int max_resident_pairs(const TileCfg& c, int sms) {
 
 TileCfg tile_cfg(int BN, int epi, bool bf16, bool bk) {
   TileCfg c;
-  c.BN = BN == 256 || BN == 128 ? BN : 64;
+  c.BN = BN == 256 || BN == 192 || BN == 128 ? BN : 64;
   if (c.BN == 256) {
     c.stages = 4;
     c.smem = ge::TileSmem<256, 4>::BYTES;
+  } else if (c.BN == 192) {
+    c.stages = 4;
+    c.smem = ge::TileSmem<192, 4>::BYTES;
   } else if (c.BN == 128) {
     c.stages = 6;
     c.smem = ge::TileSmem<128, 6>::BYTES;
@@ -274,10 +277,10 @@ SkinnyCfg skinny_cfg_tp(int epi, bool bf16, int kps) {
 
 // Two k-blocks per stage (W stages of 32 KB) while X's share of a stage is
 // small: at T = 1 and 8 (N = 11008, K = 4096) 26.7 us against 28.7 us with
-// one; at T = 33..64 the two tie and at T = 128 one k-block per stage (7
-// stages against 3) is faster (35.7 against 38.8 us). Four per stage never
-// beat two.
-int default_kps(int64_t T) { return T <= 32 ? 2 : 1; }
+// one, at T = 64 28.7 against 32.8 us (both directions); at T = 128 one
+// k-block per stage (7 stages against 3) is faster (35.7 against 38.8 us).
+// Four per stage never beat two.
+int default_kps(int64_t T) { return T <= 64 ? 2 : 1; }
 
 SkinnyCfg skinny_cfg(int64_t T, int epi, bool bf16) {
   int kps = default_kps(T);
@@ -591,7 +594,7 @@ int launch_skinny(const gemm_epi_plan_s* p, const ge::SkinnyParams& k, cudaStrea
 int choose_bn(int64_t T, int64_t N, int num_sms) {
   if (const char* f = getenv("GEMM_EPI_FORCE_BN")) {
     int v = atoi(f);
-    if (v == 64 || v == 128 || v == 256) return v;
+    if (v == 64 || v == 128 || v == 192 || v == 256) return v;
   }
   const int64_t m_tiles = (T + ge::kBM - 1) / ge::kBM;
   // widest tile that still gives every SM at least one tile, else the
@@ -713,13 +716,17 @@ gemm_epi_plan_t gemm_epi_plan_ex(int64_t T, int64_t N, int64_t K, gemm_epi_dtype
     // One cluster of two CTAs per 256-row x 256-column tile, up to the number
     // of clusters the device can hold at once (a GPC with an odd number of
     // free SMs cannot place a pair on its last one). With fewer tiles than
-    // that, stream-K: every pair takes an equal share of the tiles' k-blocks
-    // (at least 8), so the idle pairs stream W too.
+    // that, optionally stream-K: every pair takes an equal share of the
+    // tiles' k-blocks (at least 8), so the idle pairs stream W too.
     const int pair_tiles = ceil_div(T, 256) * p->n_tiles;
     const int max_pairs = max_resident_pairs(p->cfg, sms);
     int pairs = pair_tiles < max_pairs ? pair_tiles : max_pairs;
-    bool split = pair_tiles < max_pairs && p->k_blocks >= 16;
-    if (const char* f = getenv("GEMM_EPI_PAIR_SPLIT")) split = split && atoi(f) != 0;  // A/B override
+    // opt-in (GEMM_EPI_PAIR_SPLIT=1): on the shapes measured so far its
+    // fixup (segment 0 reading the other segments' partials back from L2)
+    // costs more than the idle pairs give (T = 256, N = 11008, K = 4096:
+    // 61.4 us against 36.8 us; 1024 x 512 x 2048: 60.0 against 18.4 us)
+    bool split = false;
+    if (const char* f = getenv("GEMM_EPI_PAIR_SPLIT")) split = atoi(f) != 0 && pair_tiles < max_pairs && p->k_blocks >= 16;
     if (split) {
       const int64_t want = (int64_t)pair_tiles * p->k_blocks / 8;
       const int sp = (int)(want < max_pairs ? want : max_pairs);

@@ -29,6 +29,7 @@ TileKernelFn tile_epi(int epi) {
 template <bool BF, bool BK>
 TileKernelFn tile_any(int bn, int epi) {
   if (bn == 256) return tile_epi<256, 4, BF, BK>(epi);
+  if (bn == 192) return tile_epi<192, 4, BF, BK>(epi);
   if (bn == 128) return tile_epi<128, 6, BF, BK>(epi);
   if (bn == 64) return tile_epi<64, 8, BF, BK>(epi);
   return nullptr;

@@ -18,7 +18,7 @@ namespace ge_inst {
 using TileKernelFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, ge::TileParams);
 using SkinnyKernelFn = void (*)(CUtensorMap, CUtensorMap, ge::SkinnyParams);
 
-// One CTA per tile, BN = 64, 128 or 256 columns (8, 6 or 4 stages); `epi` is
+// One CTA per tile, BN = 64, 128, 192 or 256 columns (8, 6, 4 or 4 stages); `epi` is
 // a ge::EpiKind. _mn: the weight is K x N; _nk: N x K (no WGRAD: nullptr).
 TileKernelFn tile_f16_mn(int bn, int epi);
 TileKernelFn tile_f16_nk(int bn, int epi);

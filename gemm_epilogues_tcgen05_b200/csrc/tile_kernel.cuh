@@ -256,11 +256,11 @@ __device__ __forceinline__ void epi_stage_bias(const TileParams& p, int n0, floa
 // epilogue: bias, ReLU, mask word, 16-bit stores; for DRELU_BGRAD the mask
 // select and this warp's column sums into cpw[0..BN).
 // Mask words go out through shared memory and one TMA store per warp and
-// tile when a row's words span at least 16 bytes (BN >= 128); with BN = 64
-// (8 bytes) they are stored directly.
+// tile when a row's words are a multiple of 16 bytes (BN = 128, 256); with
+// BN = 64 or 192 (8 or 24 bytes) they are stored directly.
 template <int BN>
 struct AuxByTma {
-  static constexpr bool value = BN >= 128;
+  static constexpr bool value = BN == 128 || BN == 256;  // a TMA box row must be a multiple of 16 bytes
 };
 
 // DRELU_BGRAD: this row's mask words for a tile. The epilogue loads them

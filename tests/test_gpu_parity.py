@@ -28,7 +28,7 @@ PAIR_SHAPES = [(300, 264, 136), (600, 520, 328), (1000, 1032, 264), (257, 8, 64)
                (1000, 5000, 72), (1024, 5120, 64)]
 # kernel variants: the tile kernel at each width, the few-row kernel and the
 # CTA-pair tile kernel
-VARIANTS = ["tile64", "tile128", "tile256", "skinny", "pair"]
+VARIANTS = ["tile64", "tile128", "tile192", "tile256", "skinny", "pair"]
 
 
 def _force(monkeypatch, variant):
@@ -157,6 +157,7 @@ def test_pair_stream_k(monkeypatch, T, N, K, dtype):
     zero again) through the CTA-pair kernel's stream-K mode; the unfused GEMM
     and integer inputs (bit-exact whatever the split) too."""
     _force(monkeypatch, "pair")
+    monkeypatch.setenv("GEMM_EPI_PAIR_SPLIT", "1")
     inp = synth.make_shape_inputs(T, N, K, dtype, seed=T + 5 * N + K, D2=K)
     for ep in FWD_EPILOGS:
         gpu = run_forward(inp, ep, DT[dtype])
@@ -176,9 +177,9 @@ def test_pair_stream_k(monkeypatch, T, N, K, dtype):
     check_backward(iinp, ifwd["aux"], DT[dtype], run_backward(iinp, ifwd["aux"], DT[dtype]), exact=True)
 
 
-def test_pair_stream_k_can_be_switched_off(monkeypatch):
+def test_pair_stream_k_is_off_by_default(monkeypatch):
     _force(monkeypatch, "pair")
-    monkeypatch.setenv("GEMM_EPI_PAIR_SPLIT", "0")
+    monkeypatch.delenv("GEMM_EPI_PAIR_SPLIT", raising=False)
     T, N, K = 300, 520, 2048
     inp = synth.make_shape_inputs(T, N, K, "bf16", seed=5, D2=K)
     gpu = run_forward(inp, "RELU_AUX_BIAS", torch.bfloat16)
@@ -446,7 +447,7 @@ WGRAD_SHAPES = [(200, 264, 136), (1, 72, 64), (130, 520, 328), (1000, 1032, 264)
                 (777, 2056, 1104)]
 
 
-@pytest.mark.parametrize("variant", ["tile64", "tile128", "tile256", "pair"])
+@pytest.mark.parametrize("variant", ["tile64", "tile128", "tile192", "tile256", "pair"])
 @pytest.mark.parametrize("dtype", ["fp16", "bf16"])
 @pytest.mark.parametrize("T,N,K", WGRAD_SHAPES)
 def test_wgrad_matches_oracle(monkeypatch, T, N, K, dtype, variant):
@@ -548,6 +549,8 @@ def test_watchdog_reports_timeout_and_context_stays_usable(monkeypatch, epilog, 
     returns, and the host reads ERR_TIMEOUT. The same plan and a fresh one
     afterwards must compute correctly."""
     _force(monkeypatch, variant)
+    if variant == "pair" and K >= 1024:
+        monkeypatch.setenv("GEMM_EPI_PAIR_SPLIT", "1")
     monkeypatch.setenv("GEMM_EPI_WAIT_TIMEOUT_MS", "200")
     monkeypatch.setenv("GEMM_EPI_INJECT_STALL", "1")
     monkeypatch.setenv("GEMM_EPI_TEST_HOOKS", "1")
