@@ -277,10 +277,10 @@ SkinnyCfg skinny_cfg_tp(int epi, bool bf16, int kps) {
 
 // Two k-blocks per stage (W stages of 32 KB) while X's share of a stage is
 // small: at T = 1 and 8 (N = 11008, K = 4096) 26.7 us against 28.7 us with
-// one, at T = 64 28.7 against 32.8 us (both directions); at T = 128 one
-// k-block per stage (7 stages against 3) is faster (35.7 against 38.8 us).
-// Four per stage never beat two.
-int default_kps(int64_t T) { return T <= 64 ? 2 : 1; }
+// one, at T = 64 28.7 against 32.8 us, at T = 128 32.8 / 36.8 against
+// 36.8 / 38.9 us (forward / backward, current sources; an older build had
+// one k-block ahead at T = 128). Four per stage never beat two.
+int default_kps(int64_t T) { return T <= 128 ? 2 : 1; }
 
 SkinnyCfg skinny_cfg(int64_t T, int epi, bool bf16) {
   int kps = default_kps(T);
@@ -295,38 +295,80 @@ SkinnyCfg skinny_cfg(int64_t T, int epi, bool bf16) {
   return skinny_cfg_tp<256>(epi, bf16, kps);
 }
 
-// Few-row problems (T <= 256) use the swap-AB stream-K kernel unless
-// GEMM_EPI_FORCE_KERNEL says otherwise ("tile" or "skinny").
-// CTA pairs (256 x 256 tiles) when there is at least one full wave of pair
-// tiles and the row operand X is at most 1 GiB. The size limit is measured,
-// not derived: under the 1 kW power cap the pair kernel ran the
-// 65536 x 16384 x 8192 fp16 problem (X = 2 GiB) at ~860 MHz and 908 TFLOP/s
-// against the one-CTA kernel's ~1100 MHz and 1106 TFLOP/s, while at
-// T = 16384 (X = 512 MiB) and below the pair kernel was as fast or up to 6 %
-// faster. GEMM_EPI_FORCE_KERNEL=tile / pair overrides.
+// Kernel and tile choice by a small cost model, fitted to measurements on
+// one B200 (bf16, K = 4096, one tile per CTA, events around each call):
+// the one-CTA kernel's throughput per SM grows with the tile width, because
+// every stage brings the same 16 KB of X for BN/64 times the MMA work --
+// about 3.1, 5.4, 7.5 and 9.3 TFLOP/s per SM at BN = 64, 128, 192 and 256
+// (e.g. T = 512, N = K = 4096: 49.1 us with 256 tiles of BN = 64, 30.7 us
+// with 128 of BN = 128). CTA pairs (256 x 256 tiles, two thirds of the
+// operand bytes per FLOP) run about 10 per SM. A plan's estimate is rounds
+// of tiles x time per tile; the pair kernel's last round counts half when its
+// tiles fit the half-width tail split.
+double tile_rate(int bn) { return bn == 256 ? 9.3 : bn == 192 ? 7.5 : bn == 128 ? 5.4 : 3.1; }
+constexpr double kPairRate = 10.0;
+
+double est_tile_us(int64_t T, int64_t N, int64_t K, int bn, int sms) {
+  const int64_t tiles = ((T + ge::kBM - 1) / ge::kBM) * ((N + bn - 1) / bn);
+  const int64_t rounds = (tiles + sms - 1) / sms;
+  return double(rounds) * 2.0 * ge::kBM * bn * double(K) / (tile_rate(bn) * 1e6);
+}
+
+double est_pair_us(int64_t T, int64_t N, int64_t K, int pairs) {
+  const int64_t tiles = ((T + 255) / 256) * ((N + 255) / 256);
+  const int64_t full = tiles / pairs, tail = tiles % pairs;
+  const double rounds = double(full) + (tail == 0 ? 0.0 : 2 * tail <= pairs ? 0.5 : 1.0);
+  return rounds * 2.0 * 256 * 256 * double(K) / (2.0 * kPairRate * 1e6);
+}
+
+// one-CTA tile width: the fastest estimate (the wider on a tie)
+int choose_bn(int64_t T, int64_t N, int64_t K, int num_sms) {
+  if (const char* f = getenv("GEMM_EPI_FORCE_BN")) {
+    int v = atoi(f);
+    if (v == 64 || v == 128 || v == 192 || v == 256) return v;
+  }
+  int best = 256;
+  double best_us = est_tile_us(T, N, K, 256, num_sms);
+  for (int bn : {192, 128, 64}) {
+    const double us = est_tile_us(T, N, K, bn, num_sms);
+    if (us < best_us * 0.999) {
+      best = bn;
+      best_us = us;
+    }
+  }
+  return best;
+}
+
+// CTA pairs when there is at least one full wave of pair tiles (fewer would
+// leave pairs idle, and half-width tail units are fed less efficiently), X is
+// at most 1 GiB, and the estimate beats the best one-CTA tile. The size limit
+// is measured: on the 65536 x 16384 x 8192 fp16 problem (X = 2 GiB) the pair
+// kernel read 46.0 GB from DRAM per launch against the one-CTA kernel's 24.3
+// (ncu), and under the 1 kW power cap ran at 908 against 1106 TFLOP/s.
+// GEMM_EPI_FORCE_KERNEL=tile / pair overrides.
 bool use_pair(int64_t T, int64_t N, int64_t K, int num_sms) {
-  const int64_t pair_tiles = ((T + 255) / 256) * ((N + 255) / 256);
   if (const char* f = getenv("GEMM_EPI_FORCE_KERNEL")) {
     if (!strcmp(f, "tile") || !strcmp(f, "skinny")) return false;
     if (!strcmp(f, "pair")) return T > 128;
   }
-  if (T * K * 2 > ((int64_t)1 << 30)) return false;
-  // 129..256 rows: one pair tile row halves each CTA's operand feed against
-  // the few-row kernel's (measured at N = 11008, K = 4096, forward / backward:
-  // T = 256 38.0 / 40.3 us against 50.1 / 60.8; T = 192 39.4 / 41.5 against
-  // 50.3 / 53.8), given a quarter wave of tiles; at T = 128 the few-row kernel
-  // is as fast and wastes no rows
-  if (T > 128 && T <= 256) return pair_tiles >= num_sms / 4;
-  return T > 256 && pair_tiles >= num_sms / 2;
+  if (T <= 128 || T * K * 2 > ((int64_t)1 << 30)) return false;
+  const int pairs = num_sms / 2;
+  const int64_t pair_tiles = ((T + 255) / 256) * ((N + 255) / 256);
+  if (pair_tiles < pairs) return false;
+  const int bn = choose_bn(T, N, K, num_sms);
+  return est_pair_us(T, N, K, pairs) <= est_tile_us(T, N, K, bn, num_sms);
 }
 
+// The few-row kernel for T <= 128; from 129 rows on, one-CTA tiles of 192
+// columns beat it (T = 256, N = 11008, K = 4096: 34.7 / 36.9 us against
+// 47.1 / 51.2 us, and against the CTA pair's 36.6 / 40.9 us).
 bool use_skinny(int64_t T) {
   if (const char* f = getenv("GEMM_EPI_FORCE_KERNEL")) {
     if (!strcmp(f, "tile")) return false;
     if (!strcmp(f, "skinny")) return T <= 256;
     if (!strcmp(f, "pair")) return T <= 128;
   }
-  return T <= 256;
+  return T <= 128;
 }
 
 }  // namespace
@@ -506,15 +548,18 @@ int launch_tile(gemm_epi_plan_s* p, const TileCfg& c, const ge::TileParams& k_in
 }
 
 // Raster: which operand's block stays in L2 while the other streams past
-// it. Holding a group of R row tiles of X (R x tile_rows x K x 2 bytes) while
-// the group sweeps every column block streams W from HBM once per group;
-// holding C column tiles of W streams X once per group. The estimate of the
-// HBM reads of each -- X + ceil(m_tiles / R) W, or W + ceil(n_tiles / C) X --
-// picks the order, with the held block kept to about 48 MB, a little under
-// half of the 126 MB L2 (when all of X fits, W is streamed once). The column
-// order wins only when X is much larger than W (the 65536 x 16384 x 8192
-// problem: X 2 GiB, W 256 MiB). GEMM_EPI_RASTER=m|n and GEMM_EPI_GROUP_M (the
-// group size in tiles) override, for measurement.
+// it. Holding a group of R row tiles of X (about 48 MB, a little under half
+// of the 126 MB L2) while the group sweeps every column block streams W from
+// HBM once per group -- once in all when all of X fits (FFN, square). When X
+// is both larger than the L2 and at least 4x W, a group of column tiles of W
+// (about 64 MB) is held instead and X streams past it. Measured on the
+// 65536 x 16384 x 8192 fp16 problem (X 2 GiB, W 256 MiB; ncu, DRAM bytes read
+// per launch, one-CTA kernel, 256-column tiles): row groups 24.3 GB; column
+// groups of 6, 8 and 12 tiles 20.1, 18.0 and 19.2 GB, at equal time (13.4 to
+// 13.8 ms). Every order reads several times the operands there: a wave of
+// 148 tiles touches 1.8 GB of operands at K = 16384, 14 times the L2.
+// GEMM_EPI_RASTER=m|n and GEMM_EPI_GROUP_M (the group size in tiles)
+// override, for measurement.
 struct Raster {
   int group = 1;
   int by_n = 0;
@@ -522,15 +567,13 @@ struct Raster {
 
 Raster choose_raster(int64_t T, int64_t N, int64_t K, int tile_rows, int tile_cols) {
   const int64_t m_tiles = (T + tile_rows - 1) / tile_rows, n_tiles = (N + tile_cols - 1) / tile_cols;
-  const double budget = double(48 << 20);
   const double x_bytes = 2.0 * T * K, w_bytes = 2.0 * K * N;
-  int64_t R = (int64_t)(budget / (2.0 * tile_rows * K)), C = (int64_t)(budget / (2.0 * tile_cols * K));
+  int64_t R = (int64_t)(double(48 << 20) / (2.0 * tile_rows * K));
+  int64_t C = (int64_t)(double(64 << 20) / (2.0 * tile_cols * K));
   R = R < 1 ? 1 : R > m_tiles ? m_tiles : R;
   C = C < 1 ? 1 : C > n_tiles ? n_tiles : C;
-  const double by_m = x_bytes + double((m_tiles + R - 1) / R) * w_bytes;
-  const double by_n = w_bytes + double((n_tiles + C - 1) / C) * x_bytes;
   Raster r;
-  r.by_n = by_n < 0.9 * by_m ? 1 : 0;
+  r.by_n = (x_bytes > double(128 << 20) && x_bytes >= 4.0 * w_bytes) ? 1 : 0;
   r.group = (int)(r.by_n ? C : R);
   if (const char* f = getenv("GEMM_EPI_RASTER")) {  // tuning override
     if (!strcmp(f, "m") || !strcmp(f, "n")) {
@@ -589,20 +632,6 @@ int launch_skinny(const gemm_epi_plan_s* p, const ge::SkinnyParams& k, cudaStrea
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "few-row kernel launch");
   return GEMM_EPI_OK;
-}
-
-int choose_bn(int64_t T, int64_t N, int num_sms) {
-  if (const char* f = getenv("GEMM_EPI_FORCE_BN")) {
-    int v = atoi(f);
-    if (v == 64 || v == 128 || v == 192 || v == 256) return v;
-  }
-  const int64_t m_tiles = (T + ge::kBM - 1) / ge::kBM;
-  // widest tile that still gives every SM at least one tile, else the
-  // narrowest: wide tiles need the least shared-memory bandwidth per MMA
-  for (int bn : {256, 128}) {
-    if (m_tiles * ((N + bn - 1) / bn) >= num_sms) return bn;
-  }
-  return 64;
 }
 
 }  // namespace
@@ -680,7 +709,7 @@ gemm_epi_plan_t gemm_epi_plan_ex(int64_t T, int64_t N, int64_t K, gemm_epi_dtype
   p->num_sms = sms;
   const bool bf16 = dtype == GEMM_EPI_BF16;
   const bool pair = use_pair(T, N, K, sms);
-  const int bn = pair ? 256 : choose_bn(T, N, sms);
+  const int bn = pair ? 256 : choose_bn(T, N, K, sms);
   p->cfg = pair ? pair_cfg((int)epilog, bf16, w_nk) : tile_cfg(bn, (int)epilog, bf16, w_nk);
   p->cfg_store = pair ? pair_cfg(ge::EPI_STORE, bf16, w_nk) : tile_cfg(bn, ge::EPI_STORE, bf16, w_nk);
   p->kernel = pair ? 2 : 0;
@@ -1221,7 +1250,7 @@ extern "C" int drelu_bgrad_execute_noalloc(int64_t T, int64_t N, int64_t K, gemm
   int* status = reinterpret_cast<int*>(nd->scratch);
   float* partials = reinterpret_cast<float*>(nd->scratch + kNoAllocStatusBytes);
 
-  const int bn = choose_bn(T, N, sms);
+  const int bn = choose_bn(T, N, K, sms);
   const TileCfg cfg = tile_cfg(bn, ge::EPI_DRELU_BGRAD, dtype == GEMM_EPI_BF16, false);
   CUtensorMap tmA, tmB, tmY;
   rc = encode_2d(&tmA, dY2, (uint64_t)K, (uint64_t)T, ge::kBK, ge::kBM, "dY2");

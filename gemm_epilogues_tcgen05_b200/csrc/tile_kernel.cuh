@@ -467,8 +467,19 @@ __device__ __forceinline__ void epi_finish_dbias(const TileParams& p, int nb, in
     for (int c = et; c < ncols; c += 128) {
       const int n = n0 + c;
       if (n < p.N) {
+        // ascending m as always; the loads of a batch of 16 rows are issued
+        // together (the L2 round trips would otherwise run one by one)
+        const float* col = p.partials + n;
         float s = 0.f;
-        for (int m = 0; m < p.m_tiles; ++m) s += __ldcg(p.partials + static_cast<int64_t>(m) * p.N + n);
+        int m = 0;
+        for (; m + 16 <= p.m_tiles; m += 16) {
+          float x[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) x[j] = __ldcg(col + static_cast<int64_t>(m + j) * p.N);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) s += x[j];
+        }
+        for (; m < p.m_tiles; ++m) s += __ldcg(col + static_cast<int64_t>(m) * p.N);
         p.dbias[n] = s;
       }
     }
