@@ -750,14 +750,12 @@ gemm_epi_plan_t gemm_epi_plan_ex(int64_t T, int64_t N, int64_t K, gemm_epi_dtype
     const int pair_tiles = ceil_div(T, 256) * p->n_tiles;
     const int max_pairs = max_resident_pairs(p->cfg, sms);
     int pairs = pair_tiles < max_pairs ? pair_tiles : max_pairs;
-    // opt-in (GEMM_EPI_PAIR_SPLIT=1): on the shapes measured so far its
-    // fixup (segment 0 reading the other segments' partials back from L2)
-    // costs more than the idle pairs give (T = 256, N = 11008, K = 4096:
-    // 61.4 us against 36.8 us; 1024 x 512 x 2048: 60.0 against 18.4 us)
+    // opt-in (GEMM_EPI_PAIR_SPLIT=1), see the measurements in the header of
+    // tile2_kernel.cuh
     bool split = false;
-    if (const char* f = getenv("GEMM_EPI_PAIR_SPLIT")) split = atoi(f) != 0 && pair_tiles < max_pairs && p->k_blocks >= 16;
-    if (split) {
-      const int64_t want = (int64_t)pair_tiles * p->k_blocks / 8;
+    if (const char* f = getenv("GEMM_EPI_PAIR_SPLIT")) split = atoi(f) != 0 && p->k_blocks >= 16;
+    if (split && pair_tiles < max_pairs) {
+      const int64_t want = (int64_t)pair_tiles * p->k_blocks / 8;  // at least 8 k-blocks per pair
       const int sp = (int)(want < max_pairs ? want : max_pairs);
       split = sp > pair_tiles;
       if (split) pairs = sp;
@@ -767,24 +765,24 @@ gemm_epi_plan_t gemm_epi_plan_ex(int64_t T, int64_t N, int64_t K, gemm_epi_dtype
       p->pair_split = 1;
       p->cfg = pair_cfg((int)epilog, bf16, w_nk, true);
       p->cfg_store = pair_cfg(ge::EPI_STORE, bf16, w_nk, true);
-      const int64_t total = (int64_t)pair_tiles * p->k_blocks;
+      const int dp_tiles = ge::pair_dp_rounds(pair_tiles, pairs) * pairs;
+      const int64_t total = (int64_t)(pair_tiles - dp_tiles) * p->k_blocks;
       p->pair_max_segs = 1;
-      for (int t = 0; t < pair_tiles; ++t) {
+      for (int t = 0; t < pair_tiles - dp_tiles; ++t) {
         const int64_t a = ge::pair_owner((int64_t)t * p->k_blocks, pairs, total);
         const int64_t b = ge::pair_owner((int64_t)(t + 1) * p->k_blocks - 1, pairs, total);
         if (b - a + 1 > p->pair_max_segs) p->pair_max_segs = (int)(b - a + 1);
       }
-      p->pair_bytes = (size_t)pair_tiles * (p->pair_max_segs - 1) * 2 * ge::kBM * 256 * sizeof(float);
-      if (p->pair_bytes) {
-        e = cudaMalloc((void**)&p->pair_slots, p->pair_bytes);
-        if (e != cudaSuccess) return cleanup(cuda_fail(e, "cudaMalloc(stream-K partials)"));
-      }
-      e = cudaMalloc((void**)&p->pair_flags, sizeof(int) * 2 * (size_t)pair_tiles);
+      // one slot per pair and CTA (a pair hands on at most one segment: its first unit)
+      p->pair_bytes = (size_t)pairs * 2 * ge::kBM * 256 * sizeof(float);
+      e = cudaMalloc((void**)&p->pair_slots, p->pair_bytes);
+      if (e != cudaSuccess) return cleanup(cuda_fail(e, "cudaMalloc(stream-K partials)"));
+      e = cudaMalloc((void**)&p->pair_flags, sizeof(int) * 2 * (size_t)pairs);
       if (e != cudaSuccess) return cleanup(cuda_fail(e, "cudaMalloc(stream-K flags)"));
-      e = cudaMemset(p->pair_flags, 0, sizeof(int) * 2 * (size_t)pair_tiles);
+      e = cudaMemset(p->pair_flags, 0, sizeof(int) * 2 * (size_t)pairs);
       if (e != cudaSuccess) return cleanup(cuda_fail(e, "cudaMemset(stream-K flags)"));
-      p->n_pair_flags = 2 * pair_tiles;
-      p->pair_bytes += sizeof(int) * 2 * (size_t)pair_tiles;
+      p->n_pair_flags = 2 * pairs;
+      p->pair_bytes += sizeof(int) * 2 * (size_t)pairs;
     }
   }
   for (const TileCfg* c : {&p->cfg, &p->cfg_store}) {

@@ -50,7 +50,7 @@ struct Tile2Smem {
   static constexpr uint32_t OFF_A = 0;
   static constexpr uint32_t OFF_B = OFF_A + STAGES * A_BYTES;
   static constexpr uint32_t OFF_BAR = OFF_B + STAGES * B_BYTES;
-  static constexpr uint32_t N_BARS = 2 * STAGES + 5;
+  static constexpr uint32_t N_BARS = 2 * STAGES + 6;  // full, empty, tfull[2], tempty[2], drain, stream-K fixup
   static constexpr uint32_t OFF_MISC = OFF_BAR + N_BARS * 8;
   static constexpr uint32_t OFF_BIAS = (OFF_MISC + 16 + 15) / 16 * 16;
   static constexpr uint32_t OFF_COLP = OFF_BIAS + 2 * BN * 4;
@@ -99,50 +99,85 @@ struct PairSchedule {
   }
 };
 
+// Stream-K part of a split schedule: with at least two waves of tiles, the
+// first rounds - 1 waves stay whole tiles, one per pair as without the
+// split, and only the rest (between one and two waves of tiles) is cut into
+// equal k-ranges, so every range spans at least one tile's k-blocks and a
+// tile has at most two segments; with fewer tiles every tile is cut.
+__device__ __host__ __forceinline__ int pair_dp_rounds(int tiles, int npairs) {
+  const int rounds = tiles / npairs;
+  return rounds >= 2 ? rounds - 1 : 0;
+}
+
 // The sequence of units of one pair. Without SPLIT: units pair, pair +
 // npairs, ... of the schedule, each over every k-block. With SPLIT: the
-// pieces of the pair's contiguous range [lo, hi) of the flattened (tile,
-// k-block) space, tile by tile.
+// pair's whole tiles of the data-parallel rounds, then the pieces of its
+// contiguous range [lo, hi) of the flattened (tile, k-block) space of the
+// remaining tiles, tile by tile.
 template <bool SPLIT>
 struct PairWork {
   PairSchedule sched;
   int pair, npairs, m2_tiles, n_tiles, group, by_n, k_blocks;
-  int64_t total, hi, cur;
+  int dp_units, dp_tiles;  // SPLIT: whole tiles of the data-parallel rounds (this pair's, and in all)
+  int64_t total, lo, hi, cur;
   __device__ __forceinline__ PairWork(const TileParams& p, int pair_, int npairs_, int m2)
       : sched(m2 * p.n_tiles, npairs_, !SPLIT && p.tail_split != 0),
         pair(pair_), npairs(npairs_), m2_tiles(m2), n_tiles(p.n_tiles), group(p.group_m), by_n(p.raster_n),
         k_blocks(p.k_blocks) {
-    total = static_cast<int64_t>(m2) * p.n_tiles * p.k_blocks;
     if constexpr (SPLIT) {
-      cur = static_cast<int64_t>(pair) * total / npairs;
+      const int tiles = m2 * p.n_tiles;
+      const int rounds = pair_dp_rounds(tiles, npairs);
+      dp_tiles = rounds * npairs;
+      dp_units = rounds;
+      total = static_cast<int64_t>(tiles - dp_tiles) * p.k_blocks;
+      lo = static_cast<int64_t>(pair) * total / npairs;
       hi = static_cast<int64_t>(pair + 1) * total / npairs;
+      cur = -dp_units;  // negative: data-parallel rounds still to go
     } else {
       cur = pair;
       hi = sched.num_units;
     }
   }
+  // this is the pair's last unit (after next() returned it)
+  __device__ __forceinline__ bool done() const { return SPLIT ? (cur >= 0 && lo + cur >= hi) : cur >= hi; }
   __device__ __forceinline__ bool next(PairUnit& w) {
-    if (cur >= hi) return false;
     if constexpr (SPLIT) {
-      const int t = static_cast<int>(cur / k_blocks);
-      const int64_t tb = static_cast<int64_t>(t) * k_blocks;
+      if (cur < 0) {  // a whole tile of the data-parallel rounds
+        const int t = pair + (dp_units + static_cast<int>(cur)) * npairs;
+        tile_coords(t, m2_tiles, n_tiles, group, by_n, w.mb, w.nb);
+        w.half = -1;
+        w.kb0 = 0;
+        w.kb1 = k_blocks;
+        w.tile = t;
+        w.seg = 0;
+        w.nsegs = 1;
+        ++cur;
+        return true;
+      }
+      const int64_t g = lo + cur;  // stream-K index
+      if (g >= hi) return false;
+      const int tl = static_cast<int>(g / k_blocks);  // tile among the stream-K tiles
+      const int64_t tb = static_cast<int64_t>(tl) * k_blocks;
       const int64_t end = hi < tb + k_blocks ? hi : tb + k_blocks;
+      const int t = dp_tiles + tl;
       tile_coords(t, m2_tiles, n_tiles, group, by_n, w.mb, w.nb);
       w.half = -1;
-      w.kb0 = static_cast<int>(cur - tb);
+      w.kb0 = static_cast<int>(g - tb);
       w.kb1 = static_cast<int>(end - tb);
       w.tile = t;
       const int64_t first = pair_owner(tb, npairs, total);
       w.nsegs = static_cast<int>(pair_owner(tb + k_blocks - 1, npairs, total) - first + 1);
       w.seg = static_cast<int>(pair - first);
-      cur = end;
+      cur = end - lo;
+      return true;
     } else {
+      if (cur >= hi) return false;
       w = sched.unit(static_cast<int>(cur), m2_tiles, n_tiles, group, by_n);
       w.kb0 = 0;
       w.kb1 = k_blocks;
       cur += npairs;
+      return true;
     }
-    return true;
   }
 };
 
@@ -172,6 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
+  uint64_t* fixbar = drain + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
   float* bias_s = reinterpret_cast<float*>(smem + L::OFF_BIAS);  // [2][BN]
@@ -197,6 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&tempty[b], 8);
     }
     mbar_init(drain, 1);
+    mbar_init(fixbar, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -331,16 +368,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
       const uint32_t trow = tmem_base + ((ew * 32u) << 16) + buf * BN;
       const int r = static_cast<int>(ew * 32 + lane);  // this thread's row of the CTA's 128
-      // stream-K slots of this tile and CTA: segment s >= 1 at slot (s - 1)
+      // stream-K slots, one per pair and CTA: a pair's only later segment is
+      // its first unit, so segment s of the tile that pair `pair` finishes
+      // is in pair (pair + s)'s slot; the flag of a tile is its finisher's
       const int64_t slot_stride = 2 * kBM * BN;
-      float* slot0 = SPLIT ? p.sk_slots + (static_cast<int64_t>(w.tile) * (p.sk_max_segs - 1) * 2 + rank) * (kBM * BN)
-                           : nullptr;
-      int* flag = SPLIT ? p.sk_flags + w.tile * 2 + rank : nullptr;
+      float* own_slot = SPLIT ? p.sk_slots + (static_cast<int64_t>(pair) * 2 + rank) * (kBM * BN) : nullptr;
       if (SPLIT && w.seg > 0) {
         // a later segment: hand the fp32 accumulator to segment 0 and count it in
         if (ok) {
           tc_fence_after();
-          float* dst = slot0 + (w.seg - 1) * slot_stride + r * BN;
+          float* dst = own_slot + r * BN;
 #pragma unroll 1
           for (int c = 0; c < BN / 32; ++c) {
             uint32_t v[32];
@@ -358,12 +395,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __threadfence();
         named_bar_sync(1, 128);
-        if (et == 0 && ok) atomicAdd(flag, 1);
+        if (et == 0 && ok) atomicAdd(p.sk_flags + (pair - w.seg) * 2 + rank, 1);
         continue;
       }
       int nadd = 0;
+      const float* addp = nullptr;
+      bool add_smem = false;
       if (SPLIT && w.nsegs > 1) {
         // segment 0: wait until the other segments' partials are in (bounded)
+        int* flag = p.sk_flags + pair * 2 + rank;
+        // the pair's last unit with one other segment: its operand stages are
+        // idle (the MMAs that read them are complete), so that segment's
+        // 128 KB comes in with bulk copies and is added from shared memory
+        const bool bulk = w.nsegs == 2 && work.done();
         if (et == 0) {
           int got = ok ? 1 : 0;
           if (got) {
@@ -379,17 +423,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (got) *flag = 0;  // ready for the next launch
           }
           __threadfence();
+          if (got && bulk) {
+            constexpr uint32_t kPart = kBM * BN * 4, kPiece = 32768;
+            const float* src = own_slot + slot_stride;  // pair + 1's slot
+            mbar_arrive_expect_tx(fixbar, kPart);
+            for (uint32_t off = 0; off < kPart; off += kPiece)
+              bulk_load_g2s(smem + off, reinterpret_cast<const uint8_t*>(src) + off, kPiece, fixbar);
+          }
           *sflag = got;
         }
         named_bar_sync(1, 128);
         ok = ok && *sflag != 0;
+        if (ok && bulk) ok = wait_bounded(fixbar, 0, p, abort_flag, 8);
+        ok = __all_sync(0xffffffffu, ok);
         nadd = w.nsegs - 1;
+        addp = bulk ? reinterpret_cast<const float*>(smem) + r * BN : own_slot + slot_stride + r * BN;
+        add_smem = bulk;
       }
       if (ok) {
         tc_fence_after();
         epi_rows<BN, EPI, BF16>(p, trow, m0 + r, n0, bs, cp + ew * BN, &tmY, stg, scount, m0 + static_cast<int>(ew * 32),
-                                &tmAux, auxstg_s + ew * kAuxStageBytesPerWarp, mw, ncols, w.half < 0,
-                                SPLIT ? slot0 + r * BN : nullptr, nadd, slot_stride);
+                                &tmAux, auxstg_s + ew * kAuxStageBytesPerWarp, mw, ncols, w.half < 0, addp, nadd,
+                                slot_stride, add_smem);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(tempty0 + buf * 8);

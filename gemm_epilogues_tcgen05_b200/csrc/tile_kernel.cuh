@@ -114,8 +114,8 @@ struct TileParams {
   int32_t raster_n;         // tile order by column groups (see tile_coords)
   // CTA-pair stream-K (few tiles): the k-blocks of all tiles are cut into one
   // contiguous range per pair; a tile's later segments leave fp32 partials
-  float* sk_slots;          // [tiles][max_segs - 1][2 ranks][128 rows][256 cols]
-  int* sk_flags;            // [tiles][2 ranks] segments written, zero between launches
+  float* sk_slots;          // [pairs][2 ranks][128 rows][256 cols]: a pair's later segment
+  int* sk_flags;            // [pairs][2 ranks]: segments in for the tile the pair finishes; zero between launches
   int32_t sk_max_segs;
 };
 
@@ -320,7 +320,8 @@ __device__ __forceinline__ void epi_rows(const TileParams& p, uint32_t tbase, in
                                          float* cpw, const CUtensorMap* tmY, uint8_t* stg, uint32_t& scount,
                                          int wrow0, const CUtensorMap* tmAux, uint8_t* auxstg,
                                          const MaskWords<BN>& mw, int ncols = BN, bool aux_block = true,
-                                         const float* addp = nullptr, int nadd = 0, int64_t add_stride = 0) {
+                                         const float* addp = nullptr, int nadd = 0, int64_t add_stride = 0,
+                                         bool add_smem = false) {
   const uint32_t lane = lane_id();
   const bool row_ok = row < p.T;
   constexpr bool kAuxTma = EPI == EPI_RELU_AUX_BIAS && AuxByTma<BN>::value;
@@ -341,12 +342,13 @@ __device__ __forceinline__ void epi_rows(const TileParams& p, uint32_t tbase, in
 #pragma unroll
     for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
     // stream-K: this thread's row of the other k-segments' fp32 partial
-    // accumulators (written by other CTA pairs), added in segment order
+    // accumulators (written by other CTA pairs; in global memory, or brought
+    // into shared memory), added in segment order
     for (int sg = 0; sg < nadd; ++sg) {
       const float4* q = reinterpret_cast<const float4*>(addp + sg * add_stride + c * 32);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const float4 x = __ldcg(q + i);
+        const float4 x = add_smem ? q[i] : __ldcg(q + i);
         v[4 * i] += x.x;
         v[4 * i + 1] += x.y;
         v[4 * i + 2] += x.z;

@@ -180,6 +180,31 @@ def test_pair_stream_k(monkeypatch, T, N, K, dtype):
     check_backward(iinp, ifwd["aux"], DT[dtype], run_backward(iinp, ifwd["aux"], DT[dtype]), exact=True)
 
 
+# stream-K over at least one wave of tiles: every k-range spans a tile or
+# more, so a tile has at most two segments and the finishing segment brings
+# the other's partial in with bulk copies; the second shape keeps one
+# data-parallel round of whole tiles before the stream-K tiles
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+@pytest.mark.parametrize("T,N,K", [(1024, 4864, 1024), (1100, 9728, 1024)])
+def test_pair_stream_k_waves(monkeypatch, T, N, K, dtype):
+    _force(monkeypatch, "pair")
+    monkeypatch.setenv("GEMM_EPI_PAIR_SPLIT", "1")
+    inp = synth.make_shape_inputs(T, N, K, dtype, seed=T + N + 3 * K, D2=K)
+    for ep in ("RELU_AUX_BIAS", "GELU_AUX_BIAS"):
+        gpu = run_forward(inp, ep, DT[dtype])
+        assert gpu["info"]["kernel"] == 2 and gpu["info"]["split_k"] == 2, gpu["info"]
+        check_forward(inp, ep, DT[dtype], gpu)
+    fwd = run_forward(inp, "RELU_AUX_BIAS", DT[dtype])
+    outs = run_backward(inp, fwd["aux"], DT[dtype], repeats=2)
+    for gpu in outs:
+        check_backward(inp, fwd["aux"], DT[dtype], gpu)
+    assert torch.equal(outs[0]["dbias"], outs[1]["dbias"])
+    assert torch.equal(outs[0]["dZ"].view(torch.int16), outs[1]["dZ"].view(torch.int16))
+    if T == 1024:
+        iinp = synth.make_shape_inputs(T, N, K, dtype, seed=T + N, D2=K, kind="int")
+        check_forward(iinp, "BIAS", DT[dtype], run_forward(iinp, "BIAS", DT[dtype]), exact=True)
+
+
 def test_pair_stream_k_is_off_by_default(monkeypatch):
     _force(monkeypatch, "pair")
     monkeypatch.delenv("GEMM_EPI_PAIR_SPLIT", raising=False)
