@@ -374,24 +374,46 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t slot_stride = 2 * kBM * BN;
       float* own_slot = SPLIT ? p.sk_slots + (static_cast<int64_t>(pair) * 2 + rank) * (kBM * BN) : nullptr;
       if (SPLIT && w.seg > 0) {
-        // a later segment: hand the fp32 accumulator to segment 0 and count it in
+        // a later segment: hand the fp32 accumulator to segment 0 and count it
+        // in. Each warp stages its rows as 2 KB blocks of 32 rows x 16 columns
+        // (the swizzled layout of the output staging) and writes each block
+        // with one bulk copy into its 32 KB of the slot.
         if (ok) {
           tc_fence_after();
-          float* dst = own_slot + r * BN;
+          float* dst = own_slot + ew * (16 * 512);
 #pragma unroll 1
           for (int c = 0; c < BN / 32; ++c) {
             uint32_t v[32];
             tmem_ld_32x32b_x32(trow + c * 32, v);
             tmem_wait_ld();
-            float4* q = reinterpret_cast<float4*>(dst + c * 32);
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              __stcg(q + i, make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                        __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3])));
+            for (int h = 0; h < 2; ++h) {
+              uint8_t* sbuf = stg + (scount & 1u) * 2048;
+              if (lane == 0) bulk_wait_group_read<1>();
+              __syncwarp();
+              const uint32_t rbase = smem_u32(sbuf) + lane * 64;
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                st_shared_v4(rbase + ((q ^ ((lane >> 1) & 3u)) * 16),
+                             make_uint4(v[16 * h + 4 * q], v[16 * h + 4 * q + 1], v[16 * h + 4 * q + 2],
+                                        v[16 * h + 4 * q + 3]));
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                bulk_store_s2g(dst + (2 * c + h) * 512, sbuf, 2048);
+                bulk_commit_group();
+              }
+              ++scount;
+            }
           }
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive_cluster(tempty0 + buf * 8);
+          if (lane == 0) {
+            bulk_wait_group_all();  // the partial is in global memory
+            fence_proxy_async_global();
+          }
+          __syncwarp();
         }
         __threadfence();
         named_bar_sync(1, 128);
@@ -424,6 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           __threadfence();
           if (got && bulk) {
+            fence_proxy_async_global();  // the bulk copies below read what the flag announced
             constexpr uint32_t kPart = kBM * BN * 4, kPiece = 32768;
             const float* src = own_slot + slot_stride;  // pair + 1's slot
             mbar_arrive_expect_tx(fixbar, kPart);
@@ -437,7 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok && bulk) ok = wait_bounded(fixbar, 0, p, abort_flag, 8);
         ok = __all_sync(0xffffffffu, ok);
         nadd = w.nsegs - 1;
-        addp = bulk ? reinterpret_cast<const float*>(smem) + r * BN : own_slot + slot_stride + r * BN;
+        addp = bulk ? reinterpret_cast<const float*>(smem) + ew * (16 * 512) : own_slot + slot_stride + ew * (16 * 512);
         add_smem = bulk;
       }
       if (ok) {

@@ -343,16 +343,23 @@ __device__ __forceinline__ void epi_rows(const TileParams& p, uint32_t tbase, in
     for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
     // stream-K: this thread's row of the other k-segments' fp32 partial
     // accumulators (written by other CTA pairs; in global memory, or brought
-    // into shared memory), added in segment order
+    // into shared memory), added in segment order. A partial is this warp's
+    // 16 blocks of 32 rows x 16 columns (2 KB each, rows of 64 bytes whose
+    // 16-byte chunks are XOR-swizzled like the output staging); `addp` is the
+    // warp's first block of the first segment.
     for (int sg = 0; sg < nadd; ++sg) {
-      const float4* q = reinterpret_cast<const float4*>(addp + sg * add_stride + c * 32);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float4 x = add_smem ? q[i] : __ldcg(q + i);
-        v[4 * i] += x.x;
-        v[4 * i + 1] += x.y;
-        v[4 * i + 2] += x.z;
-        v[4 * i + 3] += x.w;
+      for (int h = 0; h < 2; ++h) {
+        const float* blk = addp + sg * add_stride + (2 * c + h) * 512 + lane * 16;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float4* src = reinterpret_cast<const float4*>(blk + ((q ^ ((lane >> 1) & 3u)) * 4));
+          const float4 x = add_smem ? *src : __ldcg(src);
+          v[16 * h + 4 * q] += x.x;
+          v[16 * h + 4 * q + 1] += x.y;
+          v[16 * h + 4 * q + 2] += x.z;
+          v[16 * h + 4 * q + 3] += x.w;
+        }
       }
     }
     if constexpr (EPI == EPI_DRELU_BGRAD) {
