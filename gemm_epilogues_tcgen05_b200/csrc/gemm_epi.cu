@@ -744,15 +744,23 @@ gemm_epi_plan_t gemm_epi_plan_ex(int64_t T, int64_t N, int64_t K, gemm_epi_dtype
   if (pair) {
     // One cluster of two CTAs per 256-row x 256-column tile, up to the number
     // of clusters the device can hold at once (a GPC with an odd number of
-    // free SMs cannot place a pair on its last one). With fewer tiles than
-    // that, optionally stream-K: every pair takes an equal share of the
-    // tiles' k-blocks (at least 8), so the idle pairs stream W too.
+    // free SMs cannot place a pair on its last one).
     const int pair_tiles = ceil_div(T, 256) * p->n_tiles;
     const int max_pairs = max_resident_pairs(p->cfg, sms);
     int pairs = pair_tiles < max_pairs ? pair_tiles : max_pairs;
-    // opt-in (GEMM_EPI_PAIR_SPLIT=1), see the measurements in the header of
-    // tile2_kernel.cuh
-    bool split = false;
+    // Stream-K when the whole-tile schedule's last round would keep fewer
+    // than three quarters of the pairs busy (its leftover tiles, split into
+    // column halves where they fit): then cutting the last waves into
+    // k-ranges evens the end out. Measured, alternating runs on one box: FFN
+    // (688 tiles, a last round of 44 half tiles for 74 pairs) forward 244.0
+    // against 256.8 us, backward 252.9 against 257.4; T = 1024, N = 5120
+    // (80 tiles) forward 53.2 against 55.3; square 4096^3 (68 half tiles)
+    // forward equal, backward 111.5 against 108.8, so not there. With fewer
+    // tiles than pairs it loses (fixups through L2 for up to 8 segments):
+    // opt-in only. GEMM_EPI_PAIR_SPLIT=0|1 overrides.
+    const int tail = pair_tiles % max_pairs;
+    const int last_round = tail == 0 ? max_pairs : 2 * tail <= max_pairs ? 2 * tail : tail;
+    bool split = pair_tiles >= max_pairs && p->k_blocks >= 16 && 4 * last_round < 3 * max_pairs;
     if (const char* f = getenv("GEMM_EPI_PAIR_SPLIT")) split = atoi(f) != 0 && p->k_blocks >= 16;
     if (split && pair_tiles < max_pairs) {
       const int64_t want = (int64_t)pair_tiles * p->k_blocks / 8;  // at least 8 k-blocks per pair

@@ -205,6 +205,21 @@ def test_pair_stream_k_waves(monkeypatch, T, N, K, dtype):
         check_forward(iinp, "BIAS", DT[dtype], run_forward(iinp, "BIAS", DT[dtype]), exact=True)
 
 
+def test_pair_stream_k_by_default_when_the_last_round_is_thin(monkeypatch):
+    """80 pair tiles for 74 pairs: the whole-tile schedule's last round would
+    hold 12 half tiles, so the planner cuts the tiles into k-ranges itself."""
+    for k in ("GEMM_EPI_FORCE_KERNEL", "GEMM_EPI_PAIR_SPLIT", "GEMM_EPI_FORCE_BN"):
+        monkeypatch.delenv(k, raising=False)
+    T, N, K = 1024, 5120, 1024
+    inp = synth.make_shape_inputs(T, N, K, "bf16", seed=9, D2=K)
+    gpu = run_forward(inp, "RELU_AUX_BIAS", torch.bfloat16)
+    if gpu["info"]["grid"] == 148:  # every pair resident (the rule counts resident pairs)
+        assert gpu["info"]["kernel"] == 2 and gpu["info"]["split_k"] == 2, gpu["info"]
+    check_forward(inp, "RELU_AUX_BIAS", torch.bfloat16, gpu)
+    out = run_backward(inp, gpu["aux"], torch.bfloat16)
+    check_backward(inp, gpu["aux"], torch.bfloat16, out)
+
+
 def test_pair_stream_k_is_off_by_default(monkeypatch):
     _force(monkeypatch, "pair")
     monkeypatch.delenv("GEMM_EPI_PAIR_SPLIT", raising=False)
