@@ -429,6 +429,8 @@ def run_ours(args, w: synth.Workload, rank: int, world: int, dev: torch.device):
 
     fwd_ms = [e[0].elapsed_time(e[1]) for e in evs]
     bwd_ms = [e[1].elapsed_time(e[2]) for e in evs] if bplan is not None else [0.0] * args.steps
+    spread = {"fwd_ms_median": statistics.median(fwd_ms), "fwd_ms_max": max(fwd_ms),
+              "bwd_ms_median": statistics.median(bwd_ms), "bwd_ms_max": max(bwd_ms)}
     step_ms = sum(fwd_ms) / args.steps + sum(bwd_ms) / args.steps
     step_ms, fwd_avg, bwd_avg = max_over_ranks([step_ms, sum(fwd_ms) / args.steps, sum(bwd_ms) / args.steps], dev,
                                                world)
@@ -458,7 +460,7 @@ def run_ours(args, w: synth.Workload, rank: int, world: int, dev: torch.device):
     return {"step_ms": step_ms, "fwd_ms": fwd_avg, "bwd_ms": bwd_avg, "alg": alg, "flops_step": flops_step,
             "kernel": kernel,
             "launches": launches_per_step * args.steps, "clocks": clocks, "e2e": e2e, "plan_ms": plan_ms,
-            "plan_first_ms": plan_first_ms,
+            "plan_first_ms": plan_first_ms, "spread": spread,
             "wall_s": wall1 - wall0}
 
 
@@ -476,17 +478,21 @@ def run_e2e(args, w, fwd_epi, fplan, bplan, inp_dev, dev, stream):
     aux_words = math.ceil(w.N / 32)
     h2d_s, d2h_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
+    spec = fplan.aux_spec()  # the forward's auxiliary output: mask words, or GELU's pre-activation
+    has_aux = spec is not None
+
     def buffers():
         b = {"in": {k: torch.empty_like(v, device=dev) for k, v in host.items()},
              "Y": torch.empty((w.T, w.N), dtype=dt, device=dev),
-             "aux": torch.empty((w.T, aux_words), dtype=torch.int32, device=dev)}
+             "aux": (torch.empty(spec[0], dtype=spec[1], device=dev) if has_aux and fwd_epi != "RELU_AUX_BIAS"
+                     else torch.empty((w.T, aux_words), dtype=torch.int32, device=dev))}
         if bplan is not None:
             b["dZ"] = torch.empty((w.T, w.N), dtype=dt, device=dev)
             b["dbias"] = torch.empty((w.N,), dtype=torch.float32, device=dev)
         return b
 
     sets = [buffers(), buffers()]
-    keys = ["Y"] + (["aux"] if fwd_epi == "RELU_AUX_BIAS" else []) + (["dZ", "dbias"] if bplan is not None else [])
+    keys = ["Y"] + (["aux"] if has_aux else []) + (["dZ", "dbias"] if bplan is not None else [])
     hout = [{k: torch.empty_like(s[k], device="cpu").pin_memory() for k in keys} for s in sets]
     if bplan is not None and fwd_epi != "RELU_AUX_BIAS":  # the backward's mask, from an untimed forward
         with type(fplan)(w.T, w.N, w.K, dt, "RELU_AUX_BIAS") as mplan:
@@ -510,8 +516,8 @@ def run_e2e(args, w, fwd_epi, fplan, bplan, inp_dev, dev, stream):
         stream.wait_event(up)
         if drained[i % 2] is not None:
             stream.wait_event(drained[i % 2])  # outputs of step i-2 already on the host
-        fplan.gemm_epi_execute(b["in"]["X"], b["in"]["W"], b["in"]["bias"], b["Y"],
-                               b["aux"] if fwd_epi == "RELU_AUX_BIAS" else None, stream)
+        fplan.gemm_epi_execute(b["in"]["X"], b["in"]["W"], b["in"]["bias"], b["Y"], b["aux"] if has_aux else None,
+                               stream)
         if bplan is not None:
             bplan.drelu_bgrad_execute(b["in"]["dY2"], b["in"]["W2"], b["aux"], b["dZ"], b["dbias"], stream)
         done = ev()
@@ -700,7 +706,7 @@ def main():
             "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
             "config": config_of(w, fwd_epi, has_bwd, args),
             "parallelism": f"replicas x{world} (no exchange step)",
-            "fwd_ms": res["fwd_ms"], "bwd_ms": res["bwd_ms"], "roofline": roof,
+            "fwd_ms": res["fwd_ms"], "bwd_ms": res["bwd_ms"], "per_step_spread_rank0": res["spread"], "roofline": roof,
             "gpu_launches": res["launches"], "clocks": res["clocks"]}
     if res.get("plan_ms") is not None:
         line["plan_ms"] = res["plan_ms"]  # host time to create one plan (created once, reused every step)

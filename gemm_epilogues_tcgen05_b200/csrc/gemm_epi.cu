@@ -506,15 +506,8 @@ int launch_tile(gemm_epi_plan_s* p, const TileCfg& c, const ge::TileParams& k_in
   int rc = prepare_out_map(p, k.out);
   if (rc) return rc;
   k.aux_tma = 0;
-  if (p->epilog == GEMM_EPI_GELU_AUX_BIAS && k.aux_out) {
-    // the pre-activation Z, T x N in the 16-bit type, stored like Y
-    if (k.aux_out != p->aux_ptr) {
-      rc = encode_2d(&p->tmAux, k.aux_out, (uint64_t)p->N, (uint64_t)p->T, 32, 32, "the GELU auxiliary output",
-                     CU_TENSOR_MAP_SWIZZLE_64B);
-      if (rc) return rc;
-      p->aux_ptr = k.aux_out;
-    }
-    k.aux_tma = 1;
+  if (p->epilog == GEMM_EPI_GELU_AUX_BIAS) {
+    // the pre-activation Z (T x N, 16-bit) is stored directly by the epilogue threads
   } else if (k.aux_out && aux_tma_ok(k.aux_out, p->N, c.BN)) {
     if (k.aux_out != p->aux_ptr) {
       rc = encode_aux(&p->tmAux, k.aux_out, p->T, p->N, c.BN);
@@ -760,7 +753,12 @@ gemm_epi_plan_t gemm_epi_plan_ex(int64_t T, int64_t N, int64_t K, gemm_epi_dtype
     // opt-in only. GEMM_EPI_PAIR_SPLIT=0|1 overrides.
     const int tail = pair_tiles % max_pairs;
     const int last_round = tail == 0 ? max_pairs : 2 * tail <= max_pairs ? 2 * tail : tail;
-    bool split = pair_tiles >= max_pairs && p->k_blocks >= 16 && 4 * last_round < 3 * max_pairs;
+    // Not for the GELU epilogs, whose epilogue (erff per element) is slower
+    // than a tile's MMAs: the pairs' epilogues lag behind their MMAs, the
+    // segments handed on arrive late, and the finishing segments wait (FFN
+    // GELU_BIAS forward 371 against 291 us, square 192 against 139).
+    const bool gelu = epilog == GEMM_EPI_GELU_BIAS || epilog == GEMM_EPI_GELU_AUX_BIAS;
+    bool split = !gelu && pair_tiles >= max_pairs && p->k_blocks >= 16 && 4 * last_round < 3 * max_pairs;
     if (const char* f = getenv("GEMM_EPI_PAIR_SPLIT")) split = atoi(f) != 0 && p->k_blocks >= 16;
     if (split && pair_tiles < max_pairs) {
       const int64_t want = (int64_t)pair_tiles * p->k_blocks / 8;  // at least 8 k-blocks per pair

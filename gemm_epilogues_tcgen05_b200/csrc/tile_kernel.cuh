@@ -315,6 +315,33 @@ __device__ __forceinline__ void store_block16(const float (&v)[32], const CUtens
   ++scount;
 }
 
+// This thread's 32 consecutive values of row `row` from column nc0, rounded
+// to the 16-bit type, into the T x N auxiliary output (GELU_AUX_BIAS):
+// four 16-byte stores when the whole segment is inside the tensor (and
+// 16-byte aligned, as it is when N is a multiple of 8), else element by
+// element up to N.
+template <bool BF16>
+__device__ __forceinline__ void store_row16(const float (&v)[32], const TileParams& p, int row, int nc0) {
+  if (row >= p.T) return;
+  uint16_t* base = reinterpret_cast<uint16_t*>(p.aux_out) + static_cast<int64_t>(row) * p.N + nc0;
+  if (nc0 + 32 <= p.N) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint4 w;
+      w.x = pack2<BF16>(v[8 * q + 0], v[8 * q + 1]);
+      w.y = pack2<BF16>(v[8 * q + 2], v[8 * q + 3]);
+      w.z = pack2<BF16>(v[8 * q + 4], v[8 * q + 5]);
+      w.w = pack2<BF16>(v[8 * q + 6], v[8 * q + 7]);
+      reinterpret_cast<uint4*>(base)[q] = w;
+    }
+  } else {
+    for (int j = 0; j < 32 && nc0 + j < p.N; ++j) {
+      const uint32_t h = pack2<BF16>(v[j], 0.f);
+      base[j] = static_cast<uint16_t>(h & 0xffffu);
+    }
+  }
+}
+
 template <int BN, int EPI, bool BF16>
 __device__ __forceinline__ void epi_rows(const TileParams& p, uint32_t tbase, int row, int n0, const float* bs,
                                          float* cpw, const CUtensorMap* tmY, uint8_t* stg, uint32_t& scount,
@@ -369,8 +396,11 @@ __device__ __forceinline__ void epi_rows(const TileParams& p, uint32_t tbase, in
     } else if constexpr (!PlainStore<EPI>::value) {
 #pragma unroll
       for (int j = 0; j < 32; ++j) v[j] += bs[c * 32 + j];
-      // GELU_AUX_BIAS: the pre-activation Z goes out (16-bit) before GELU
-      if constexpr (EPI == EPI_GELU_AUX_BIAS) store_block16<BF16>(v, tmAux, stg, scount, nc0, wrow0);
+      // GELU_AUX_BIAS: the pre-activation Z goes out (16-bit) before GELU, this
+      // thread's 32 columns as one 64-byte row segment written directly (the
+      // staging buffers and TMA stores are Y's; sharing them doubles the
+      // epilogue's store waits)
+      if constexpr (EPI == EPI_GELU_AUX_BIAS) store_row16<BF16>(v, p, row, nc0);
       if constexpr (AppliesGelu<EPI>::value) {
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = gelu_erf(v[j]);
