@@ -25,17 +25,19 @@
 // the pairs, each of them is processed as two 128-column halves (MMA N =
 // 128), so the last round takes half a tile's time instead of a whole one.
 //
-// Stream-K (SPLIT): with fewer tiles than pairs (the few-row problems, e.g.
-// 256 rows x 43 column tiles for 74 pairs), the (tile, k-block) space is cut
-// into one contiguous k-range per pair, so every pair streams the same share
-// of W. A tile covered by several pairs has one segment per pair; segment 0
-// (the one that starts at k-block 0) finishes the tile. The others write
-// their fp32 accumulator (each CTA its 128 rows) to a workspace slot and
-// count themselves on the tile's flag; segment 0 waits (bounded) until all
-// are in, adds them to its own in segment order (so the sum is the same on
-// every run) and runs the epilogue. Only segment 0 waits, and it waits only
-// on segments that never wait, and every pair is resident (one CTA per SM),
-// so the waits always end.
+// Stream-K (SPLIT): the tiles that would leave the last round of whole
+// tiles partly idle (between one and two waves of them; all tiles when there
+// are fewer tiles than pairs) are cut into one contiguous k-range per pair,
+// so every pair does the same share of the MMAs. A tile covered by several
+// pairs has one segment per pair; segment 0 (the one that starts at k-block
+// 0) finishes the tile. The others write their fp32 accumulator (each CTA
+// its 128 rows) to a workspace slot and count themselves on the tile's flag;
+// segment 0 waits (bounded) until all are in, adds them to its own in
+// segment order (so the sum is the same on every run) and runs the epilogue.
+// Only segment 0 waits, and it waits only on segments that never wait, and
+// every pair is resident (one CTA per SM), so the waits always end. By
+// default the stream-K tiles come before the whole tiles, so that the fixups
+// overlap later MMAs instead of ending the kernel.
 #pragma once
 
 #include "tile_kernel.cuh"
@@ -99,11 +101,11 @@ struct PairSchedule {
   }
 };
 
-// Stream-K part of a split schedule: with at least two waves of tiles, the
-// first rounds - 1 waves stay whole tiles, one per pair as without the
-// split, and only the rest (between one and two waves of tiles) is cut into
-// equal k-ranges, so every range spans at least one tile's k-blocks and a
-// tile has at most two segments; with fewer tiles every tile is cut.
+// Stream-K part of a split schedule: with at least two waves of tiles,
+// rounds - 1 waves stay whole tiles, one per pair as without the split, and
+// only the rest (between one and two waves of tiles) is cut into equal
+// k-ranges, so every range spans at least one tile's k-blocks and a tile has
+// at most two segments; with fewer tiles every tile is cut.
 __device__ __host__ __forceinline__ int pair_dp_rounds(int tiles, int npairs) {
   const int rounds = tiles / npairs;
   return rounds >= 2 ? rounds - 1 : 0;
@@ -111,14 +113,19 @@ __device__ __host__ __forceinline__ int pair_dp_rounds(int tiles, int npairs) {
 
 // The sequence of units of one pair. Without SPLIT: units pair, pair +
 // npairs, ... of the schedule, each over every k-block. With SPLIT: the
-// pair's whole tiles of the data-parallel rounds, then the pieces of its
-// contiguous range [lo, hi) of the flattened (tile, k-block) space of the
-// remaining tiles, tile by tile.
+// pieces of the pair's contiguous range [lo, hi) of the flattened (tile,
+// k-block) space of the stream-K tiles, tile by tile, and the pair's whole
+// tiles of the data-parallel rounds. With sk_first the stream-K pieces come
+// first (they are the first sk_tiles tiles of the raster order): a tile's
+// fixup then runs in an epilogue that the next whole tile's MMAs overlap,
+// and every pair ends on a whole tile. Otherwise the whole tiles come first
+// and the stream-K tiles are the last ones.
 template <bool SPLIT>
 struct PairWork {
   PairSchedule sched;
   int pair, npairs, m2_tiles, n_tiles, group, by_n, k_blocks;
-  int dp_units, dp_tiles;  // SPLIT: whole tiles of the data-parallel rounds (this pair's, and in all)
+  int dp_units, dp_tiles, sk_tiles, dp_done;  // SPLIT: the data-parallel rounds' whole tiles
+  bool sk_first;
   int64_t total, lo, hi, cur;
   __device__ __forceinline__ PairWork(const TileParams& p, int pair_, int npairs_, int m2)
       : sched(m2 * p.n_tiles, npairs_, !SPLIT && p.tail_split != 0),
@@ -126,24 +133,29 @@ struct PairWork {
         k_blocks(p.k_blocks) {
     if constexpr (SPLIT) {
       const int tiles = m2 * p.n_tiles;
-      const int rounds = pair_dp_rounds(tiles, npairs);
-      dp_tiles = rounds * npairs;
-      dp_units = rounds;
-      total = static_cast<int64_t>(tiles - dp_tiles) * p.k_blocks;
+      dp_units = pair_dp_rounds(tiles, npairs);
+      dp_tiles = dp_units * npairs;
+      sk_tiles = tiles - dp_tiles;
+      dp_done = 0;
+      sk_first = p.sk_first != 0;
+      total = static_cast<int64_t>(sk_tiles) * p.k_blocks;
       lo = static_cast<int64_t>(pair) * total / npairs;
       hi = static_cast<int64_t>(pair + 1) * total / npairs;
-      cur = -dp_units;  // negative: data-parallel rounds still to go
+      cur = 0;
     } else {
       cur = pair;
       hi = sched.num_units;
     }
   }
   // this is the pair's last unit (after next() returned it)
-  __device__ __forceinline__ bool done() const { return SPLIT ? (cur >= 0 && lo + cur >= hi) : cur >= hi; }
+  __device__ __forceinline__ bool done() const {
+    return SPLIT ? (lo + cur >= hi && dp_done >= dp_units) : cur >= hi;
+  }
   __device__ __forceinline__ bool next(PairUnit& w) {
     if constexpr (SPLIT) {
-      if (cur < 0) {  // a whole tile of the data-parallel rounds
-        const int t = pair + (dp_units + static_cast<int>(cur)) * npairs;
+      const bool sk_left = lo + cur < hi;
+      if (dp_done < dp_units && !(sk_first && sk_left)) {  // a whole tile of the data-parallel rounds
+        const int t = (sk_first ? sk_tiles : 0) + pair + dp_done * npairs;
         tile_coords(t, m2_tiles, n_tiles, group, by_n, w.mb, w.nb);
         w.half = -1;
         w.kb0 = 0;
@@ -151,15 +163,15 @@ struct PairWork {
         w.tile = t;
         w.seg = 0;
         w.nsegs = 1;
-        ++cur;
+        ++dp_done;
         return true;
       }
+      if (!sk_left) return false;
       const int64_t g = lo + cur;  // stream-K index
-      if (g >= hi) return false;
       const int tl = static_cast<int>(g / k_blocks);  // tile among the stream-K tiles
       const int64_t tb = static_cast<int64_t>(tl) * k_blocks;
       const int64_t end = hi < tb + k_blocks ? hi : tb + k_blocks;
-      const int t = dp_tiles + tl;
+      const int t = (sk_first ? 0 : dp_tiles) + tl;
       tile_coords(t, m2_tiles, n_tiles, group, by_n, w.mb, w.nb);
       w.half = -1;
       w.kb0 = static_cast<int>(g - tb);
@@ -369,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t trow = tmem_base + ((ew * 32u) << 16) + buf * BN;
       const int r = static_cast<int>(ew * 32 + lane);  // this thread's row of the CTA's 128
       // stream-K slots, one per pair and CTA: a pair's only later segment is
-      // its first unit, so segment s of the tile that pair `pair` finishes
+      // its first stream-K piece, so segment s of the tile that pair `pair` finishes
       // is in pair (pair + s)'s slot; the flag of a tile is its finisher's
       const int64_t slot_stride = 2 * kBM * BN;
       float* own_slot = SPLIT ? p.sk_slots + (static_cast<int64_t>(pair) * 2 + rank) * (kBM * BN) : nullptr;
@@ -426,9 +438,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (SPLIT && w.nsegs > 1) {
         // segment 0: wait until the other segments' partials are in (bounded)
         int* flag = p.sk_flags + pair * 2 + rank;
-        // the pair's last unit with one other segment: its operand stages are
-        // idle (the MMAs that read them are complete), so that segment's
-        // 128 KB comes in with bulk copies and is added from shared memory
+        // the pair's last unit with one other segment (stream-K tiles last,
+        // or no whole tiles): its operand stages are idle (the MMAs that read
+        // them are complete), so that segment's 128 KB comes in with bulk
+        // copies and is added from shared memory; otherwise the epilogue
+        // reads it from global memory while the next tile's MMAs run
         const bool bulk = w.nsegs == 2 && work.done();
         if (et == 0) {
           int got = ok ? 1 : 0;

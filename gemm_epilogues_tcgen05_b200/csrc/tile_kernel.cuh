@@ -117,6 +117,7 @@ struct TileParams {
   float* sk_slots;          // [pairs][2 ranks][128 rows][256 cols]: a pair's later segment
   int* sk_flags;            // [pairs][2 ranks]: segments in for the tile the pair finishes; zero between launches
   int32_t sk_max_segs;
+  int32_t sk_first;         // stream-K tiles before the whole tiles (else after them)
 };
 
 constexpr int kBM = 128;

@@ -181,14 +181,18 @@ def test_pair_stream_k(monkeypatch, T, N, K, dtype):
 
 
 # stream-K over at least one wave of tiles: every k-range spans a tile or
-# more, so a tile has at most two segments and the finishing segment brings
-# the other's partial in with bulk copies; the second shape keeps one
-# data-parallel round of whole tiles before the stream-K tiles
+# more, so a tile has at most two segments; the second shape keeps one
+# data-parallel round of whole tiles, after the stream-K tiles (their
+# finishing segments read the other's partial from global memory while the
+# next tile's MMAs run) or before them (the pair's last unit brings it in
+# with bulk copies)
+@pytest.mark.parametrize("sk_first", ["1", "0"])
 @pytest.mark.parametrize("dtype", ["fp16", "bf16"])
 @pytest.mark.parametrize("T,N,K", [(1024, 4864, 1024), (1100, 9728, 1024)])
-def test_pair_stream_k_waves(monkeypatch, T, N, K, dtype):
+def test_pair_stream_k_waves(monkeypatch, T, N, K, dtype, sk_first):
     _force(monkeypatch, "pair")
     monkeypatch.setenv("GEMM_EPI_PAIR_SPLIT", "1")
+    monkeypatch.setenv("GEMM_EPI_PAIR_SK_FIRST", sk_first)
     inp = synth.make_shape_inputs(T, N, K, dtype, seed=T + N + 3 * K, D2=K)
     for ep in ("RELU_AUX_BIAS", "GELU_AUX_BIAS"):
         gpu = run_forward(inp, ep, DT[dtype])
