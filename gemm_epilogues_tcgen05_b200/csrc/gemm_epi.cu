@@ -743,24 +743,18 @@ gemm_epi_plan_t gemm_epi_plan_ex(int64_t T, int64_t N, int64_t K, gemm_epi_dtype
     const int pair_tiles = ceil_div(T, 256) * p->n_tiles;
     const int max_pairs = max_resident_pairs(p->cfg, sms);
     int pairs = pair_tiles < max_pairs ? pair_tiles : max_pairs;
-    // Stream-K when the whole-tile schedule's last round would keep fewer
-    // than three quarters of the pairs busy (its leftover tiles, split into
-    // column halves where they fit): then cutting the last waves into
-    // k-ranges evens the end out. Measured, alternating runs on one box: FFN
-    // (688 tiles, a last round of 44 half tiles for 74 pairs) forward 244.0
-    // against 256.8 us, backward 252.9 against 257.4; T = 1024, N = 5120
-    // (80 tiles) forward 53.2 against 55.3; square 4096^3 (68 half tiles)
-    // forward equal, backward 111.5 against 108.8, so not there. With fewer
-    // tiles than pairs it loses (fixups through L2 for up to 8 segments):
-    // opt-in only. GEMM_EPI_PAIR_SPLIT=0|1 overrides.
-    const int tail = pair_tiles % max_pairs;
-    const int last_round = tail == 0 ? max_pairs : 2 * tail <= max_pairs ? 2 * tail : tail;
-    // Not for the GELU epilogs, whose epilogue (erff per element) is slower
-    // than a tile's MMAs: the pairs' epilogues lag behind their MMAs, the
-    // segments handed on arrive late, and the finishing segments wait (FFN
-    // GELU_BIAS forward 371 against 291 us, square 192 against 139).
-    const bool gelu = epilog == GEMM_EPI_GELU_BIAS || epilog == GEMM_EPI_GELU_AUX_BIAS;
-    bool split = !gelu && pair_tiles >= max_pairs && p->k_blocks >= 16 && 4 * last_round < 3 * max_pairs;
+    // Stream-K (the last waves cut into k-ranges) is opt-in,
+    // GEMM_EPI_PAIR_SPLIT=1. It evened out the end of the FFN forward while
+    // the MMA stream ran at 83 % of the tensor peak (244.0 against 256.8 us),
+    // but since the waits suspend instead of spinning and a tile runs at the
+    // peak rate, whole tiles are as fast or faster everywhere measured
+    // (interleaved runs on one box, forward / backward, us, whole against
+    // stream-K): FFN 252.9 / 257.0 against 252.9 / 255.0; T = 1024, N = 5120
+    // 51.2 / 56.3 against 53.3 / 60.4; T = 1000, N = 5000, K = 1024
+    // 23.6 / 29.7 against 34.8 / 42.0; square 97.3 / 104.7 against
+    // 98.3 / 109.6; T = 2048, N = 8192 94.2 / 99.3 against 97.3 / 103.5.
+    // The GELU epilogs slow down most with it (FFN GELU_BIAS 443 against 316).
+    bool split = false;
     if (const char* f = getenv("GEMM_EPI_PAIR_SPLIT")) split = atoi(f) != 0 && p->k_blocks >= 16;
     if (split && pair_tiles < max_pairs) {
       const int64_t want = (int64_t)pair_tiles * p->k_blocks / 8;  // at least 8 k-blocks per pair

@@ -178,18 +178,18 @@ static __device__ __noinline__ void report_timeout(int* status, volatile int* ab
 
 // Wait for the phase of parity `parity` on `bar`. Returns false if the CTA
 // is aborting or the wait exceeded the time limit (then it raises the abort).
+// Each test suspends the thread for up to ~20 us (mbar_try_wait), so the
+// abort flag and the clock are checked after every test.
 __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, const TileParams& p,
                                              volatile int* abort_flag, int site, bool honour_abort = true) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  for (uint32_t n = 1;; ++n) {
+  for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((n & 63u) == 0) {
-      if (honour_abort && *abort_flag) return false;
-      if (globaltimer_ns() - t0 > p.timeout_ns) {
-        report_timeout(p.status, abort_flag, site);
-        return false;
-      }
+    if (honour_abort && *abort_flag) return false;
+    if (globaltimer_ns() - t0 > p.timeout_ns) {
+      report_timeout(p.status, abort_flag, site);
+      return false;
     }
   }
 }

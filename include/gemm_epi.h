@@ -45,10 +45,9 @@
  *   GEMM_EPI_FORCE_KERNEL=tile|pair|skinny, GEMM_EPI_FORCE_BN=64|128|192|256,
  *   GEMM_EPI_RASTER=m|n, GEMM_EPI_GROUP_M, GEMM_EPI_SKINNY_GRID, GEMM_EPI_SKINNY_KPS=1|2,
  *   GEMM_EPI_SKINNY_PREFETCH, GEMM_EPI_TAIL_SPLIT=0|1, GEMM_EPI_CACHE_HINTS=0|1,
- *   GEMM_EPI_PAIR_SPLIT=0|1 (stream-K CTA pairs; by default on when the last round of
- *   whole tiles would leave a quarter of the pairs idle, not for the GELU epilogs),
- *   GEMM_EPI_PAIR_SK_FIRST=0|1 (the stream-K tiles before the whole tiles, the default,
- *   or after them)
+ *   GEMM_EPI_PAIR_SPLIT=0|1 (stream-K CTA pairs; off by default),
+ *   GEMM_EPI_PAIR_SK_FIRST=0|1 (with stream-K: its tiles before the whole tiles, the
+ *   default, or after them)
  *   fault injection for the library's own tests, honoured only while
  *   GEMM_EPI_TEST_HOOKS=1 is also set: GEMM_EPI_INJECT_STALL (a kernel
  *   withholds its first tile's completion signal, so its watchdog fires),
