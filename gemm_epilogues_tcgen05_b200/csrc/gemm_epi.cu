@@ -182,6 +182,7 @@ struct TileCfg {
   TileKernelFn fn = nullptr;
   uint32_t smem = 0;
   bool pair = false;  // CTA-pair kernel, launched in clusters of 2
+  int threads = ge::kThreads;
 };
 
 // bk: the weight is given N x K (GEMM_EPI_FLAG_W_NK); never with WGRAD
@@ -190,6 +191,12 @@ TileCfg pair_cfg(int epi, bool bf16, bool bk, bool split = false) {
   c.BN = 256;
   c.stages = 6;
   c.smem = ge::Tile2Smem<256, 6>::BYTES;
+  if (!split && (epi == ge::EPI_GELU_BIAS || epi == ge::EPI_GELU_AUX_BIAS)) {
+    // eight epilogue warps (ge::PairEpiWarps), five stages
+    c.stages = 5;
+    c.smem = ge::Tile2Smem<256, 5, 8>::BYTES;
+    c.threads = 64 + 32 * 8;
+  }
   if (split)
     c.fn = bf16 ? ge_inst::pair_split_bf16(epi, bk) : ge_inst::pair_split_f16(epi, bk);
   else
@@ -207,7 +214,7 @@ int max_resident_pairs(const TileCfg& c, int sms) {
   }
   cudaLaunchConfig_t lc = {};
   lc.gridDim = dim3((unsigned)(sms / 2 * 2), 1, 1);
-  lc.blockDim = dim3(ge::kThreads, 1, 1);
+  lc.blockDim = dim3((unsigned)c.threads, 1, 1);
   lc.dynamicSmemBytes = c.smem;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -522,7 +529,7 @@ int launch_tile(gemm_epi_plan_s* p, const TileCfg& c, const ge::TileParams& k_in
   if (c.pair) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)p->grid, 1, 1);
-    cfg.blockDim = dim3(ge::kThreads, 1, 1);
+    cfg.blockDim = dim3((unsigned)c.threads, 1, 1);
     cfg.dynamicSmemBytes = c.smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];

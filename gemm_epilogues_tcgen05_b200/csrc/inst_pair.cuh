@@ -14,8 +14,9 @@ TileKernelFn pair_epi(int epi) {
     case ge::EPI_RELU_BIAS: return ge::tile2_kernel<256, 6, ge::EPI_RELU_BIAS, BF, BK, SPLIT>;
     case ge::EPI_RELU_AUX_BIAS: return ge::tile2_kernel<256, 6, ge::EPI_RELU_AUX_BIAS, BF, BK, SPLIT>;
     case ge::EPI_DRELU_BGRAD: return ge::tile2_kernel<256, 6, ge::EPI_DRELU_BGRAD, BF, BK, SPLIT>;
-    case ge::EPI_GELU_BIAS: return ge::tile2_kernel<256, 6, ge::EPI_GELU_BIAS, BF, BK, SPLIT>;
-    case ge::EPI_GELU_AUX_BIAS: return ge::tile2_kernel<256, 6, ge::EPI_GELU_AUX_BIAS, BF, BK, SPLIT>;
+    // eight epilogue warps (whole tiles): their staging leaves room for 5 stages
+    case ge::EPI_GELU_BIAS: return ge::tile2_kernel<256, SPLIT ? 6 : 5, ge::EPI_GELU_BIAS, BF, BK, SPLIT>;
+    case ge::EPI_GELU_AUX_BIAS: return ge::tile2_kernel<256, SPLIT ? 6 : 5, ge::EPI_GELU_AUX_BIAS, BF, BK, SPLIT>;
     case ge::EPI_WGRAD:
       if constexpr (BK)
         return nullptr;

@@ -17,7 +17,7 @@
 //   empty[s]  (each CTA's) one arrival from the leader's MMA commit,
 //             multicast to both CTAs
 //   tfull[b]  (each CTA's) the leader's commit after a tile, multicast
-//   tempty[b] (leader's) eight arrivals: four epilogue warps of each CTA,
+//   tempty[b] (leader's) one arrival per epilogue warp of each CTA (4 or 8),
 //             the peer's through its shared::cluster address
 // No load uses TMA multicast. Every wait is bounded as in the 1-CTA kernel.
 //
@@ -44,7 +44,20 @@
 
 namespace ge {
 
-template <int BN, int STAGES>
+// Epilogue warps of the pair kernel: one per TMEM lane quarter, or two for
+// the GELU epilogs (each with half of a tile's columns). A warp reaches only
+// its own quarter of the TMEM lanes, so the four quarters sit on the four
+// SM sub-partitions, one warp each; with one warp per sub-partition a GELU
+// epilogue (erff per element, a chain of dependent operations) ran about
+// five times longer than a ReLU one and bounded the launch, and a second
+// warp per sub-partition overlaps two such chains. Stream-K instances keep
+// four (their partial slots are laid out per quarter).
+template <int EPI, bool SPLIT>
+struct PairEpiWarps {
+  static constexpr int value = AppliesGelu<EPI>::value && !SPLIT ? 8 : 4;
+};
+
+template <int BN, int STAGES, int EW = 4>
 struct Tile2Smem {
   static constexpr uint32_t A_BYTES = kBM * kBK * 2;          // this CTA's 128 rows x 64 k
   static constexpr uint32_t B_CHUNK = kBK * 64 * 2;           // 64 k x 64 n
@@ -57,8 +70,8 @@ struct Tile2Smem {
   static constexpr uint32_t OFF_BIAS = (OFF_MISC + 16 + 15) / 16 * 16;
   static constexpr uint32_t OFF_COLP = OFF_BIAS + 2 * BN * 4;
   static constexpr uint32_t OFF_STG = (OFF_COLP + 2 * 4 * BN * 4 + 1023) / 1024 * 1024;
-  static constexpr uint32_t OFF_AUXSTG = OFF_STG + kStageBytesPerWarp * 4;
-  static constexpr uint32_t END = OFF_AUXSTG + kAuxStageBytesPerWarp * 4;
+  static constexpr uint32_t OFF_AUXSTG = OFF_STG + kStageBytesPerWarp * EW;
+  static constexpr uint32_t END = OFF_AUXSTG + kAuxStageBytesPerWarp * EW;
   static constexpr uint32_t BYTES = END + 1024;
 };
 
@@ -194,11 +207,13 @@ struct PairWork {
 };
 
 template <int BN, int STAGES, int EPI, bool BF16, bool BK = false, bool SPLIT = false>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(64 + 32 * PairEpiWarps<EPI, SPLIT>::value, 1)
     tile2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmAux,
                  const TileParams p) {
-  using L = Tile2Smem<BN, STAGES>;
+  constexpr int EW = PairEpiWarps<EPI, SPLIT>::value;  // epilogue warps
+  constexpr int ET = 32 * EW;                          // epilogue threads
+  using L = Tile2Smem<BN, STAGES, EW>;
   static_assert(BN == 128 || BN == 256, "the pair kernel splits BN in 64-column chunks per CTA");
   constexpr uint32_t TMEM_COLS = 2 * BN;
   static_assert(BN == 256, "the tail split halves 256-column tiles");
@@ -224,8 +239,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
   float* bias_s = reinterpret_cast<float*>(smem + L::OFF_BIAS);  // [2][BN]
   float* colp_s = reinterpret_cast<float*>(smem + L::OFF_COLP);  // [2][4][BN]
-  uint8_t* stg_s = smem + L::OFF_STG;                             // [4 warps][2][2 KB]
-  uint8_t* auxstg_s = smem + L::OFF_AUXSTG;                       // [4 warps][1 KB]
+  uint8_t* stg_s = smem + L::OFF_STG;                             // [EW warps][2][2 KB]
+  uint8_t* auxstg_s = smem + L::OFF_AUXSTG;                       // [EW warps][1 KB]
   volatile int* dflag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 8);
   volatile int* sflag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 12);  // stream-K wait result
 
@@ -242,7 +257,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 8);
+      mbar_init(&tempty[b], 2 * EW);
     }
     mbar_init(drain, 1);
     mbar_init(fixbar, 1);
@@ -354,9 +369,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
-    const uint32_t ew = warp & 3u;
-    const uint32_t et = threadIdx.x - 64;
-    uint8_t* stg = stg_s + ew * kStageBytesPerWarp;
+    const uint32_t ew = warp & 3u;             // TMEM lane quarter
+    const uint32_t eh = (warp - 2u) >> 2;      // column half (EW == 8), else 0
+    const uint32_t et = threadIdx.x - 64;      // 0 .. ET - 1
+    uint8_t* stg = stg_s + (warp - 2u) * kStageBytesPerWarp;
     uint32_t scount = 0;
     uint32_t tcount = 0;
     bool ok = true;
@@ -372,10 +388,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t tph = (tcount >> 1) & 1u;
       float* bs = bias_s + buf * BN;
       float* cp = colp_s + buf * 4 * BN;
-      epi_stage_bias<BN, EPI, BF16>(p, n0, bs, et, ncols);
+      epi_stage_bias<BN, EPI, BF16, ET>(p, n0, bs, et, ncols);
       MaskWords<BN> mw{};
       if constexpr (EPI == EPI_DRELU_BGRAD) mw = load_mask_words<BN>(p, m0 + static_cast<int>(ew * 32 + lane), n0);
-      named_bar_sync(1, 128);
+      named_bar_sync(1, ET);
       if (ok) ok = wait_bounded(&tfull[buf], tph, p, abort_flag, 6);
       ok = __all_sync(0xffffffffu, ok);
       const uint32_t trow = tmem_base + ((ew * 32u) << 16) + buf * BN;
@@ -428,7 +444,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
         }
         __threadfence();
-        named_bar_sync(1, 128);
+        named_bar_sync(1, ET);
         if (et == 0 && ok) atomicAdd(p.sk_flags + (pair - w.seg) * 2 + rank, 1);
         continue;
       }
@@ -469,7 +485,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           *sflag = got;
         }
-        named_bar_sync(1, 128);
+        named_bar_sync(1, ET);
         ok = ok && *sflag != 0;
         if (ok && bulk) ok = wait_bounded(fixbar, 0, p, abort_flag, 8);
         ok = __all_sync(0xffffffffu, ok);
@@ -479,15 +495,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (ok) {
         tc_fence_after();
-        epi_rows<BN, EPI, BF16>(p, trow, m0 + r, n0, bs, cp + ew * BN, &tmY, stg, scount, m0 + static_cast<int>(ew * 32),
-                                &tmAux, auxstg_s + ew * kAuxStageBytesPerWarp, mw, ncols, w.half < 0, addp, nadd,
-                                slot_stride, add_smem);
+        if constexpr (EW == 8) {
+          // this warp's half of the columns (the GELU epilogs: no mask words,
+          // no column sums, no stream-K addends)
+          const int hc = ncols / 2, c0 = static_cast<int>(eh) * hc;
+          epi_rows<BN, EPI, BF16>(p, trow + c0, m0 + r, n0 + c0, bs + c0, nullptr, &tmY, stg, scount,
+                                  m0 + static_cast<int>(ew * 32), &tmAux, nullptr, mw, hc, false);
+        } else {
+          epi_rows<BN, EPI, BF16>(p, trow, m0 + r, n0, bs, cp + ew * BN, &tmY, stg, scount,
+                                  m0 + static_cast<int>(ew * 32), &tmAux, auxstg_s + ew * kAuxStageBytesPerWarp, mw,
+                                  ncols, w.half < 0, addp, nadd, slot_stride, add_smem);
+        }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(tempty0 + buf * 8);
       }
       if constexpr (EPI == EPI_DRELU_BGRAD) {
-        named_bar_sync(1, 128);
+        named_bar_sync(1, ET);
         const bool has_row = prow < p.m_tiles;
         if (ok && has_row) epi_write_partials<BN>(p, prow, n0, cp, et, ncols);
         // tickets count per 128-column half block, so whole tiles and tail halves mix

@@ -242,10 +242,10 @@ __device__ __forceinline__ void warp_transpose_reduce32(float (&v)[32]) {
 // epilogue thread owns one accumulator row (its TMEM lane) of a 128-row block.
 
 // Stage the tile's bias values (fp32) in shared memory.
-template <int BN, int EPI, bool BF16>
+template <int BN, int EPI, bool BF16, int NT = 128>
 __device__ __forceinline__ void epi_stage_bias(const TileParams& p, int n0, float* bs, uint32_t et, int ncols = BN) {
   if constexpr (AddsBias<EPI>::value) {
-    for (int c = et; c < ncols; c += 128) {
+    for (int c = et; c < ncols; c += NT) {
       const int n = n0 + c;
       bs[c] = n < p.N ? load_bias<BF16>(p.bias, p.bias_f32, n) : 0.f;
     }
