@@ -623,6 +623,29 @@ def test_watchdog_reports_timeout_and_context_stays_usable(monkeypatch, epilog, 
         check_backward(inp, gpu["aux"], dt, out)
 
 
+@pytest.mark.parametrize("epilog", ["GELU_BIAS", "GELU_AUX_BIAS"])
+def test_watchdog_with_eight_epilogue_warps(monkeypatch, epilog):
+    """The CTA-pair kernel's GELU instances (two epilogue warps per TMEM lane
+    quarter): the same injected stall, the same report, and correct results
+    afterwards."""
+    _force(monkeypatch, "pair")
+    monkeypatch.setenv("GEMM_EPI_WAIT_TIMEOUT_MS", "200")
+    monkeypatch.setenv("GEMM_EPI_INJECT_STALL", "1")
+    monkeypatch.setenv("GEMM_EPI_TEST_HOOKS", "1")
+    T, N, K = 600, 1032, 264
+    inp = synth.make_shape_inputs(T, N, K, "bf16", seed=19)
+    g = {k: v.cuda() for k, v in inp.items()}
+    with binding.Plan(T, N, K, torch.bfloat16, epilog) as plan:
+        assert plan.info()["kernel"] == 2
+        plan.forward(g["X"], g["W"], g["bias"])
+        torch.cuda.synchronize()
+        assert plan.status() == binding.ERR_TIMEOUT
+    monkeypatch.delenv("GEMM_EPI_INJECT_STALL")
+    gpu = run_forward(inp, epilog, torch.bfloat16)
+    assert gpu["info"]["kernel"] == 2
+    check_forward(inp, epilog, torch.bfloat16, gpu)
+
+
 def test_stall_hook_needs_the_test_switch(monkeypatch):
     """GEMM_EPI_INJECT_STALL alone (without GEMM_EPI_TEST_HOOKS=1) changes nothing."""
     _force(monkeypatch, "tile64")
