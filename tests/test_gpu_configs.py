@@ -13,8 +13,8 @@ import torch
 import oracle
 from gemm_epilogues_tcgen05_b200 import Plan, synth
 
-from _parity import (Y_REL, assert_dbias, assert_dbias_is_column_sum, assert_within, check_wgrad, odt, run_wgrad,
-                     unit_roundoff)
+from _parity import (Y_REL, assert_dbias, assert_dbias_is_column_sum, assert_within, check_forward, check_wgrad, odt,
+                     run_forward, run_wgrad, unit_roundoff)
 
 pytestmark = pytest.mark.gpu
 
@@ -143,6 +143,21 @@ def test_ffn_wgrad_sampled():
     cols = synth.sample_indices(w.N, SAMPLE, seed=w.seed + 14)
     check_wgrad(inp, w.torch_dtype, gpu, rows=rows, dz_key="dZ")
     check_wgrad(inp, w.torch_dtype, gpu, cols=cols, dz_key="dZ")
+
+
+@pytest.mark.parametrize("epilog", ["GELU_BIAS", "GELU_AUX_BIAS"])
+def test_ffn_gelu_sampled(epilog):
+    """The GELU epilogs on the FFN shape, in the launch configuration the bench
+    times (CTA pairs with eight epilogue warps), checked on 256 sampled rows
+    and 256 sampled columns of Y (and of Z for GELU_AUX_BIAS)."""
+    w = synth.WORKLOADS["ffn"]
+    inp = synth.make_inputs(w, parts=("fwd",))
+    gpu = run_forward(inp, epilog, w.torch_dtype)
+    assert gpu["info"]["kernel"] == 2
+    rows = synth.sample_indices(w.T, SAMPLE, seed=w.seed + 15)
+    cols = synth.sample_indices(w.N, SAMPLE, seed=w.seed + 16)
+    check_forward(inp, epilog, w.torch_dtype, gpu, rows=rows)
+    check_forward(inp, epilog, w.torch_dtype, gpu, cols=cols)
 
 
 @pytest.mark.slow
