@@ -127,9 +127,10 @@ __device__ __forceinline__ void store_out(const SkinnyParams& p, int64_t i, floa
 }
 
 // DRELU_BGRAD: the mask words of rows t0 .. t0+15 for this warp's 32
-// features (one word per row). Callers load them ahead of use -- before the
-// accumulator wait, or before the previous rows' stores -- so the loads are
-// in flight while other work proceeds.
+// features (one word per row), held by every lane. A whole tile's words are
+// all loaded before the accumulator wait and handed out 16 rows at a time by
+// shuffles; the split-tile fixup loads a batch's words before it reads the
+// partials, so the loads are in flight together.
 struct Mask16 {
   uint32_t m[16];
 };
@@ -412,9 +413,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         bias_n = n_ok ? load_bias<BF16>(p.bias, p.bias_f32, n) : 0.f;
       float dbias_acc = 0.f;
       const bool whole = s.kb0 == 0 && s.kb1 == p.kbt;
-      Mask16 mk{};
+      // DRELU_BGRAD, whole tile: every mask word the tile needs, loaded before
+      // the accumulator wait so that none of them is fetched while the
+      // epilogue runs (lane l holds the word of row 32·i + l in mrow[i])
+      constexpr int MR = (TP + 31) / 32;
+      uint32_t mrow[MR];
+#pragma unroll
+      for (int i = 0; i < MR; ++i) mrow[i] = 0u;
       if constexpr (EPI == EPI_DRELU_BGRAD)
-        if (whole) mk = skinny_mask16(p, 0, word);  // in flight during the accumulator wait
+        if (whole)
+#pragma unroll
+          for (int i = 0; i < MR; ++i) {
+            const int t = i * 32 + static_cast<int>(lane);
+            if (t < p.T && word < p.aux_words) mrow[i] = __ldg(p.aux_in + static_cast<int64_t>(t) * p.aux_words + word);
+          }
       if (ok) ok = wait_bounded(&tfull[buf], tph, wp, abort_flag, 6);
       ok = __all_sync(0xffffffffu, ok);
       const uint32_t tbase = tmem_base + ((ew * 32u) << 16) + buf * TP;
@@ -424,9 +436,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
         for (int c = 0; c < TP / 16; ++c) {
           if (c * 16 >= p.T) break;  // warp-uniform
-          Mask16 mk_next{};
+          Mask16 mk{};
           if constexpr (EPI == EPI_DRELU_BGRAD)
-            if (whole && (c + 1) * 16 < p.T) mk_next = skinny_mask16(p, (c + 1) * 16, word);
+            if (whole) {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) mk.m[j] = __shfl_sync(0xffffffffu, mrow[0], (c & 1) * 16 + j);
+              if (c & 1)
+#pragma unroll
+                for (int i = 0; i + 1 < MR; ++i) mrow[i] = mrow[i + 1];
+            }
           uint32_t r[16];
           tmem_ld_32x32b_x16(tbase + c * 16, r);
           tmem_wait_ld();
@@ -435,7 +453,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
           if (whole) {
             skinny_finish16<EPI, BF16>(p, v, c * 16, n, n_ok, word, bias_n, dbias_acc, mk);
-            mk = mk_next;
           } else {
 #pragma unroll
             for (int j = 0; j < 16; ++j)
