@@ -369,6 +369,13 @@ bool use_pair(int64_t T, int64_t N, int64_t K, int num_sms) {
 // The few-row kernel for T <= 128; from 129 rows on, one-CTA tiles of 192
 // columns beat it (T = 256, N = 11008, K = 4096: 34.7 / 36.9 us against
 // 47.1 / 51.2 us, and against the CTA pair's 36.6 / 40.9 us).
+// The few-row kernel's range arithmetic is 32-bit: (k-blocks + 1) x grid must
+// stay below 2^31 (k-blocks of 64 at most, grid at most one CTA per SM).
+bool skinny_fits(int64_t N, int64_t K, int sms) {
+  const int64_t kblocks = ((N + 127) / 128) * ((K + 63) / 64);
+  return (kblocks + 1) * (int64_t)sms < (int64_t(1) << 31);
+}
+
 bool use_skinny(int64_t T) {
   if (const char* f = getenv("GEMM_EPI_FORCE_KERNEL")) {
     if (!strcmp(f, "tile")) return false;
@@ -808,7 +815,7 @@ gemm_epi_plan_t gemm_epi_plan_ex(int64_t T, int64_t N, int64_t K, gemm_epi_dtype
   // 4096: T = 1 25.1 / 24.5 us against 27.3 / 26.8, T = 64 32.6 / 33.4 against
   // 33.2 / 34.3). The tile kernels load without hints: there they did not help
   // the FFN and square shapes and slowed the large one (17.6 against 16.8 ms).
-  if (!pair && epilog != GEMM_EPI_WGRAD && !w_nk && use_skinny(T)) {
+  if (!pair && epilog != GEMM_EPI_WGRAD && !w_nk && use_skinny(T) && skinny_fits(N, K, sms)) {
     p->kernel = 1;
     p->cache_hints = 1;
     p->sk = skinny_cfg(T, (int)epilog, bf16);
@@ -830,7 +837,7 @@ gemm_epi_plan_t gemm_epi_plan_ex(int64_t T, int64_t N, int64_t K, gemm_epi_dtype
     }
     if (const char* f = getenv("GEMM_EPI_SKINNY_GRID")) {  // tuning override
       const int v = atoi(f);
-      if (v >= 1 && v <= p->sk_total) p->sk_grid = v;
+      if (v >= 1 && v <= p->sk_total && (int64_t)(p->sk_total + 1) * v < (int64_t(1) << 31)) p->sk_grid = v;
     }
     if (const char* f = getenv("GEMM_EPI_SKINNY_PREFETCH")) p->sk_prefetch = atoi(f) > 0 ? atoi(f) : 0;
     p->sk_max_segs = 1;

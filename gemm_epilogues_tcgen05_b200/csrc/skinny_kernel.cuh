@@ -76,27 +76,35 @@ __device__ __host__ __forceinline__ int64_t skinny_owner(int64_t x, int64_t grid
   return ((x + 1) * grid - 1) / total;
 }
 
+// The same in 32-bit arithmetic, for the kernel: the plan keeps (k-blocks + 1)
+// x grid below 2^31. (64-bit divisions in the range and segment arithmetic
+// sit between the kernel's start and its first load.)
+__device__ __forceinline__ uint32_t skinny_owner32(uint32_t x, uint32_t grid, uint32_t total) {
+  return ((x + 1u) * grid - 1u) / total;
+}
+
 struct Segment {
   int tile, kb0, kb1;  // k-blocks [kb0, kb1) of the tile, local to it
   int seg, nsegs;      // index among the CTAs sharing the tile, and their count
 };
 
-// The idx-th segment of this CTA's range, or false when there are no more.
-__device__ __forceinline__ bool skinny_segment(const SkinnyParams& p, int64_t lo, int64_t hi, int64_t& g, Segment& s) {
+// The next segment of this CTA's k-block range [g, hi), or false when there
+// are no more.
+__device__ __forceinline__ bool skinny_segment(const SkinnyParams& p, uint32_t hi, uint32_t& g, Segment& s) {
   if (g >= hi) return false;
-  const int tile = static_cast<int>(g / p.kbt);
-  const int64_t tbeg = static_cast<int64_t>(tile) * p.kbt;
-  const int64_t tend = tbeg + p.kbt;
-  const int64_t end = hi < tend ? hi : tend;
-  s.tile = tile;
+  const uint32_t kbt = static_cast<uint32_t>(p.kbt), total = static_cast<uint32_t>(p.total_kb);
+  const uint32_t tile = g / kbt;
+  const uint32_t tbeg = tile * kbt;
+  const uint32_t tend = tbeg + kbt;
+  const uint32_t end = hi < tend ? hi : tend;
+  s.tile = static_cast<int>(tile);
   s.kb0 = static_cast<int>(g - tbeg);
   s.kb1 = static_cast<int>(end - tbeg);
-  const int64_t first = skinny_owner(tbeg, gridDim.x, p.total_kb);
-  const int64_t last = skinny_owner(tend - 1, gridDim.x, p.total_kb);
-  s.nsegs = static_cast<int>(last - first + 1);
+  const uint32_t first = skinny_owner32(tbeg, gridDim.x, total);
+  const uint32_t last = skinny_owner32(tend - 1u, gridDim.x, total);
+  s.nsegs = static_cast<int>(last - first + 1u);
   s.seg = static_cast<int>(blockIdx.x - first);
   g = end;
-  (void)lo;
   return true;
 }
 
@@ -288,8 +296,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const uint32_t warp = threadIdx.x >> 5;
   const uint32_t lane = lane_id();
-  const int64_t lo = static_cast<int64_t>(blockIdx.x) * p.total_kb / gridDim.x;
-  const int64_t hi = static_cast<int64_t>(blockIdx.x + 1) * p.total_kb / gridDim.x;
+  const uint32_t lo = blockIdx.x * static_cast<uint32_t>(p.total_kb) / gridDim.x;
+  const uint32_t hi = (blockIdx.x + 1u) * static_cast<uint32_t>(p.total_kb) / gridDim.x;
 
   // the tile kernel's bounded wait reads its timeout and status from TileParams
   TileParams wp{};
@@ -328,25 +336,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t it = 0;
       bool ok = true;
-      int64_t g = lo;
+      uint32_t g = lo;
       Segment s;
       // W tiles may also be prefetched into L2 p.prefetch k-blocks ahead of
       // the shared-memory ring, so that the ring's loads hit L2.
-      int64_t pf = lo;
-      const auto prefetch_upto = [&](int64_t upto) {
+      uint32_t pf = lo;
+      const auto prefetch_upto = [&](uint32_t upto) {
         for (; pf < upto && pf < hi; ++pf) {
-          const int t = static_cast<int>(pf / p.kbt);
-          const int kb = static_cast<int>(pf - static_cast<int64_t>(t) * p.kbt);
+          const int t = static_cast<int>(pf / static_cast<uint32_t>(p.kbt));
+          const int kb = static_cast<int>(pf - static_cast<uint32_t>(t) * static_cast<uint32_t>(p.kbt));
           tma_prefetch_l2_2d(&tmW, t * 128, kb * L::BK);
           tma_prefetch_l2_2d(&tmW, t * 128 + 64, kb * L::BK);
         }
       };
-      int64_t gk = lo;  // global k-block index of the next load
+      uint32_t gk = lo;  // global k-block index of the next load
       const uint64_t pol_w = l2_policy_evict_first(), pol_x = l2_policy_evict_last();
-      while (ok && skinny_segment(p, lo, hi, g, s)) {
+      while (ok && skinny_segment(p, hi, g, s)) {
         const int n0 = s.tile * 128;
         for (int kb = s.kb0; kb < s.kb1; ++kb, ++it, ++gk) {
-          if (p.prefetch > 0) prefetch_upto(gk + p.prefetch);
+          if (p.prefetch > 0) prefetch_upto(gk + static_cast<uint32_t>(p.prefetch));
           const uint32_t st = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
           if (!wait_bounded(&empty[st], ph ^ 1u, wp, abort_flag, 1)) {
@@ -379,9 +387,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t it = 0, scount = 0;
       bool ok = true;
-      int64_t g = lo;
+      uint32_t g = lo;
       Segment s;
-      while (ok && skinny_segment(p, lo, hi, g, s)) {
+      while (ok && skinny_segment(p, hi, g, s)) {
         const uint32_t buf = scount & 1u;
         const uint32_t tph = (scount >> 1) & 1u;
         ++scount;
@@ -425,9 +433,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t et = threadIdx.x - 64;
     uint32_t scount = 0;
     bool ok = true;
-    int64_t g = lo;
+    uint32_t g = lo;
     Segment s;
-    while (skinny_segment(p, lo, hi, g, s)) {
+    while (skinny_segment(p, hi, g, s)) {
       const uint32_t buf = scount & 1u;
       const uint32_t tph = (scount >> 1) & 1u;
       ++scount;
