@@ -517,12 +517,10 @@ __global__ void __launch_bounds__(64 + 32 * PairEpiWarps<EPI, SPLIT>::value, 1)
         // tickets count per 128-column half block, so whole tiles and tail halves mix
         if (p.col_tickets) {
           const int rows = (ok && has_row) ? 1 : 0;
-          if (w.half < 0) {
-            epi_finish_dbias<BN>(p, 2 * w.nb, n0, rows, et, dflag, BN / 2);
-            epi_finish_dbias<BN>(p, 2 * w.nb + 1, n0 + BN / 2, rows, et, dflag, BN / 2);
-          } else {
+          if (w.half < 0)
+            epi_finish_dbias<BN>(p, 2 * w.nb, n0, rows, et, dflag, BN / 2, 2);
+          else
             epi_finish_dbias<BN>(p, 2 * w.nb + w.half, n0, rows, et, dflag, BN / 2);
-          }
         }
       }
     }

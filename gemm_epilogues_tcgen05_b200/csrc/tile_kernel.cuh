@@ -484,44 +484,73 @@ __device__ __forceinline__ void epi_write_partials(const TileParams& p, int prow
   }
 }
 
+// Column sums of the partial rows 0 .. m_tiles-1 for up to two columns na, nb
+// (used where ua / ub), each in ascending row order, one row at a time -- the
+// same order whichever tile runs it. The loads of 16 rows of both columns are
+// issued together (32 L2 round trips in flight): issued one by one they were
+// most of the finishing time at few row blocks.
+__device__ __forceinline__ void sum_partials2(const TileParams& p, int na, bool ua, int nb, bool ub, float& sa,
+                                              float& sb) {
+  sa = 0.f;
+  sb = 0.f;
+  const float* ca = p.partials + na;
+  const float* cb = p.partials + nb;
+  for (int m0 = 0; m0 < p.m_tiles; m0 += 16) {
+    float xa[16], xb[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const bool v = m0 + j < p.m_tiles;
+      const int64_t off = static_cast<int64_t>(m0 + j) * p.N;
+      xa[j] = (ua && v) ? __ldcg(ca + off) : 0.f;
+      xb[j] = (ub && v) ? __ldcg(cb + off) : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      if (m0 + j < p.m_tiles) {
+        sa += xa[j];
+        sb += xb[j];
+      }
+    }
+  }
+}
+
 // DRELU_BGRAD, second pass inside the kernel: after its partial rows are
-// written, a tile takes `rows` tickets on its column block; the tile that
-// takes the block's last ticket sums every partial row of the block in
-// ascending row order -- the same order whichever tile is last -- writes
-// dbias and resets the counter for the next launch. Called by the 128
-// epilogue threads; `flag` is a shared-memory word.
+// written, a tile takes `rows` tickets on each of its `nblocks` column blocks
+// of `ncols` columns (nb, nb + 1, ...; a whole CTA-pair tile spans two); for
+// each block where it takes the last ticket it sums every partial row of the
+// block in ascending row order -- the same order whichever tile is last --
+// writes dbias and resets the counter for the next launch. Called by the 128
+// epilogue threads, each taking columns et and et + 128 of the tile;
+// `flag` is a shared-memory word.
 template <int BN>
 __device__ __forceinline__ void epi_finish_dbias(const TileParams& p, int nb, int n0, int rows, uint32_t et,
-                                                 volatile int* flag, int ncols = BN) {
+                                                 volatile int* flag, int ncols = BN, int nblocks = 1) {
   __threadfence();
   named_bar_sync(1, 128);
   if (et == 0) {
-    const int prev = atomicAdd(p.col_tickets + nb, rows);
-    const int last = prev + rows == p.m_tiles;
-    if (last) p.col_tickets[nb] = 0;
-    *flag = last;
+    int bits = 0;
+    for (int b = 0; b < nblocks; ++b) {
+      const int prev = atomicAdd(p.col_tickets + nb + b, rows);
+      if (prev + rows == p.m_tiles) {
+        p.col_tickets[nb + b] = 0;
+        bits |= 1 << b;
+      }
+    }
+    *flag = bits;
   }
   named_bar_sync(1, 128);
-  if (*flag) {
+  const int bits = *flag;
+  if (bits) {
     __threadfence();
-    for (int c = et; c < ncols; c += 128) {
-      const int n = n0 + c;
-      if (n < p.N) {
-        // ascending m as always; the loads of a batch of 16 rows are issued
-        // together (the L2 round trips would otherwise run one by one)
-        const float* col = p.partials + n;
-        float s = 0.f;
-        int m = 0;
-        for (; m + 16 <= p.m_tiles; m += 16) {
-          float x[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) x[j] = __ldcg(col + static_cast<int64_t>(m + j) * p.N);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) s += x[j];
-        }
-        for (; m < p.m_tiles; ++m) s += __ldcg(col + static_cast<int64_t>(m) * p.N);
-        p.dbias[n] = s;
-      }
+    const int total = nblocks * ncols;
+    const int ca = static_cast<int>(et), cb = static_cast<int>(et) + 128;
+    const bool ua = ca < total && ((bits >> (ca / ncols)) & 1) && n0 + ca < p.N;
+    const bool ub = cb < total && ((bits >> (cb / ncols)) & 1) && n0 + cb < p.N;
+    if (ua || ub) {
+      float sa, sb;
+      sum_partials2(p, n0 + ca, ua, n0 + cb, ub, sa, sb);
+      if (ua) p.dbias[n0 + ca] = sa;
+      if (ub) p.dbias[n0 + cb] = sb;
     }
   }
   named_bar_sync(1, 128);  // the flag word is reused by the next tile
