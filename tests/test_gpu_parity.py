@@ -103,6 +103,27 @@ def test_pair_kernel_ragged(monkeypatch, T, N, K, dtype):
         check_forward(inp, ep, DT[dtype], run_forward(inp, ep, DT[dtype], unfused=True), stored_xw=True)
 
 
+# The bias gradient's finishing pass over more than 16 row blocks with a
+# partial batch last (T = 2300: 18 blocks of 128 rows) and a ragged last
+# column tile (N = 776), for each layout of its tickets: 128 or 256 columns
+# per ticket on one-CTA tiles, two 128-column tickets per CTA-pair tile.
+@pytest.mark.parametrize("variant", ["tile128", "tile256", "pair"])
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+def test_dbias_finish_over_many_row_blocks(monkeypatch, dtype, variant):
+    _force(monkeypatch, variant)
+    T, N, K, D2 = 2300, 776, 64, 136
+    inp = synth.make_shape_inputs(T, N, K, dtype, seed=T + N, D2=D2)
+    fwd = run_forward(inp, "RELU_AUX_BIAS", DT[dtype])
+    outs = run_backward(inp, fwd["aux"], DT[dtype], repeats=2)  # tickets reset between launches
+    for gpu in outs:
+        _expect_variant(gpu["info"], variant, T)
+        check_backward(inp, fwd["aux"], DT[dtype], gpu)
+    assert torch.equal(outs[0]["dbias"], outs[1]["dbias"])
+    iinp = synth.make_shape_inputs(T, N, K, dtype, seed=T + N + 1, D2=D2, kind="int")
+    ifwd = run_forward(iinp, "RELU_AUX_BIAS", DT[dtype])
+    check_backward(iinp, ifwd["aux"], DT[dtype], run_backward(iinp, ifwd["aux"], DT[dtype]), exact=True)
+
+
 @pytest.mark.parametrize("dtype", ["fp16", "bf16"])
 @pytest.mark.parametrize("T,N,K", SKINNY_SHAPES)
 def test_skinny_split_tiles(monkeypatch, T, N, K, dtype):
