@@ -336,6 +336,18 @@ def test_dbias_bitwise_reproducible_across_runs_and_streams():
     assert torch.equal(other["dbias"], outs[0]["dbias"])
 
 
+def test_few_row_kernel_only_where_its_32_bit_ranges_fit(monkeypatch):
+    """The few-row kernel's range arithmetic is 32-bit, so the planner gives
+    it a few-row shape only while (64-deep k-blocks + 1) x SMs stays below
+    2^31; a legal shape beyond that (N = K = 2^20: 2^27 k-blocks) goes to the
+    tile kernel. Planning only: nothing of that size is allocated or run."""
+    monkeypatch.delenv("GEMM_EPI_FORCE_KERNEL", raising=False)
+    with binding.Plan(1, 11008, 4096, torch.bfloat16, "RELU_BIAS") as small:
+        assert small.info()["kernel"] == 1
+    with binding.Plan(1, 1 << 20, 1 << 20, torch.bfloat16, "RELU_BIAS") as huge:
+        assert huge.info()["kernel"] == 0
+
+
 def test_plan_reuse_many_executes():
     """One plan, several executes with different buffers (tensor maps re-encoded)."""
     T, N, K = 300, 264, 136
